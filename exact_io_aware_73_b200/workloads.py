@@ -1,0 +1,129 @@
+"""Seeded synthetic inputs for the attention forward pass.
+
+This module is the one thing the CUDA path and the fp64 oracle share: it
+makes Q, K and V and nothing else.  It holds none of the attention
+arithmetic.  Every tensor is sampled in fp32 on the CPU from a seeded
+``torch.Generator`` and rounded to bfloat16 (round-to-nearest-even), so the
+same bits go to the GPU and to the oracle.
+
+The named workloads are the shapes the method is measured on: a small
+single-head case, a GPT-2-small-shaped layer (12 heads of 64), a d=128
+causal case, one full trading day at one-second resolution (23,400 steps,
+12 heads; the score-matrix size quoted in the marketmaker.cc post "Apakah
+Konteks Sehari Penuh Mengalahkan Konteks Sepuluh Menit? ...", introduction)
+and a long non-causal d=128 case with wide score spread.  No dataset is
+involved: the post's BTC one-second series is replaced by these synthetic
+draws.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    q_std: float = 1.0
+    k_std: float = 1.0
+    v_dist: str = "normal"  # "normal" (std 1) or "uniform" (U(-1, 1))
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """Metric FLOPs: the two GEMMs, 4*B*H*N^2*d, halved when causal."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2.0 if self.causal else f
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+WORKLOADS = {
+    "small_b1h1n256d64": Workload("small_b1h1n256d64", 1, 1, 256, 64, False,
+                                  seed=1001),
+    "gpt2s_b4h12n1024d64": Workload("gpt2s_b4h12n1024d64", 4, 12, 1024, 64,
+                                    False, seed=1002),
+    "gpt2s_b4h12n1024d64_causal": Workload("gpt2s_b4h12n1024d64_causal", 4, 12,
+                                           1024, 64, True, seed=1002),
+    "b2h16n4096d128_causal": Workload("b2h16n4096d128_causal", 2, 16, 4096,
+                                      128, True, v_dist="uniform", seed=1003),
+    "tradingday_b1h12n23400d64_causal": Workload(
+        "tradingday_b1h12n23400d64_causal", 1, 12, 23400, 64, True, seed=1004),
+    "long_b1h32n16384d128": Workload("long_b1h32n16384d128", 1, 32, 16384,
+                                     128, False, q_std=2.0, k_std=2.0,
+                                     seed=1005),
+}
+
+# The non-causal N >= 4096, d = 128 case the throughput target is set on.
+HEADLINE = "long_b1h32n16384d128"
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def _normal(shape, std: float, seed: int) -> torch.Tensor:
+    x = torch.randn(shape, generator=_gen(seed), dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.bfloat16)
+
+
+def _uniform(shape, seed: int) -> torch.Tensor:
+    x = torch.rand(shape, generator=_gen(seed), dtype=torch.float32)
+    x.mul_(2.0).sub_(1.0)
+    return x.to(torch.bfloat16)
+
+
+def make_qkv(w: Workload, seed: int | None = None):
+    """(q, k, v) bf16 CPU tensors shaped [B, H, N, d].  Q uses ``seed``, K
+    ``seed + 1`` and V ``seed + 2`` (default: the workload's seed)."""
+    s = w.seed if seed is None else int(seed)
+    shape = (w.B, w.H, w.N, w.d)
+    q = _normal(shape, w.q_std, s)
+    k = _normal(shape, w.k_std, s + 1)
+    if w.v_dist == "normal":
+        v = _normal(shape, 1.0, s + 2)
+    elif w.v_dist == "uniform":
+        v = _uniform(shape, s + 2)
+    else:
+        raise ValueError(f"unknown value distribution {w.v_dist!r}")
+    return q, k, v
+
+
+def shape_case(B: int, H: int, N: int, d: int, causal: bool, seed: int,
+               q_std: float = 1.0, k_std: float = 1.0,
+               v_dist: str = "normal") -> Workload:
+    """An ad-hoc workload for parity sweeps over shapes."""
+    return Workload(f"case_b{B}h{H}n{N}d{d}{'_causal' if causal else ''}",
+                    B, H, N, d, causal, q_std, k_std, v_dist, seed)
+
+
+def sample_rows(w: Workload, count: int, seed: int = 7):
+    """Flat row indices (bh * N + i) for sampled parity checks: always the
+    first and last row of every (b, h) head block that is sampled, the ragged
+    tail rows, plus uniform draws."""
+    g = _gen(seed)
+    total = w.B * w.H * w.N
+    picks = set()
+    for bh in (0, w.B * w.H - 1):
+        base = bh * w.N
+        for i in (0, 1, 127, 128, w.N - 1, w.N - 2):
+            if 0 <= i < w.N:
+                picks.add(base + i)
+    r = torch.randint(0, total, (max(0, count - len(picks)),), generator=g)
+    picks.update(int(x) for x in r)
+    return sorted(picks)

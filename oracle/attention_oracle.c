@@ -1,0 +1,322 @@
+/*
+ * attention_oracle.c -- plain, slow, fp64 CPU oracle for exact attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no code, header, table or constant
+ * with the CUDA library, and it does not include any of the library's files.
+ *
+ * Source cited throughout as [MM]: the marketmaker.cc blog post (Indonesian
+ * edition) "Apakah Konteks Sehari Penuh Mengalahkan Konteks Sepuluh Menit?
+ * Perhatian Kilat dan Pertanyaan Panjang Urutan", cited by section heading.
+ *
+ * What it computes ([MM] "Mengapa perhatian terikat pada memori" and the
+ * explicit three-line PyTorch path in "Integrasinya delapan baris"):
+ *
+ *     S = scale * Q K^T          (scale = 1/sqrt(d_k) in every workload)
+ *     S[i, j] = -inf  if causal and key j lies in the future of query i (j > i)
+ *     O = softmax_rows(S) V
+ *     lse[i] = log(sum_j exp(S[i, j]))     -- natural log over the scaled,
+ *                                             masked scores; this is the
+ *                                             (m, l) pair that section
+ *                                             "Backward pass" says is kept,
+ *                                             folded into one number m + ln l.
+ *
+ * The softmax is the plain two-pass, max-subtracted form (pass 1 finds the
+ * row maximum m, pass 2 sums exp(s - m)); the score row is materialised in
+ * full before either pass.  All arithmetic is IEEE double via libm exp/log,
+ * summed in ascending key order.  Build without -ffast-math.
+ *
+ * A second, deliberately different implementation follows the blocked
+ * algorithm of [MM] "Algoritma Flash Attention" step by step (per-block local
+ * max and sum, running statistics, output rescaled and renormalised at every
+ * block).  It exists only so that the two-pass oracle can be cross-checked
+ * against the pages' own algorithm; it calls none of the two-pass helpers.
+ *
+ * Layout conventions: Q, K, V, O are contiguous row-major [B, H, N, d];
+ * lse is contiguous [B, H, N].  bf16 inputs are passed as their raw 16-bit
+ * patterns and widened exactly to double (bf16 -> fp32 is exact, fp32 ->
+ * fp64 is exact).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EBADARG 1
+#define ORACLE_ENOMEM 2
+
+/* Exact widening of a bfloat16 bit pattern: the pattern is the top half of
+ * an IEEE binary32 value. */
+static double bf16_bits_to_double(uint16_t bits) {
+  uint32_t u = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Number of keys visible to query i: all N keys, or keys 0..i when causal
+ * ([MM] "Causal masking adalah tempat perdagangan mendapat diskon": a query
+ * may not attend to the future; the explicit path masks with -inf, so key i
+ * itself stays visible). */
+static int64_t visible_keys(int64_t i, int64_t N, int causal) {
+  return causal ? (i + 1) : N;
+}
+
+/* The softmax-and-weighted-sum step on one materialised score row.
+ * s[0..n) are finite scores of the visible keys; V points at n rows of d.
+ * Writes o[0..d) and *lse.  p (n doubles, may be NULL) receives the softmax
+ * probabilities when the caller wants to inspect them. */
+static void attend_row(const double *s, int64_t n, const double *V, int64_t d,
+                       double *o, double *lse, double *p) {
+  /* pass 1: row maximum */
+  double m = -INFINITY;
+  for (int64_t j = 0; j < n; ++j)
+    if (s[j] > m) m = s[j];
+  /* pass 2: exponentials and their sum */
+  double l = 0.0;
+  for (int64_t t = 0; t < d; ++t) o[t] = 0.0;
+  for (int64_t j = 0; j < n; ++j) {
+    double e = exp(s[j] - m);
+    l += e;
+    for (int64_t t = 0; t < d; ++t) o[t] += e * V[j * d + t];
+  }
+  for (int64_t t = 0; t < d; ++t) o[t] /= l;
+  *lse = m + log(l);
+  if (p)
+    for (int64_t j = 0; j < n; ++j) p[j] = exp(s[j] - m) / l;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Public entry points (ctypes).                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Softmax of one score row; the pin "every row of probabilities sums to 1"
+ * reads this.  No values are involved: the value width passed down is 0. */
+int oracle_softmax_row(const double *s, int64_t n, double *p) {
+  if (!s || !p || n < 1) return ORACLE_EBADARG;
+  double v_dummy = 0.0, o_dummy = 0.0, lse = 0.0;
+  attend_row(s, n, &v_dummy, 0, &o_dummy, &lse, p);
+  return ORACLE_OK;
+}
+
+/* Attention given an already-materialised score matrix S [rows, n_keys] and
+ * V [n_keys, d]: O[rows, d] = softmax_rows(S) V, lse[rows].  Entries of S
+ * equal to -inf are masked keys and are dropped before the two passes. */
+int oracle_attend_scores(const double *S, const double *V, int64_t rows,
+                         int64_t n_keys, int64_t d, double *O, double *lse) {
+  if (!S || !V || !O || !lse || rows < 0 || n_keys < 1 || d < 1)
+    return ORACLE_EBADARG;
+  double *s = (double *)malloc(sizeof(double) * (size_t)n_keys);
+  double *vv = (double *)malloc(sizeof(double) * (size_t)(n_keys * d));
+  if (!s || !vv) { free(s); free(vv); return ORACLE_ENOMEM; }
+  for (int64_t i = 0; i < rows; ++i) {
+    int64_t n = 0;
+    for (int64_t j = 0; j < n_keys; ++j) {
+      double x = S[i * n_keys + j];
+      if (x == -INFINITY) continue;
+      s[n] = x;
+      memcpy(vv + n * d, V + j * d, sizeof(double) * (size_t)d);
+      ++n;
+    }
+    if (n == 0) { free(s); free(vv); return ORACLE_EBADARG; }
+    attend_row(s, n, vv, d, O + i * d, lse + i, NULL);
+  }
+  free(s);
+  free(vv);
+  return ORACLE_OK;
+}
+
+/* Full attention over fp64 inputs: the definition, one (b, h, i) row at a
+ * time.  For each row the whole score row is materialised, then the two
+ * softmax passes run over it.  OpenMP parallel over rows. */
+int oracle_attention_f64(const double *Q, const double *K, const double *V,
+                         double *O, double *lse, int64_t B, int64_t H,
+                         int64_t N, int64_t d, int causal, double scale,
+                         int nthreads) {
+  if (!Q || !K || !V || !O || !lse || B < 0 || H < 0 || N < 0 || d < 1)
+    return ORACLE_EBADARG;
+  const int64_t rows = B * H * N;
+  if (rows == 0) return ORACLE_OK;
+  int err = ORACLE_OK;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!s) {
+#pragma omp atomic write
+      err = ORACLE_ENOMEM;
+    }
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t r = 0; r < rows; ++r) {
+      if (!s) continue;
+      const int64_t bh = r / N, i = r % N;
+      const double *Kh = K + bh * N * d, *Vh = V + bh * N * d;
+      const double *qi = Q + r * d;
+      const int64_t n = visible_keys(i, N, causal);
+      for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < d; ++t) acc += qi[t] * Kh[j * d + t];
+        s[j] = scale * acc;
+      }
+      attend_row(s, n, Vh, d, O + r * d, lse + r, NULL);
+    }
+    free(s);
+  }
+  return err;
+}
+
+/* Attention on selected rows of bf16 inputs (raw bit patterns).  rows[k] is
+ * a flat row index bh * N + i; O_out is [nrows, d] fp64, lse_out [nrows].
+ * The key and value rows a query needs are widened to fp64 on the fly, so
+ * full-size workloads can be checked row by row without an fp64 copy. */
+int oracle_attention_rows_bf16(const uint16_t *Q, const uint16_t *K,
+                               const uint16_t *V, int64_t B, int64_t H,
+                               int64_t N, int64_t d, int causal, double scale,
+                               const int64_t *rows, int64_t nrows,
+                               double *O_out, double *lse_out, int nthreads) {
+  if (!Q || !K || !V || !rows || !O_out || !lse_out || B < 0 || H < 0 ||
+      N < 1 || d < 1 || nrows < 0)
+    return ORACLE_EBADARG;
+  for (int64_t k = 0; k < nrows; ++k)
+    if (rows[k] < 0 || rows[k] >= B * H * N) return ORACLE_EBADARG;
+  int err = ORACLE_OK;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *qi = (double *)malloc(sizeof(double) * (size_t)d);
+    double *vv = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    if (!s || !qi || !vv) {
+#pragma omp atomic write
+      err = ORACLE_ENOMEM;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t k = 0; k < nrows; ++k) {
+      if (!s || !qi || !vv) continue;
+      const int64_t r = rows[k];
+      const int64_t bh = r / N, i = r % N;
+      const uint16_t *Kh = K + bh * N * d, *Vh = V + bh * N * d;
+      for (int64_t t = 0; t < d; ++t) qi[t] = bf16_bits_to_double(Q[r * d + t]);
+      const int64_t n = visible_keys(i, N, causal);
+      for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < d; ++t)
+          acc += qi[t] * bf16_bits_to_double(Kh[j * d + t]);
+        s[j] = scale * acc;
+        for (int64_t t = 0; t < d; ++t)
+          vv[j * d + t] = bf16_bits_to_double(Vh[j * d + t]);
+      }
+      attend_row(s, n, vv, d, O_out + k * d, lse_out + k, NULL);
+    }
+    free(s);
+    free(qi);
+    free(vv);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The pages' blocked algorithm, as a second opinion on the oracle.         */
+/* ------------------------------------------------------------------------ */
+
+/* [MM] "Algoritma Flash Attention": Q is cut into blocks of Br rows and K, V
+ * into blocks of Bc rows.  For every query block the output O_i starts at 0,
+ * the running maximum m_i at -inf and the running sum l_i at 0.  For every
+ * key/value block: form the block of scores, take its row maximum m_ij,
+ * exponentiate against that local maximum to get P_ij, take its row sum
+ * l_ij, then merge into the running statistics with
+ *     m_new = max(m_i, m_ij)
+ *     l_new = l_i e^(m_i - m_new) + l_ij e^(m_ij - m_new)
+ * and replace O_i by the renormalised mix of the old output (weight
+ * l_i e^(m_i - m_new) / l_new) and P_ij V_j (weight e^(m_ij - m_new) / l_new).
+ * [MM] "Pengulangan softmax online" says this equals the two-pass softmax in
+ * exact arithmetic.  lse is m_i + ln l_i after the last block.
+ *
+ * Reading where the pages are silent: with a causal mask a row of a block
+ * can be entirely masked (all keys in its future).  Such a row has no local
+ * maximum; it contributes nothing and its running statistics are left as
+ * they were.  Blocks whose keys all lie in every query's future are skipped
+ * outright ([MM] "Causal masking ...").  Works on fp64 inputs. */
+int oracle_attention_blocked_f64(const double *Q, const double *K,
+                                 const double *V, double *O, double *lse,
+                                 int64_t B, int64_t H, int64_t N, int64_t d,
+                                 int causal, double scale, int64_t Br,
+                                 int64_t Bc) {
+  if (!Q || !K || !V || !O || !lse || B < 0 || H < 0 || N < 0 || d < 1 ||
+      Br < 1 || Bc < 1)
+    return ORACLE_EBADARG;
+  double *Sij = (double *)malloc(sizeof(double) * (size_t)(Br * Bc));
+  double *PV = (double *)malloc(sizeof(double) * (size_t)(Br * d));
+  double *mi = (double *)malloc(sizeof(double) * (size_t)Br);
+  double *li = (double *)malloc(sizeof(double) * (size_t)Br);
+  if (!Sij || !PV || !mi || !li) {
+    free(Sij); free(PV); free(mi); free(li);
+    return ORACLE_ENOMEM;
+  }
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    const double *Qh = Q + bh * N * d, *Kh = K + bh * N * d,
+                 *Vh = V + bh * N * d;
+    double *Oh = O + bh * N * d, *lh = lse + bh * N;
+    for (int64_t q0 = 0; q0 < N; q0 += Br) {
+      const int64_t nr = (N - q0 < Br) ? (N - q0) : Br;
+      for (int64_t r = 0; r < nr; ++r) {
+        mi[r] = -INFINITY;
+        li[r] = 0.0;
+        for (int64_t t = 0; t < d; ++t) Oh[(q0 + r) * d + t] = 0.0;
+      }
+      for (int64_t k0 = 0; k0 < N; k0 += Bc) {
+        if (causal && k0 > q0 + nr - 1) break; /* whole block in the future */
+        const int64_t nc = (N - k0 < Bc) ? (N - k0) : Bc;
+        /* S_ij = Q_i K_j^T * scale, masked */
+        for (int64_t r = 0; r < nr; ++r)
+          for (int64_t c = 0; c < nc; ++c) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < d; ++t)
+              acc += Qh[(q0 + r) * d + t] * Kh[(k0 + c) * d + t];
+            Sij[r * Bc + c] =
+                (causal && k0 + c > q0 + r) ? -INFINITY : scale * acc;
+          }
+        for (int64_t r = 0; r < nr; ++r) {
+          /* m_ij = rowmax(S_ij) */
+          double mij = -INFINITY;
+          for (int64_t c = 0; c < nc; ++c)
+            if (Sij[r * Bc + c] > mij) mij = Sij[r * Bc + c];
+          if (mij == -INFINITY) continue; /* row fully masked in this block */
+          /* P_ij = exp(S_ij - m_ij), l_ij = rowsum(P_ij), (P_ij V_j) */
+          double lij = 0.0;
+          for (int64_t t = 0; t < d; ++t) PV[r * d + t] = 0.0;
+          for (int64_t c = 0; c < nc; ++c) {
+            double pc = exp(Sij[r * Bc + c] - mij);
+            lij += pc;
+            for (int64_t t = 0; t < d; ++t) PV[r * d + t] += pc * Vh[(k0 + c) * d + t];
+          }
+          /* merge into the running statistics */
+          const double mnew = (mi[r] > mij) ? mi[r] : mij;
+          const double wold = li[r] * exp(mi[r] - mnew); /* 0 when li = 0 */
+          const double wnew = exp(mij - mnew);
+          const double lnew = wold + lij * wnew;
+          double *orow = Oh + (q0 + r) * d;
+          for (int64_t t = 0; t < d; ++t)
+            orow[t] = orow[t] * (wold / lnew) + PV[r * d + t] * (wnew / lnew);
+          mi[r] = mnew;
+          li[r] = lnew;
+        }
+      }
+      for (int64_t r = 0; r < nr; ++r) lh[q0 + r] = mi[r] + log(li[r]);
+    }
+  }
+  free(Sij); free(PV); free(mi); free(li);
+  return ORACLE_OK;
+}
+
+/* Threads OpenMP would use by default (for reporting). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
