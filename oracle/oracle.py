@@ -21,7 +21,9 @@ def library_path() -> str:
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(_build())
+        # ORACLE_LIBRARY lets the mutation test point the pins at a copy of
+        # the oracle with a planted mistake; normally the built library loads.
+        lib = ctypes.CDLL(os.environ.get("ORACLE_LIBRARY") or _build())
         dp = ctypes.POINTER(ctypes.c_double)
         u16p = ctypes.POINTER(ctypes.c_uint16)
         i64p = ctypes.POINTER(ctypes.c_int64)

@@ -1,0 +1,70 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case copies ``oracle/attention_oracle.c``, plants one mistake (a dropped
+term, a wrong sign or index, a swapped operand, a misplaced mask boundary),
+compiles the copy on the CPU and runs ``tests/test_oracle_pins.py`` against
+it.  The pins pass on the real oracle (that file's own run) and must fail on
+every mutant.  Mistakes are chosen so that every memory access stays in
+bounds.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "attention_oracle.c")
+
+MUTANTS = {
+    "mask_hides_diagonal": ("return causal ? (i + 1) : N;",
+                            "return causal ? (i > 0 ? i : 1) : N;"),
+    "mask_leaks_next_key": ("return causal ? (i + 1) : N;",
+                            "return causal ? (i + 1 < N ? i + 2 : N) : N;"),
+    "no_max_subtraction": ("double e = exp(s[j] - m);", "double e = exp(s[j]);"),
+    "lse_drops_max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "no_normalisation": ("for (int64_t t = 0; t < d; ++t) o[t] /= l;", ""),
+    "scale_dropped": ("s[j] = scale * acc;", "s[j] = acc;"),
+    "scale_squared": ("s[j] = scale * acc;", "s[j] = scale * scale * acc;"),
+    "keys_replaced_by_values": ("acc += qi[t] * Kh[j * d + t];",
+                                "acc += qi[t] * Vh[j * d + t];"),
+    "values_reversed": ("o[t] += e * V[j * d + t];",
+                        "o[t] += e * V[(n - 1 - j) * d + t];"),
+    "max_sign_flipped": ("if (s[j] > m) m = s[j];",
+                         "if (-s[j] > m) m = -s[j];"),
+    "sum_sign_flipped": ("l += e;", "l -= e;"),
+}
+
+
+def _build_mutant(name, tmpdir):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    path_c = os.path.join(tmpdir, f"{name}.c")
+    path_so = os.path.join(tmpdir, f"{name}.so")
+    with open(path_c, "w") as f:
+        f.write(src.replace(old, new))
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                    path_c, "-o", path_so, "-lm"], check=True)
+    return path_so
+
+
+def test_every_planted_mistake_fails_a_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        procs = {}
+        for name in MUTANTS:
+            so = _build_mutant(name, tmp)
+            env = dict(os.environ, ORACLE_LIBRARY=so)
+            procs[name] = subprocess.Popen(
+                [sys.executable, "-m", "pytest", "-q", "-x", "-p",
+                 "no:cacheprovider", os.path.join(ROOT, "tests",
+                                                  "test_oracle_pins.py")],
+                cwd=ROOT, env=env, stdout=subprocess.PIPE,
+                stderr=subprocess.STDOUT)
+        survivors = []
+        for name, p in procs.items():
+            out, _ = p.communicate(timeout=600)
+            if p.returncode == 0:
+                survivors.append(name)
+        assert not survivors, f"pins did not catch: {survivors}"
