@@ -1,0 +1,391 @@
+"""Benchmark of the B200 exact attention forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+A step is one attention forward pass over the whole workload (default: the
+non-causal B=1, H=32, N=16384, d=128 case the throughput target is set on),
+i.e. one launch of the sm_100a kernel through the C ABI.  Inputs are seeded
+synthetic bf16 tensors (``exact_io_aware_73_b200.workloads``), resident in
+HBM before timing starts.  Metric: TFLOP/s with FLOPs = 4 B H N^2 d (halved
+when causal), the convention of the two attention GEMMs.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the full workload
+on its own GPU with its own seed -- independent problems, no collective on
+the data path (weak scaling); value = all ranks' FLOPs / max-over-ranks time.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this
+repository: the pages ship no runnable code) on a bounded sample of rows of
+the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_73_b200 import workloads as W  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (bf16, causal/non-causal) and % of B200 dense BF16 peak"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+KERNEL_NAME = "attn_fwd_sm100_kernel"
+CSRC = os.path.join(ROOT, "exact_io_aware_73_b200", "csrc")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu capture of this workload,
+    or None when there is none or the kernel changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return t.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(w, qkv, budget_s: float, seed: int = 11):
+    """The fp64 oracle (as it stands) on sampled rows of the workload, all
+    host cores; returns the baseline object for the JSON line."""
+    import numpy as np
+    import oracle
+    q, k, v = qkv
+    bits = [oracle.bf16_bits(t) for t in (q, k, v)]
+    threads = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(seed)
+    total_rows = w.B * w.H * w.N
+
+    def row_flops(rows):
+        i = rows % w.N
+        keys = (i + 1) if w.causal else np.full_like(i, w.N)
+        return float(np.sum(4.0 * keys * w.d))
+
+    # calibrate on a small batch, then run a batch sized to the budget
+    done_rows, done_flops, elapsed = 0, 0.0, 0.0
+    batch = max(threads, 8)
+    while elapsed < budget_s:
+        rows = rng.integers(0, total_rows, size=batch)
+        t0 = time.perf_counter()
+        oracle.attention_rows_bf16(*bits, w.causal, w.scale, rows, threads)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        done_rows += batch
+        done_flops += row_flops(rows)
+        rate = batch / max(dt, 1e-6)
+        batch = int(min(max(threads, rate * (budget_s - elapsed) * 0.9),
+                        total_rows))
+        if budget_s - elapsed < 0.5:
+            break
+    return {"value": done_flops / elapsed / 1e12, "unit": "TFLOP/s",
+            "cores": threads, "kind": "oracle",
+            "sample": f"{done_rows} random query rows of {w.name} "
+                      f"({done_rows / total_rows:.2e} of the workload), fp64 "
+                      f"two-pass oracle, {elapsed:.1f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    qkv = W.make_qkv(w)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, qkv, per_step / 4)
+    vals = []
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        vals.append(cpu_baseline(w, qkv, per_step, seed=100 + s))
+    wall = time.perf_counter() - t0
+    value = statistics.mean(v["value"] for v in vals)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    cb["sample"] = (f"each step: {per_step:.0f} s of random query rows of "
+                    f"{w.name}; " + vals[-1]["sample"])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * wall / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_73_b200 import attn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- inputs (seeded per rank), resident in HBM before timing
+    seed = w.seed + 7919 * rank
+    qkv_host = W.make_qkv(w, seed=seed)
+    q, k, v = (t.to(dev) for t in qkv_host)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    in_bytes = 3 * q.numel() * 2
+    flush = None if in_bytes > L2_BYTES else torch.empty(
+        2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        rc = attn.attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                               o.data_ptr(), lse.data_ptr(), w.B, w.H, w.N,
+                               w.d, w.causal, w.scale, sh)
+        if rc != 0:
+            raise attn.AttnError(rc, "attn_fwd")
+
+    for _ in range(args.warmup):
+        step()
+    rc = attn.status()
+    if rc != 0:
+        raise attn.AttnError(rc, "warm-up")
+
+    # ---- device-timed region
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    if flush is None:
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+        torch.cuda.synchronize(dev)
+        kernel_ms = ev0.elapsed_time(ev1)
+        l2_note = (f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB of Q/K/V "
+                   f"vs 126 MiB); back-to-back launches")
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            step()
+            b.record(stream)
+        barrier()
+        torch.cuda.synchronize(dev)
+        kernel_ms = sum(a.elapsed_time(b) for a, b in evs)
+        l2_note = "L2 flushed between steps (252 MiB write outside the events)"
+    clk = clocks.stop()
+    rc = attn.status()
+    if rc != 0:
+        raise attn.AttnError(rc, "timed region")
+
+    t = torch.tensor([kernel_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    ms_per_step = max_ms / args.steps
+    flops = w.flops()
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the host-buffer C entry point
+    qh, kh, vh = (x.pin_memory() for x in qkv_host)
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    ws = torch.empty(attn.host_workspace_bytes(w.B, w.H, w.N, w.d),
+                     dtype=torch.uint8, device=dev)
+    del q, k, v, o, lse
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        attn.attn_fwd_host(qh, kh, vh, oh, lh, w.causal, w.scale, ws, stream=sh)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        attn.attn_fwd_host(qh, kh, vh, oh, lh, w.causal, w.scale, ws, stream=sh)
+    e1.record(stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    rc = attn.status()
+    if rc != 0:
+        raise attn.AttnError(rc, "e2e region")
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item()) / e2e_steps
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    h2d = 3 * qh.numel() * 2
+    d2h = oh.numel() * 2 + lh.numel() * 4
+
+    # ---- roofline of the one kernel (the whole step is one launch)
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    roofline = {
+        "bound": "tensor", "achieved": achieved,
+        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+        "frac": achieved / peaks["bf16_tflops"],
+        "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+        "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
+        "traffic": load_traffic(w.name),
+        "algorithmic_flops_per_launch": flops,
+        "kernel": KERNEL_NAME,
+    }
+
+    cb = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_baseline(w, qkv_host, args.cpu_budget_s)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian/uniform bf16 inputs)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N,
+                       "d": w.d, "causal": w.causal, "scale": w.scale,
+                       "l2": l2_note,
+                       "parallelism": (f"{world} independent replicas (one "
+                                       "workload per GPU, no collective)")},
+            "roofline": roofline,
+            "cpu_baseline": cb,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "steps": e2e_steps,
+                    "api": "attn_fwd_host (pinned host buffers)"},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

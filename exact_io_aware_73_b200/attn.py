@@ -1,0 +1,151 @@
+"""Thin ctypes binding of ``libattn_b200.so`` (C ABI in ``include/attn_b200.h``).
+
+Argument marshalling only: every step of the attention forward pass runs in
+the library's sm_100a kernel.  There is no fallback of any kind -- if the
+library is missing or refuses the call, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libattn_b200.so")
+
+ATTN_OK = 0
+ERROR_NAMES = {
+    1: "ATTN_ERR_NULL_POINTER", 2: "ATTN_ERR_INVALID_SIZE",
+    3: "ATTN_ERR_UNSUPPORTED_HEAD_DIM", 4: "ATTN_ERR_MISALIGNED",
+    5: "ATTN_ERR_INVALID_SCALE", 6: "ATTN_ERR_ALIAS",
+    7: "ATTN_ERR_UNSUPPORTED_DEVICE", 8: "ATTN_ERR_CUDA",
+    9: "ATTN_ERR_TENSOR_MAP", 10: "ATTN_ERR_NOT_DEVICE_MEMORY",
+    11: "ATTN_ERR_WORKSPACE", 16: "ATTN_ERR_DEVICE_TIMEOUT",
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        msg = lib().attn_strerror(code).decode()
+        super().__init__(f"{what}: {ERROR_NAMES.get(code, code)} ({msg})")
+
+
+def lib():
+    """Load the CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m exact_io_aware_73_b200.build` (no fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i,
+                               ctypes.c_float, vp]
+        L.attn_fwd.restype = i
+        L.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i,
+                                    ctypes.c_float, vp, ctypes.c_size_t, vp]
+        L.attn_fwd_host.restype = i
+        L.attn_fwd_host_workspace_bytes.argtypes = [i, i, i, i]
+        L.attn_fwd_host_workspace_bytes.restype = ctypes.c_size_t
+        L.attn_status.argtypes = [vp]
+        L.attn_status.restype = i
+        L.attn_last_status_bits.argtypes = []
+        L.attn_last_status_bits.restype = ctypes.c_uint32
+        L.attn_strerror.argtypes = [i]
+        L.attn_strerror.restype = ctypes.c_char_p
+        L.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.attn_set_wait_timeout_ns.restype = None
+        L.attn_set_fault_injection.argtypes = [ctypes.c_uint32]
+        L.attn_set_fault_injection.restype = None
+        _lib = L
+    return _lib
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return int(getattr(stream, "cuda_stream", stream))
+
+
+def _check(rc: int, what: str):
+    if rc != ATTN_OK:
+        raise AttnError(rc, what)
+
+
+def attn_fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal,
+                 scale, stream_handle) -> int:
+    """Direct call with integer pointers; returns the library's code."""
+    return lib().attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, int(B), int(H),
+                          int(N), int(d), int(bool(causal)), float(scale),
+                          stream_handle)
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None,
+             out=None, lse=None, stream=None):
+    """O, lse = exact attention forward of bf16 CUDA tensors [B, H, N, d].
+
+    Allocates O (bf16) and lse (fp32 [B, H, N]) with torch unless given.
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 4:
+            raise TypeError(f"{name} must be a 4-D bf16 CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, d]")
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                      lse.data_ptr(), B, H, N, d, causal, scale,
+                      _stream_handle(stream))
+    _check(rc, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_host(q, k, v, out, lse, causal: bool, scale: float, workspace,
+                  stream=None):
+    """End-to-end call on host (ideally pinned) bf16 tensors; `workspace` is a
+    CUDA uint8 tensor of at least ``host_workspace_bytes`` bytes.  Queued on
+    `stream`; synchronise before reading `out` / `lse`."""
+    B, H, N, d = q.shape
+    rc = lib().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                             out.data_ptr(), lse.data_ptr(), B, H, N, d,
+                             int(bool(causal)), float(scale),
+                             workspace.data_ptr(), workspace.numel(),
+                             _stream_handle(stream))
+    _check(rc, "attn_fwd_host")
+
+
+def host_workspace_bytes(B, H, N, d) -> int:
+    return int(lib().attn_fwd_host_workspace_bytes(B, H, N, d))
+
+
+def status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status."""
+    return int(lib().attn_status(_stream_handle(stream)))
+
+
+def last_status_bits() -> int:
+    return int(lib().attn_last_status_bits())
+
+
+def strerror(code: int) -> str:
+    return lib().attn_strerror(int(code)).decode()
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    lib().attn_set_wait_timeout_ns(int(ns))
+
+
+def set_fault_injection(flags: int) -> None:
+    lib().attn_set_fault_injection(int(flags))

@@ -1,0 +1,344 @@
+// attn_api.cu -- host side of the C ABI declared in include/attn_b200.h:
+// argument validation, TMA descriptor encoding, kernel selection and launch,
+// the per-device status word, and the host-buffer (end-to-end) entry point.
+//
+// The operation and its layouts are defined in the header.  This file makes
+// no CUDA call before every argument check has passed.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_b200.h"
+#include "attn_fwd_kernel.cuh"
+
+namespace {
+
+using attn_b200::FwdParams;
+using attn_b200::Smem;
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
+
+struct DeviceState {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  uint32_t *status = nullptr;  // 4-byte device status word, lazily allocated
+  bool smem_attr_set[4] = {false, false, false, false};
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<uint32_t> g_inject{0};
+std::atomic<uint32_t> g_last_bits{0};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
+                                  void *, const cuuint64_t *, const cuuint64_t *,
+                                  const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int get_encode_fn(EncodeTiledFn *out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion(
+        "cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+      return ATTN_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *out = g_encode;
+  return ATTN_OK;
+}
+
+// Current device, checked to be a B200 (compute capability 10.0); allocates
+// the device's status word on first use.
+int current_device(int *dev_out, DeviceState **st_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return ATTN_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState &st = g_dev[dev];
+  if (!st.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_UNSUPPORTED_DEVICE;
+    }
+    st.probed = true;
+    st.supported = (major == 10 && minor == 0);
+    st.sm_count = sms;
+  }
+  if (!st.supported) return ATTN_ERR_UNSUPPORTED_DEVICE;
+  if (!st.status) {
+    void *p = nullptr;
+    if (cudaMalloc(&p, sizeof(uint32_t)) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    if (cudaMemset(p, 0, sizeof(uint32_t)) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(p);
+      return ATTN_ERR_CUDA;
+    }
+    st.status = static_cast<uint32_t *>(p);
+  }
+  *dev_out = dev;
+  *st_out = &st;
+  return ATTN_OK;
+}
+
+bool is_device_memory_of(const void *p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) &&
+         a.device == dev;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a);
+  const uintptr_t y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Shape / pointer checks shared by both entry points (no CUDA calls).
+int check_args(const void *q, const void *k, const void *v, const void *o,
+               const float *lse, int B, int H, int N, int d, float scale,
+               bool check_alignment) {
+  if (B < 0 || H < 0 || N < 0) return ATTN_ERR_INVALID_SIZE;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID_SCALE;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL_POINTER;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  if (N > ATTN_MAX_SEQ || bh > ATTN_MAX_HEADS) return ATTN_ERR_INVALID_SIZE;
+  const int64_t units = bh * ((N + 255) / 256);
+  if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_SIZE;
+  if (check_alignment) {
+    auto al = [](const void *p, uintptr_t a) {
+      return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+    };
+    if (!al(q, 16) || !al(k, 16) || !al(v, 16) || !al(o, 16) || !al(lse, 4))
+      return ATTN_ERR_MISALIGNED;
+  }
+  const size_t tbytes = static_cast<size_t>(bh) * N * d * 2;
+  const size_t lbytes = static_cast<size_t>(bh) * N * 4;
+  if (overlaps(o, tbytes, q, tbytes) || overlaps(o, tbytes, k, tbytes) ||
+      overlaps(o, tbytes, v, tbytes) || overlaps(lse, lbytes, q, tbytes) ||
+      overlaps(lse, lbytes, k, tbytes) || overlaps(lse, lbytes, v, tbytes) ||
+      overlaps(lse, lbytes, o, tbytes))
+    return ATTN_ERR_ALIAS;
+  return ATTN_OK;
+}
+
+// [B*H, N, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 64 x 128
+// rows, 128-byte swizzle -- the shared-memory layout the UMMA descriptors in
+// the kernel expect.  Rows beyond N read as zero.
+int encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *ptr, int bh,
+               int N, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void *>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_TENSOR_MAP;
+}
+
+template <int D, bool CAUSAL>
+int launch(DeviceState &st, int variant, const CUtensorMap *maps,
+           const FwdParams &p, cudaStream_t stream) {
+  auto kern = attn_b200::attn_fwd_sm100_kernel<D, CAUSAL>;
+  const uint32_t smem = Smem<D>::kAlloc;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!st.smem_attr_set[variant]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      st.smem_attr_set[variant] = true;
+    }
+  }
+  const int grid = p.num_units < st.sm_count ? p.num_units : st.sm_count;
+  kern<<<grid, attn_b200::kThreads, smem, stream>>>(maps[0], maps[1], maps[2], p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int H, int N, int d, int causal, float scale,
+             attn_stream_t stream) {
+  int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, true);
+  if (rc != ATTN_OK || B == 0 || H == 0 || N == 0) return rc;
+
+  int dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  if (!is_device_memory_of(q, dev) || !is_device_memory_of(k, dev) ||
+      !is_device_memory_of(v, dev) || !is_device_memory_of(o, dev) ||
+      !is_device_memory_of(lse, dev))
+    return ATTN_ERR_NOT_DEVICE_MEMORY;
+
+  EncodeTiledFn enc;
+  if ((rc = get_encode_fn(&enc)) != ATTN_OK) return rc;
+  const int bh = B * H;
+  CUtensorMap maps[3];
+  if ((rc = encode_map(enc, &maps[0], q, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[1], k, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[2], v, bh, N, d)) != ATTN_OK) return rc;
+
+  FwdParams p;
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.status = st->status;
+  p.bh = bh;
+  p.n = N;
+  p.num_units = bh * ((N + 255) / 256);
+  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.timeout_ns = g_timeout_ns.load();
+  p.debug_flags = g_inject.load();
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch<128, true>(*st, 0, maps, p, s)
+                  : launch<128, false>(*st, 1, maps, p, s);
+  return causal ? launch<64, true>(*st, 2, maps, p, s)
+                : launch<64, false>(*st, 3, maps, p, s);
+}
+
+size_t attn_fwd_host_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128)) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return 4 * round256(rows * d * 2) + round256(rows * 4);
+}
+
+int attn_fwd_host(const void *q, const void *k, const void *v, void *o,
+                  float *lse, int B, int H, int N, int d, int causal,
+                  float scale, void *workspace, size_t workspace_bytes,
+                  attn_stream_t stream) {
+  int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, false);
+  if (rc != ATTN_OK || B == 0 || H == 0 || N == 0) return rc;
+  const size_t need = attn_fwd_host_workspace_bytes(B, H, N, d);
+  if (!workspace || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+    return ATTN_ERR_WORKSPACE;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  const size_t tb = rows * d * 2, tbr = round256(tb);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  void *dq = ws, *dk = ws + tbr, *dv = ws + 2 * tbr, *dout = ws + 3 * tbr;
+  float *dl = reinterpret_cast<float *>(ws + 4 * tbr);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  if (cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  rc = attn_fwd(dq, dk, dv, dout, dl, B, H, N, d, causal, scale, stream);
+  if (rc != ATTN_OK) return rc;
+  if (cudaMemcpyAsync(o, dout, tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(lse, dl, rows * 4, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+int attn_status(attn_stream_t stream) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return ATTN_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  uint32_t *word;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    word = g_dev[dev].status;
+  }
+  if (!word) return ATTN_OK;
+  uint32_t bits = 0;
+  if (cudaMemcpy(&bits, word, sizeof bits, cudaMemcpyDeviceToHost) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  if (bits == 0) return ATTN_OK;
+  g_last_bits.store(bits);
+  if (cudaMemset(word, 0, sizeof bits) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return (bits & attn_b200::kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT
+                                            : ATTN_ERR_CUDA;
+}
+
+uint32_t attn_last_status_bits(void) { return g_last_bits.load(); }
+
+const char *attn_strerror(int code) {
+  switch (code) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case ATTN_ERR_INVALID_SIZE: return "B, H or N negative or beyond the supported limits";
+    case ATTN_ERR_UNSUPPORTED_HEAD_DIM: return "head dimension must be 64 or 128";
+    case ATTN_ERR_MISALIGNED: return "q/k/v/o must be 16-byte aligned and lse 4-byte aligned";
+    case ATTN_ERR_INVALID_SCALE: return "scale must be finite and > 0";
+    case ATTN_ERR_ALIAS: return "o or lse overlaps an input or each other";
+    case ATTN_ERR_UNSUPPORTED_DEVICE: return "no CUDA device, or the current device is not a B200 (compute capability 10.0)";
+    case ATTN_ERR_CUDA: return "a CUDA runtime call or the kernel launch failed";
+    case ATTN_ERR_TENSOR_MAP: return "TMA tensor-map encoding failed";
+    case ATTN_ERR_NOT_DEVICE_MEMORY: return "a buffer is not device memory of the current device";
+    case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "a pipeline wait in the kernel ran out of time; outputs are invalid";
+    default: return "unknown error code";
+  }
+}
+
+void attn_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs);
+}
+
+void attn_set_fault_injection(uint32_t flags) { g_inject.store(flags & 1u); }
+
+}  // extern "C"

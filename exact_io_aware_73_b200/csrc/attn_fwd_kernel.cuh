@@ -1,0 +1,606 @@
+// attn_fwd_kernel.cuh -- exact attention forward for B200 (sm_100a).
+//
+// Computes, per (batch, head), O = softmax(scale * Q K^T [causal mask]) V and
+// lse = ln(row sum of exp(scaled scores)), walking key/value tiles with the
+// online-softmax recurrence so the N x N score matrix never reaches HBM.
+//
+// Source cited as [MM]: the marketmaker.cc blog post (Indonesian edition)
+// "Apakah Konteks Sehari Penuh Mengalahkan Konteks Sepuluh Menit? Perhatian
+// Kilat dan Pertanyaan Panjang Urutan", by section heading.
+//
+//   * tiles Q_i (128 rows) and K_j, V_j (128 keys) staged on chip, one pass
+//     over the key/value blocks per query block  ([MM] "Algoritma Flash
+//     Attention");
+//   * running max / running sum with retroactive rescaling of the output,
+//     normalised once at the end ([MM] "Pengulangan softmax online",
+//     "FA2: paralelisme" item 1);
+//   * work split over batch x heads x query blocks ([MM] "FA2: paralelisme"
+//     item 2); each softmax thread owns one query row, so no cross-warp
+//     reduction is needed (item 3);
+//   * a loader warp issuing asynchronous tensor copies for the next key/value
+//     block while the other warps compute on the current one, and the two
+//     GEMMs of one query tile overlapping the softmax of the other
+//     ([MM] "FA3: Mekanika hopper" items 1 and 2);
+//   * key/value blocks entirely in a query block's future are never loaded
+//     or computed ([MM] "Causal masking adalah tempat perdagangan mendapat
+//     diskon").
+//
+// Blackwell mapping (not the pages' Hopper design):
+//   * a persistent CTA per SM walks "units" = two 128-row Q tiles of one
+//     (batch, head) that share every K/V tile it loads;
+//   * warps 0-3 / 4-7: softmax warpgroups for Q tile 0 / 1 (one TMEM lane =
+//     one query row per thread); warp 8: TMA loader; warp 9: tcgen05 MMA
+//     issuer (one thread) and TMEM owner;
+//   * TMEM (512 columns x 128 lanes x 32 bit): S0 | S1 | O0 | O1.  The
+//     softmax writes P (bf16) back over the first 64 columns of its S tile;
+//     the P.V MMA reads it from TMEM as its A operand;
+//   * S = Q K^T: tcgen05.mma kind::f16, M=128 N=128 K=d, A and B K-major in
+//     128B-swizzled shared memory (exactly the layout the TMA writes);
+//     O += P V: M=128 N=d K=128, A from TMEM, B (V) MN-major in shared memory;
+//   * each softmax thread writes its own output row straight from TMEM to
+//     HBM (16-byte stores); Q tiles are released by a tcgen05.commit after
+//     their last S MMA, so the next unit's Q load overlaps this epilogue;
+//   * the row max is rescaled lazily: the output is only corrected when a
+//     row's running max grows by more than 2^8 (in exp2 units); P then stays
+//     below 256, and O / l is unchanged because m and l always move together;
+//   * every wait is bounded in time; a wait that runs out records it in a
+//     device status word, the CTA drains its in-flight copies, frees its
+//     tensor memory and exits.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <math_constants.h>
+
+#include "ptx_sm100.cuh"
+
+namespace attn_b200 {
+
+constexpr int kBlockM = 128;   // query rows per Q tile (= TMEM lanes)
+constexpr int kBlockN = 128;   // keys per K/V tile
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P <= 2^8
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Device status word bits.
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kRoleProducer = 1u << 8;
+constexpr uint32_t kRoleMma = 1u << 9;
+constexpr uint32_t kRoleSoftmax = 1u << 10;
+constexpr uint32_t kRoleEpilogue = 1u << 11;
+constexpr uint32_t kRoleDrain = 1u << 12;
+
+struct FwdParams {
+  uint16_t *o;         // [BH, N, D] bf16
+  float *lse;          // [BH, N] fp32
+  uint32_t *status;    // device status word
+  int bh;              // B * H
+  int n;               // sequence length
+  int num_units;       // bh * ceil(n / 256)
+  float c_log2;        // scale * log2(e)
+  unsigned long long timeout_ns;
+  uint32_t debug_flags;  // bit 0: first CTA skips its first Q copy
+};
+
+// Shared-memory map (offsets from a 1024-byte aligned base).
+template <int D>
+struct Smem {
+  static constexpr int kSub = D / 64;                         // 64-col panels
+  static constexpr uint32_t kPanelBytes = kBlockM * 128;      // 128 rows x 128 B
+  static constexpr uint32_t kTileBytes = kBlockM * D * 2;     // one Q/K/V tile
+  static constexpr int kStages = (D == 128) ? 2 : 4;          // K and V ring depth
+  static constexpr uint32_t kQ = 0;                           // 2 Q tiles
+  static constexpr uint32_t kK = kQ + 2 * kTileBytes;         // K ring
+  static constexpr uint32_t kV = kK + kStages * kTileBytes;   // V ring
+  static constexpr uint32_t kBars = kV + kStages * kTileBytes;
+  // barrier indices
+  static constexpr int Q_FULL = 0, Q_EMPTY = 2, S_FULL = 4, P_FULL = 6,
+                       O_FULL = 8, O_EMPTY = 10, DRAIN = 12,
+                       K_FULL = 13, K_EMPTY = K_FULL + kStages,
+                       V_FULL = K_EMPTY + kStages, V_EMPTY = V_FULL + kStages,
+                       NUM_BARS = V_EMPTY + kStages;
+  static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;  // tmem slot, abort
+  static constexpr uint32_t kBytes = kMisc + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for alignment
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+// One work unit: rows [q0, q0 + 256) of head bh, as two Q tiles; n0 / n1 =
+// number of K/V tiles each Q tile visits (0 = tile lies beyond N).
+struct Unit {
+  int bh, q0, n0, n1;
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ Unit decode_unit(int u, int bh_count, int n) {
+  const int qpairs = (n + 255) >> 8;
+  const int tiles = (n + 127) >> 7;
+  Unit w;
+  int qp;
+  if (CAUSAL) {
+    // heaviest units (last query rows) first, heads interleaved
+    qp = qpairs - 1 - u / bh_count;
+    w.bh = u % bh_count;
+  } else {
+    // consecutive units share a head's K/V in L2
+    w.bh = u / qpairs;
+    qp = u % qpairs;
+  }
+  w.q0 = qp * 256;
+  const int qt0 = w.q0 >> 7;
+  w.n0 = CAUSAL ? min(tiles, qt0 + 1) : tiles;
+  w.n1 = (w.q0 + 128 < n) ? (CAUSAL ? min(tiles, qt0 + 2) : tiles) : 0;
+  return w;
+}
+
+struct WaitCtx {
+  volatile int *abort;
+  uint32_t *status;
+  unsigned long long timeout_ns;
+};
+
+// Bounded wait for the phase of `bar` with parity `parity`.  Returns false
+// (after flagging the CTA and the device status word) when the time limit
+// runs out, or when another thread of the CTA already gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          const WaitCtx &wc, uint32_t role) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*wc.abort) return false;
+    if (global_timer_ns() - t0 > wc.timeout_ns) {
+      *wc.abort = 1;
+      atomicOr(wc.status, kStatusTimeout | role);
+      return false;
+    }
+  }
+}
+
+// Bounded wait used while draining after an abort: ignores the abort flag.
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,
+                                                const WaitCtx &wc) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > wc.timeout_ns) {
+      atomicOr(wc.status, kStatusTimeout | kRoleDrain);
+      return;
+    }
+  }
+}
+
+// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version bits.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr,
+                                                    uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+  const uint32_t lo = ((addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+  const uint32_t hi = ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// ------------------------------------------------------------------ loader
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void producer_role(uint32_t base,
+                                              const CUtensorMap *tq,
+                                              const CUtensorMap *tk,
+                                              const CUtensorMap *tv,
+                                              const FwdParams &p,
+                                              const WaitCtx &wc) {
+  using L = Smem<D>;
+  auto bar = [&](int i) { return base + L::kBars + 8u * i; };
+  int qocc[2] = {0, 0};     // non-empty occurrences of each Q tile so far
+  int q_issued[2] = {0, 0};
+  int k_issued = 0, v_issued = 0;
+  bool skip_first_q = (p.debug_flags & 1u) && blockIdx.x == 0;
+  bool ok = true;
+  const uint64_t pol_kv = policy_evict_last();
+  const uint64_t pol_q = policy_evict_first();
+
+  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
+    const int nt[2] = {w.n0, w.n1};
+    for (int t = 0; t < 2; ++t) {
+      if (nt[t] == 0) continue;
+      if (qocc[t] > 0) {
+        ok = mbar_wait(bar(L::Q_EMPTY + t), (qocc[t] - 1) & 1, wc, kRoleProducer);
+        if (!ok) break;
+      }
+      ++qocc[t];
+      if (skip_first_q && t == 0) {  // injected fault: this copy never happens
+        skip_first_q = false;
+        continue;
+      }
+      mbar_arrive_expect_tx(bar(L::Q_FULL + t), L::kTileBytes);
+      for (int s = 0; s < L::kSub; ++s)
+        tma_load_3d_hint(base + L::kQ + t * L::kTileBytes + s * L::kPanelBytes,
+                         tq, bar(L::Q_FULL + t), s * 64, w.q0 + kBlockM * t,
+                         w.bh, pol_q);
+      ++q_issued[t];
+    }
+    if (!ok) break;
+    const int nmax = max(nt[0], nt[1]);
+    for (int j = 0; j < nmax; ++j) {
+      const int st = k_issued % L::kStages;
+      const uint32_t ph = (k_issued / L::kStages) & 1;
+      ok = mbar_wait(bar(L::K_EMPTY + st), ph ^ 1, wc, kRoleProducer);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bar(L::K_FULL + st), L::kTileBytes);
+      for (int s = 0; s < L::kSub; ++s)
+        tma_load_3d_hint(base + L::kK + st * L::kTileBytes + s * L::kPanelBytes,
+                         tk, bar(L::K_FULL + st), s * 64, j * kBlockN, w.bh,
+                         pol_kv);
+      ++k_issued;
+      ok = mbar_wait(bar(L::V_EMPTY + st), ph ^ 1, wc, kRoleProducer);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bar(L::V_FULL + st), L::kTileBytes);
+      for (int s = 0; s < L::kSub; ++s)
+        tma_load_3d_hint(base + L::kV + st * L::kTileBytes + s * L::kPanelBytes,
+                         tv, bar(L::V_FULL + st), s * 64, j * kBlockN, w.bh,
+                         pol_kv);
+      ++v_issued;
+    }
+  }
+
+  if (*wc.abort) {
+    // Every copy issued must land before the CTA may exit.
+    for (int t = 0; t < 2; ++t)
+      if (q_issued[t] > 0)
+        mbar_wait_drain(bar(L::Q_FULL + t), (q_issued[t] - 1) & 1, wc);
+    for (int st = 0; st < L::kStages; ++st) {
+      if (k_issued > st) {
+        const int last = st + ((k_issued - 1 - st) / L::kStages) * L::kStages;
+        mbar_wait_drain(bar(L::K_FULL + st), (last / L::kStages) & 1, wc);
+      }
+      if (v_issued > st) {
+        const int last = st + ((v_issued - 1 - st) / L::kStages) * L::kStages;
+        mbar_wait_drain(bar(L::V_FULL + st), (last / L::kStages) & 1, wc);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ MMA
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem,
+                                         uint32_t k_smem) {
+  // S[128 x 128] = Q[128 x D] K[128 x D]^T; both K-major, 128B swizzle.
+  constexpr uint32_t idesc = (1u << 4)              // D: f32
+                             | (1u << 7)            // A: bf16
+                             | (1u << 10)           // B: bf16
+                             | ((uint32_t)(kBlockN >> 3) << 17)  // N
+                             | ((uint32_t)(kBlockM >> 4) << 24); // M
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * Smem<D>::kPanelBytes + (kk & 3) * 32;
+    mma_bf16_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024),
+                smem_desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
+                                         uint32_t v_smem, bool accumulate) {
+  // O[128 x D] (+)= P[128 x 128] V[128 x D]; P in TMEM (K-major, bf16
+  // packed two per column), V MN-major (D contiguous) with 128B swizzle:
+  // 64-wide D panels are kPanelBytes apart (LBO), 8-key groups 1024 B (SBO).
+  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10)
+                             | (1u << 16)           // B: MN-major
+                             | ((uint32_t)(D >> 3) << 17)
+                             | ((uint32_t)(kBlockM >> 4) << 24);
+#pragma unroll
+  for (int kk = 0; kk < kBlockN / 16; ++kk) {
+    mma_bf16_ts(d_tmem, p_tmem + kk * 8,
+                smem_desc_sw128(v_smem + kk * 2048, Smem<D>::kPanelBytes, 1024),
+                idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
+                                         const FwdParams &p, const WaitCtx &wc) {
+  using L = Smem<D>;
+  auto bar = [&](int i) { return base + L::kBars + 8u * i; };
+  const uint32_t tS[2] = {tmem + 0, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+  const uint32_t sQ[2] = {base + L::kQ, base + L::kQ + L::kTileBytes};
+  int qocc[2] = {0, 0}, pcnt[2] = {0, 0}, oocc[2] = {0, 0};
+  int kcons = 0, vcons = 0;
+  bool ok = true;
+
+  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
+    const int nt[2] = {w.n0, w.n1};
+    const int nmax = max(nt[0], nt[1]);
+    for (int t = 0; t < 2 && ok; ++t)
+      if (nt[t] > 0) {
+        ok = mbar_wait(bar(L::Q_FULL + t), qocc[t] & 1, wc, kRoleMma);
+        ++qocc[t];
+      }
+    if (!ok) break;
+    {  // S_0 for both tiles
+      const int ks = kcons % L::kStages;
+      ok = mbar_wait(bar(L::K_FULL + ks), (kcons / L::kStages) & 1, wc, kRoleMma);
+      if (!ok) break;
+      tc_fence_after_sync();
+      for (int t = 0; t < 2; ++t)
+        if (nt[t] > 0) {
+          issue_qk<D>(tS[t], sQ[t], base + L::kK + ks * L::kTileBytes);
+          mma_commit(bar(L::S_FULL + t));
+          if (nt[t] == 1) mma_commit(bar(L::Q_EMPTY + t));  // last read of Q_t
+        }
+      mma_commit(bar(L::K_EMPTY + ks));
+      ++kcons;
+    }
+    for (int j = 0; j < nmax && ok; ++j) {
+      const int vs = vcons % L::kStages;
+      ok = mbar_wait(bar(L::V_FULL + vs), (vcons / L::kStages) & 1, wc, kRoleMma);
+      if (!ok) break;
+      const int ks = kcons % L::kStages;
+      bool k_next = false;
+      for (int t = 0; t < 2; ++t) {
+        if (j >= nt[t]) continue;
+        ok = mbar_wait(bar(L::P_FULL + t), pcnt[t] & 1, wc, kRoleMma);
+        ++pcnt[t];
+        if (!ok) break;
+        if (j == 0 && oocc[t] > 0) {
+          // previous unit's epilogue must have read O out of TMEM
+          ok = mbar_wait(bar(L::O_EMPTY + t), (oocc[t] - 1) & 1, wc, kRoleMma);
+          if (!ok) break;
+        }
+        tc_fence_after_sync();
+        issue_pv<D>(tO[t], tS[t], base + L::kV + vs * L::kTileBytes, j > 0);
+        mma_commit(bar(L::O_FULL + t));
+        if (j + 1 < nt[t]) {
+          if (!k_next) {
+            ok = mbar_wait(bar(L::K_FULL + ks), (kcons / L::kStages) & 1, wc,
+                           kRoleMma);
+            if (!ok) break;
+            tc_fence_after_sync();
+            k_next = true;
+          }
+          // issued after this tile's P.V in the same thread: the tensor pipe
+          // reads P before this MMA overwrites the S columns holding it
+          issue_qk<D>(tS[t], sQ[t], base + L::kK + ks * L::kTileBytes);
+          mma_commit(bar(L::S_FULL + t));
+          if (j + 2 == nt[t]) mma_commit(bar(L::Q_EMPTY + t));  // last read of Q_t
+        }
+      }
+      if (!ok) break;
+      mma_commit(bar(L::V_EMPTY + vs));
+      ++vcons;
+      if (k_next) {
+        mma_commit(bar(L::K_EMPTY + ks));
+        ++kcons;
+      }
+    }
+    for (int t = 0; t < 2; ++t)
+      if (nt[t] > 0) ++oocc[t];
+  }
+  // All tensor-core work must finish before TMEM is released.
+  mma_commit(bar(L::DRAIN));
+  mbar_wait_drain(bar(L::DRAIN), 0, wc);
+}
+
+// ------------------------------------------------------------------ softmax
+
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld_32x32b_x32(tO + c * 32, o);
+    tmem_wait_ld(o);
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+    tmem_st_32x32b_x32(tO + c * 32, o);
+  }
+}
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
+                                             const FwdParams &p,
+                                             const WaitCtx &wc, int warp,
+                                             int lane) {
+  using L = Smem<D>;
+  auto bar = [&](int i) { return base + L::kBars + 8u * i; };
+  const int t = warp >> 2;          // which Q tile of the unit
+  const int wq = warp & 3;          // TMEM lane quarter of this warp
+  const int r = wq * 32 + lane;     // query row within the tile
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const uint32_t tS = lane_base + t * 128;
+  const uint32_t tO = lane_base + 256 + t * D;
+  const float cl2 = p.c_log2;
+  int scnt = 0, ocnt = 0;
+  bool ok = true;
+
+  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
+    const int n = t ? w.n1 : w.n0;
+    if (n == 0) continue;
+    const int qs = w.q0 + kBlockM * t;
+    float m_run = -CUDART_INF_F;  // running max, log2 units (x = s * scale * log2 e)
+    float l_run = 0.f;            // running sum of exp2(x - m_run)
+
+    for (int j = 0; j < n; ++j) {
+      ok = mbar_wait(bar(L::S_FULL + t), scnt & 1, wc, kRoleSoftmax);
+      ++scnt;
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after_sync();
+
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+      tmem_wait_ld(s[0]);
+      reg_fence(s[1]);
+      reg_fence(s[2]);
+      reg_fence(s[3]);
+
+      if (j == n - 1 && (CAUSAL || (p.n & (kBlockN - 1)))) {
+        // diagonal tile (causal: key c visible iff c <= row) or ragged tail
+        // (keys at or beyond N do not exist)
+        const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > limit) s[c >> 5][c & 31] = __float_as_uint(-CUDART_INF_F);
+      }
+
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[0][i]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c)
+        mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c >> 5][c & 31]));
+      const float m_tile =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * cl2;
+
+      // Lazy max update (warp-uniform decision, per-row values).
+      const bool update =
+          __any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold);
+      float alpha = 1.f;
+      if (update) {
+        const float m_new = fmaxf(m_run, m_tile);
+        alpha = ex2_approx(m_run - m_new);  // 0 on the first tile (m_run = -inf)
+        l_run *= alpha;
+        m_run = m_new;
+      }
+
+      const float neg_m = -m_run;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float x0 = __uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]);
+        const float x1 = __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
+        const float p0 = ex2_approx(fmaf(x0, cl2, neg_m));
+        const float p1 = ex2_approx(fmaf(x1, cl2, neg_m));
+        ls[c & 3] += p0 + p1;
+        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+      }
+      tmem_st_32x32b_x32(tS + 0, pk[0]);
+      tmem_st_32x32b_x32(tS + 32, pk[1]);
+      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // O holds the earlier P.V products; the S_FULL commit for this tile was
+      // issued after the previous P.V, so that MMA has completed.
+      if (update && j > 0) rescale_o<D>(tO, alpha);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::P_FULL + t));
+    }
+    if (!ok) break;
+
+    // ---- epilogue: O / l -> bf16 -> this row of O in HBM; lse
+    ocnt += n;
+    ok = mbar_wait(bar(L::O_FULL + t), (ocnt - 1) & 1, wc, kRoleEpilogue);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    tc_fence_after_sync();
+    const float inv_l = __frcp_rn(l_run);
+    const bool row_ok = qs + r < p.n;
+    uint4 *orow = reinterpret_cast<uint4 *>(
+        p.o + (static_cast<int64_t>(w.bh) * p.n + qs + r) * D);
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld_32x32b_x32(tO + c * 32, o);
+      tmem_wait_ld(o);
+      uint32_t h[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                           __uint_as_float(o[2 * i + 1]) * inv_l);
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          orow[c * 4 + i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2],
+                                       h[4 * i + 3]);
+      }
+    }
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::O_EMPTY + t));  // O columns reusable
+    if (row_ok)
+      p.lse[static_cast<int64_t>(w.bh) * p.n + qs + r] =
+          (m_run + lg2_approx(l_run)) * kLn2;
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const FwdParams p) {
+  using L = Smem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    const uint32_t b0 = base + L::kBars;
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(b0 + 8 * (L::Q_FULL + t), 1);
+      mbar_init(b0 + 8 * (L::Q_EMPTY + t), 1);
+      mbar_init(b0 + 8 * (L::S_FULL + t), 1);
+      mbar_init(b0 + 8 * (L::P_FULL + t), 4);
+      mbar_init(b0 + 8 * (L::O_FULL + t), 1);
+      mbar_init(b0 + 8 * (L::O_EMPTY + t), 4);
+    }
+    mbar_init(b0 + 8 * L::DRAIN, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(b0 + 8 * (L::K_FULL + s), 1);
+      mbar_init(b0 + 8 * (L::K_EMPTY + s), 1);
+      mbar_init(b0 + 8 * (L::V_FULL + s), 1);
+      mbar_init(b0 + 8 * (L::V_EMPTY + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+
+  if (warp < 8) {
+    softmax_role<D, CAUSAL>(base, tmem, p, wc, warp, lane);
+  } else if (warp == kProducerWarp) {
+    if (lane == 0) producer_role<D, CAUSAL>(base, &tm_q, &tm_k, &tm_v, p, wc);
+    __syncwarp();
+  } else {
+    if (lane == 0) mma_role<D, CAUSAL>(base, tmem, p, wc);
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace attn_b200

@@ -1,0 +1,167 @@
+/*
+ * attn_b200.h -- C ABI of the B200 (sm_100a) exact attention forward pass.
+ *
+ * Operation (marketmaker.cc post "Apakah Konteks Sehari Penuh Mengalahkan
+ * Konteks Sepuluh Menit? Perhatian Kilat dan Pertanyaan Panjang Urutan",
+ * sections "Mengapa perhatian terikat pada memori" and "Algoritma Flash
+ * Attention"; causal mask as in "Causal masking adalah tempat perdagangan
+ * mendapat diskon" and "Integrasinya delapan baris"):
+ *
+ *   for every batch b < B and head h < H, with S = scale * Q K^T (N x N):
+ *     S[i][j] = -inf when causal != 0 and j > i   (key j in query i's future)
+ *     O   = softmax_rows(S) V                     (bf16 output, fp32 math)
+ *     lse[i] = ln( sum_j exp(S[i][j]) )           (fp32; the saved softmax
+ *                                                  statistics (m, l) of the
+ *                                                  section "Backward pass",
+ *                                                  folded into m + ln l)
+ *
+ * S is never written to memory: the kernel walks key/value tiles with the
+ * online-softmax recurrence ("Pengulangan softmax online"), which is exact
+ * up to rounding.
+ *
+ * Layouts.  q, k, v, o: contiguous row-major bf16 [B, H, N, d] (d innermost,
+ * then the sequence, then heads, then batch) -- the (batch, heads, seq,
+ * head_dim) layout of the post's SDPA call.  lse: contiguous fp32 [B, H, N].
+ * Q and K/V have the same sequence length N (self-attention).
+ *
+ * Ownership.  The caller allocates and owns every buffer.  attn_fwd does not
+ * allocate per call; the first call on a device allocates one 4-byte device
+ * status word for that device, kept until process exit (so make the first
+ * call outside any CUDA-graph capture).  o and lse must not overlap q, k, v
+ * or each other.
+ *
+ * Concurrency.  Calls are asynchronous on `stream` (no host synchronisation).
+ * Concurrent calls on different streams are safe; they share the device
+ * status word, so a timeout reported by attn_status may belong to any of
+ * them.
+ *
+ * Errors.  Every function returns 0 (ATTN_OK) or a positive code below.
+ * Argument errors are detected before any CUDA call, so nothing is launched
+ * and the CUDA context is untouched.  Device-side failures (a pipeline wait
+ * that exceeded its time limit) are reported later by attn_status.
+ */
+#ifndef ATTN_B200_H_
+#define ATTN_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (cudaStream_t / CUstream); NULL = legacy
+ * default stream. */
+typedef struct CUstream_st *attn_stream_t;
+
+enum {
+  ATTN_OK = 0,
+  ATTN_ERR_NULL_POINTER = 1,     /* a required pointer is NULL */
+  ATTN_ERR_INVALID_SIZE = 2,     /* B, H or N negative or beyond the limits */
+  ATTN_ERR_UNSUPPORTED_HEAD_DIM = 3, /* d is not 64 or 128 */
+  ATTN_ERR_MISALIGNED = 4,       /* q/k/v/o not 16-byte or lse not 4-byte aligned */
+  ATTN_ERR_INVALID_SCALE = 5,    /* scale not finite or not > 0 */
+  ATTN_ERR_ALIAS = 6,            /* o or lse overlaps an input or each other */
+  ATTN_ERR_UNSUPPORTED_DEVICE = 7, /* no CUDA device, or not compute 10.0 (B200) */
+  ATTN_ERR_CUDA = 8,             /* a CUDA runtime call or the launch failed */
+  ATTN_ERR_TENSOR_MAP = 9,       /* TMA descriptor encoding failed */
+  ATTN_ERR_NOT_DEVICE_MEMORY = 10, /* q/k/v/o/lse not device memory of the
+                                      current device */
+  ATTN_ERR_WORKSPACE = 11,       /* attn_fwd_host workspace NULL or too small */
+  ATTN_ERR_DEVICE_TIMEOUT = 16   /* (attn_status) a pipeline wait in the
+                                    kernel ran past its time limit; the kernel
+                                    stopped early and its outputs are invalid */
+};
+
+/* Size limits (inclusive).  N <= ATTN_MAX_SEQ; B * H <= ATTN_MAX_HEADS. */
+#define ATTN_MAX_SEQ (1 << 24)
+#define ATTN_MAX_HEADS (1 << 24)
+
+/*
+ * attn_fwd -- exact attention forward on device buffers.
+ *
+ *   q, k, v  device pointers, bf16 [B, H, N, d], 16-byte aligned.
+ *   o        device pointer, bf16 [B, H, N, d], 16-byte aligned (output).
+ *   lse      device pointer, fp32 [B, H, N], 4-byte aligned (output): natural
+ *            log of each row's softmax denominator over the scaled, masked
+ *            scores.
+ *   B, H, N  batch, heads, sequence length; any of them 0 is a valid empty
+ *            problem (nothing is launched, ATTN_OK).
+ *   d        head dimension: 64 or 128.
+ *   causal   nonzero: key j is hidden from query i when j > i (the diagonal
+ *            stays visible, so no row is ever fully masked).
+ *   scale    multiplier of Q K^T, finite and > 0 (1/sqrt(d) for the usual
+ *            attention).
+ *   stream   CUDA stream the work is queued on.
+ *
+ * The current CUDA device must be a B200 (compute capability 10.0) and all
+ * pointers must be its device memory.  Returns ATTN_OK once the kernel is
+ * queued; runtime timeouts surface through attn_status.
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int H, int N, int d, int causal, float scale,
+             attn_stream_t stream);
+
+/*
+ * attn_fwd_host -- the same operation on HOST buffers, end to end.
+ *
+ * Queues on `stream`: copies of q, k, v from the host into `workspace`, the
+ * attn_fwd kernel on the workspace copies, and copies of o and lse back into
+ * the host buffers.  Returns once queued; the host outputs are valid after
+ * the stream is synchronised.  For asynchronous copies the host buffers must
+ * be page-locked (cudaHostAlloc / pinned); pageable buffers work but the
+ * copies then block the calling thread.
+ *
+ *   workspace        device memory of at least attn_fwd_host_workspace_bytes
+ *                    (B, H, N, d) bytes, 256-byte aligned, caller-owned.
+ *   workspace_bytes  its size.
+ * Other arguments as attn_fwd; q, k, v, o, lse are host pointers here.
+ */
+int attn_fwd_host(const void *q, const void *k, const void *v, void *o,
+                  float *lse, int B, int H, int N, int d, int causal,
+                  float scale, void *workspace, size_t workspace_bytes,
+                  attn_stream_t stream);
+
+/* Workspace bytes attn_fwd_host needs for this problem (0 on bad sizes):
+ * q, k, v, o (each B*H*N*d*2 bytes) and lse (B*H*N*4 bytes), each rounded up
+ * to 256 bytes. */
+size_t attn_fwd_host_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * attn_status -- synchronise `stream`, then read and clear the current
+ * device's status word.  Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT when a
+ * kernel launched since the last call stopped on a wait time limit, or
+ * ATTN_ERR_CUDA when the synchronisation itself failed.
+ */
+int attn_status(attn_stream_t stream);
+
+/* Raw status bits of the last attn_status that reported a device error
+ * (which pipeline role gave up), for diagnostics; 0 when none. */
+uint32_t attn_last_status_bits(void);
+
+/* Human-readable text for an error code (static string, never NULL). */
+const char *attn_strerror(int code);
+
+/*
+ * attn_set_wait_timeout_ns -- time limit of every pipeline wait inside the
+ * kernel, for launches made after the call (process-wide).  0 restores the
+ * default of 1e9 ns (one second).  A wait that runs out sets the device
+ * status word, and the kernel drains its in-flight copies, frees its tensor
+ * memory and exits.
+ */
+void attn_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * attn_set_fault_injection -- test hook.  flags = 1: in later launches the
+ * first CTA's loader never issues its first Q-tile copy, so the MMA warp's
+ * wait on it runs out after the wait time limit and the launch ends with
+ * ATTN_ERR_DEVICE_TIMEOUT in attn_status.  flags = 0 (the default) turns it
+ * off.  No other value is defined.
+ */
+void attn_set_fault_injection(uint32_t flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H_ */

@@ -1,0 +1,136 @@
+"""The C-ABI library on the CPU: it loads, exports every function the header
+declares, and rejects bad arguments before touching CUDA (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def attn():
+    from exact_io_aware_73_b200 import build
+    build.build()
+    from exact_io_aware_73_b200 import attn as a
+    return a
+
+
+def _declared_functions():
+    names = set()
+    for f in os.listdir(HEADER_DIR):
+        if not f.endswith(".h"):
+            continue
+        src = open(os.path.join(HEADER_DIR, f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", src,
+                             flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for required in ("attn_fwd", "attn_fwd_host", "attn_status",
+                     "attn_strerror", "attn_fwd_host_workspace_bytes"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(attn):
+    lib = attn.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", attn.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name), name
+
+
+def test_build_targets_sm100a_only():
+    from exact_io_aware_73_b200 import build
+    f = build.flags()
+    gencodes = [f[i + 1] for i, x in enumerate(f) if x == "-gencode"]
+    assert gencodes == ["arch=compute_100a,code=sm_100a"]
+
+
+def _call(attn, q=8, k=8, v=8, o=8, lse=8, B=1, H=1, N=16, d=64, causal=0,
+          scale=0.125):
+    # fake (non-null) pointers: every one of these cases must be refused
+    # before any CUDA call, so nothing is ever dereferenced
+    return attn.attn_fwd_raw(q, k, v, o, lse, B, H, N, d, causal, scale, None)
+
+
+def test_argument_errors_need_no_device(attn):
+    far = 1 << 40
+    assert _call(attn, q=None) == 1
+    assert _call(attn, lse=None) == 1
+    assert _call(attn, B=-1) == 2
+    assert _call(attn, N=(1 << 24) + 1, q=far, k=2 * far, v=3 * far,
+                 o=4 * far, lse=5 * far) == 2
+    assert _call(attn, d=96) == 3
+    assert _call(attn, d=256) == 3
+    assert _call(attn, q=far + 8, k=2 * far, v=3 * far, o=4 * far,
+                 lse=5 * far) == 4
+    assert _call(attn, q=far, k=2 * far, v=3 * far, o=4 * far,
+                 lse=5 * far + 2) == 4
+    assert _call(attn, scale=0.0) == 5
+    assert _call(attn, scale=float("nan")) == 5
+    assert _call(attn, scale=float("inf")) == 5
+    assert _call(attn, scale=-0.5) == 5
+    # o overlapping q
+    assert _call(attn, q=far, k=2 * far, v=3 * far, o=far + 1024,
+                 lse=5 * far) == 6
+    # lse overlapping o
+    assert _call(attn, q=far, k=2 * far, v=3 * far, o=4 * far,
+                 lse=4 * far + 64) == 6
+
+
+def test_empty_problem_is_a_no_op(attn):
+    for B, H, N in ((0, 1, 16), (1, 0, 16), (1, 1, 0)):
+        assert _call(attn, q=None, k=None, v=None, o=None, lse=None, B=B, H=H,
+                     N=N) == 0
+
+
+def test_no_device_is_reported_not_crashed(attn):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    far = 1 << 40
+    assert _call(attn, q=far, k=2 * far, v=3 * far, o=4 * far,
+                 lse=5 * far) == 7
+
+
+def test_host_entry_workspace_checks(attn):
+    assert attn.host_workspace_bytes(2, 3, 100, 64) == \
+        4 * ((2 * 3 * 100 * 64 * 2 + 255) // 256 * 256) + \
+        (2 * 3 * 100 * 4 + 255) // 256 * 256
+    assert attn.host_workspace_bytes(1, 1, 16, 96) == 0
+    lib = attn.lib()
+    buf = ctypes.create_string_buffer(1 << 16)
+    p = ctypes.addressof(buf)
+    # workspace missing / too small are refused before any CUDA call
+    rc = lib.attn_fwd_host(p, p + 4096, p + 8192, p + 12288, p + 16384, 1, 1,
+                           16, 64, 0, 0.125, None, 0, None)
+    assert rc == 11
+    rc = lib.attn_fwd_host(p, p + 4096, p + 8192, p + 12288, p + 16384, 1, 1,
+                           16, 64, 0, 0.125, 1 << 40, 16, None)
+    assert rc == 11
+
+
+def test_strerror_covers_every_code(attn):
+    for code in list(attn.ERROR_NAMES) + [0]:
+        text = attn.strerror(code)
+        assert text and text != "unknown error code"
+    assert attn.strerror(12345) == "unknown error code"
+
+
+def test_python_binding_has_no_fallback(tmp_path, monkeypatch):
+    """With the library missing, the binding raises instead of computing."""
+    from exact_io_aware_73_b200 import attn as a
+    monkeypatch.setattr(a, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(a, "_lib", None)
+    with pytest.raises(ImportError):
+        a.lib()
