@@ -43,9 +43,14 @@ KERNEL_NAME = "attn_fwd_sm100_kernel"
 CSRC = os.path.join(ROOT, "exact_io_aware_73_b200", "csrc")
 
 
+KERNEL_SOURCES = ("attn_fwd_kernel.cuh", "ptx_sm100.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the device-code sources; a committed traffic figure is only
+    used while it matches (the counters describe that exact kernel)."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
+    for f in KERNEL_SOURCES:
         with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]

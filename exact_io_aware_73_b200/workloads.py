@@ -63,6 +63,11 @@ WORKLOADS = {
     "long_b1h32n16384d128": Workload("long_b1h32n16384d128", 1, 32, 16384,
                                      128, False, q_std=2.0, k_std=2.0,
                                      seed=1005),
+    # profiling case: the headline's per-head shape with half the heads
+    # (Q/K/V still 201 MB, above the 126 MB L2), for full counter captures
+    "prof_b1h16n16384d128": Workload("prof_b1h16n16384d128", 1, 16, 16384,
+                                     128, False, q_std=2.0, k_std=2.0,
+                                     seed=1006),
 }
 
 # The non-causal N >= 4096, d = 128 case the throughput target is set on.
