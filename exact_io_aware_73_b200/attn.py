@@ -19,7 +19,8 @@ ERROR_NAMES = {
     5: "ATTN_ERR_INVALID_SCALE", 6: "ATTN_ERR_ALIAS",
     7: "ATTN_ERR_UNSUPPORTED_DEVICE", 8: "ATTN_ERR_CUDA",
     9: "ATTN_ERR_TENSOR_MAP", 10: "ATTN_ERR_NOT_DEVICE_MEMORY",
-    11: "ATTN_ERR_WORKSPACE", 16: "ATTN_ERR_DEVICE_TIMEOUT",
+    11: "ATTN_ERR_WORKSPACE", 12: "ATTN_ERR_NOALLOC_TOO_LARGE",
+    16: "ATTN_ERR_DEVICE_TIMEOUT",
 }
 
 _lib = None
@@ -149,3 +150,29 @@ def set_wait_timeout_ns(ns: int) -> None:
 
 def set_fault_injection(flags: int) -> None:
     lib().attn_set_fault_injection(int(flags))
+
+
+# Scratch size of attn_fwd_host_noalloc's static device array (bytes).
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def _noalloc_fn():
+    f = lib().attn_fwd_host_noalloc
+    if f.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        f.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, ctypes.c_float, vp]
+        f.restype = i
+    return f
+
+
+def attn_fwd_host_noalloc(q, k, v, out, lse, causal: bool, scale: float,
+                          stream=None):
+    """Host-buffer attention that allocates no device memory: its scratch is
+    a static 32 MiB device array inside the library, shared by every call on
+    the device (so overlapping calls race).  Synchronous: `out` and `lse` are
+    filled on return.  For callers without a device allocator of their own."""
+    B, H, N, d = q.shape
+    rc = _noalloc_fn()(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                       out.data_ptr(), lse.data_ptr(), B, H, N, d,
+                       int(bool(causal)), float(scale), _stream_handle(stream))
+    _check(rc, "attn_fwd_host_noalloc")

@@ -330,6 +330,7 @@ const char *attn_strerror(int code) {
     case ATTN_ERR_TENSOR_MAP: return "TMA tensor-map encoding failed";
     case ATTN_ERR_NOT_DEVICE_MEMORY: return "a buffer is not device memory of the current device";
     case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case ATTN_ERR_NOALLOC_TOO_LARGE: return "problem needs more device scratch than the static ATTN_NOALLOC_SCRATCH_BYTES array of attn_fwd_host_noalloc";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a pipeline wait in the kernel ran out of time; outputs are invalid";
     default: return "unknown error code";
   }
@@ -342,3 +343,139 @@ void attn_set_wait_timeout_ns(uint64_t ns) {
 void attn_set_fault_injection(uint32_t flags) { g_inject.store(flags & 1u); }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// attn_fwd_host_noalloc: the host-buffer path with its device scratch in a
+// static array instead of caller- or library-allocated memory.
+// ------------------------------------------------------------------------
+namespace {
+
+// [0, 256): device status word of these calls; [256, end): q | k | v | o |
+// lse staging, laid out as attn_fwd_host lays out its workspace.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+constexpr size_t kNoallocStatusBytes = 256;
+
+struct NoallocState {
+  bool ready = false;
+  uint8_t *base = nullptr;  // device address of g_noalloc_scratch
+};
+NoallocState g_noalloc[kMaxDevices];
+
+// Current device checked to be a B200, without touching the lazily
+// allocated status word of attn_fwd (so nothing is allocated here); looks up
+// the scratch array's device address once per device.
+int noalloc_device(int *dev_out, DeviceState **st_out, uint8_t **base_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return ATTN_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState &st = g_dev[dev];
+  if (!st.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_UNSUPPORTED_DEVICE;
+    }
+    st.probed = true;
+    st.supported = (major == 10 && minor == 0);
+    st.sm_count = sms;
+  }
+  if (!st.supported) return ATTN_ERR_UNSUPPORTED_DEVICE;
+  NoallocState &na = g_noalloc[dev];
+  if (!na.ready) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    na.base = static_cast<uint8_t *>(p);
+    na.ready = true;
+  }
+  *dev_out = dev;
+  *st_out = &st;
+  *base_out = na.base;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_fwd_host_noalloc(const void *q, const void *k,
+                                     const void *v, void *o, float *lse, int B,
+                                     int H, int N, int d, int causal,
+                                     float scale, attn_stream_t stream) {
+  int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, false);
+  if (rc != ATTN_OK || B == 0 || H == 0 || N == 0) return rc;
+  const size_t need = attn_fwd_host_workspace_bytes(B, H, N, d);
+  if (need > ATTN_NOALLOC_SCRATCH_BYTES - kNoallocStatusBytes)
+    return ATTN_ERR_NOALLOC_TOO_LARGE;
+
+  int dev;
+  DeviceState *st;
+  uint8_t *base;
+  if ((rc = noalloc_device(&dev, &st, &base)) != ATTN_OK) return rc;
+  uint32_t *status = reinterpret_cast<uint32_t *>(base);
+  uint8_t *ws = base + kNoallocStatusBytes;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  const size_t tb = rows * d * 2, tbr = round256(tb);
+  void *dq = ws, *dk = ws + tbr, *dv = ws + 2 * tbr, *dout = ws + 3 * tbr;
+  float *dl = reinterpret_cast<float *>(ws + 4 * tbr);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  // The array keeps the previous call's contents: the status word must
+  // start at zero; the staging area is fully overwritten below.
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess ||
+      cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  EncodeTiledFn enc;
+  if ((rc = get_encode_fn(&enc)) != ATTN_OK) return rc;
+  const int bh = B * H;
+  CUtensorMap maps[3];
+  if ((rc = encode_map(enc, &maps[0], dq, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[1], dk, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[2], dv, bh, N, d)) != ATTN_OK) return rc;
+  FwdParams p;
+  p.o = static_cast<uint16_t *>(dout);
+  p.lse = dl;
+  p.status = status;
+  p.bh = bh;
+  p.n = N;
+  p.num_units = bh * ((N + 255) / 256);
+  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.timeout_ns = g_timeout_ns.load();
+  p.debug_flags = g_inject.load();
+  if (d == 128)
+    rc = causal ? launch<128, true>(*st, 0, maps, p, s)
+                : launch<128, false>(*st, 1, maps, p, s);
+  else
+    rc = causal ? launch<64, true>(*st, 2, maps, p, s)
+                : launch<64, false>(*st, 3, maps, p, s);
+  if (rc != ATTN_OK) return rc;
+  uint32_t bits = 0;
+  if (cudaMemcpyAsync(o, dout, tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(lse, dl, rows * 4, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(&bits, status, sizeof bits, cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  if (bits != 0) {
+    g_last_bits.store(bits);
+    return (bits & attn_b200::kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT
+                                              : ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}

@@ -68,6 +68,8 @@ enum {
   ATTN_ERR_NOT_DEVICE_MEMORY = 10, /* q/k/v/o/lse not device memory of the
                                       current device */
   ATTN_ERR_WORKSPACE = 11,       /* attn_fwd_host workspace NULL or too small */
+  ATTN_ERR_NOALLOC_TOO_LARGE = 12, /* attn_fwd_host_noalloc: problem needs more
+                                      than ATTN_NOALLOC_SCRATCH_BYTES */
   ATTN_ERR_DEVICE_TIMEOUT = 16   /* (attn_status) a pipeline wait in the
                                     kernel ran past its time limit; the kernel
                                     stopped early and its outputs are invalid */
@@ -138,6 +140,49 @@ int attn_status(attn_stream_t stream);
 /* Raw status bits of the last attn_status that reported a device error
  * (which pipeline role gave up), for diagnostics; 0 when none. */
 uint32_t attn_last_status_bits(void);
+
+/* Size of the static device scratch array behind attn_fwd_host_noalloc:
+ * 256 bytes of status followed by the q, k, v, o, lse staging area. */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * attn_fwd_host_noalloc -- attn_fwd_host for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is a deployment
+ * variant of the host-buffer entry point.
+ *
+ * Who needs it: a host program that holds only host buffers and has no
+ * device allocator of its own -- or runs in a process whose device memory
+ * belongs to another allocator that must not see untracked cudaMalloc
+ * calls, or cannot afford the device-wide synchronisation cudaMalloc and
+ * cudaFree may imply.  It allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.  Its device scratch is one static array of
+ * ATTN_NOALLOC_SCRATCH_BYTES (32 MiB) compiled into this library; every GPU
+ * that loads the library holds that array until the process exits.
+ *
+ * Arguments as attn_fwd_host (q, k, v, o, lse are host pointers; pinned
+ * memory makes the copies asynchronous) minus the workspace.  The call
+ * queues the copies in, the kernel and the copies out on `stream`, then
+ * synchronises `stream` and returns: the outputs are in o and lse on return,
+ * and the return value already includes the kernel's device status
+ * (ATTN_ERR_DEVICE_TIMEOUT if a pipeline wait ran out), so attn_status is
+ * not needed for it.
+ *
+ * Limits: attn_fwd_host_workspace_bytes(B, H, N, d) must not exceed
+ * ATTN_NOALLOC_SCRATCH_BYTES - 256, else ATTN_ERR_NOALLOC_TOO_LARGE is
+ * returned and nothing is queued (for d = 64, B*H*N up to about 65,000 rows;
+ * for d = 128, about 32,700).
+ *
+ * Set-up: the first call on each device looks up the device address of the
+ * scratch array (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  Sharing: every call on a device
+ * uses the same array, which keeps the last call's contents (the status
+ * word is cleared at the start of every call).  Calls that overlap on the
+ * GPU -- from different host threads or on different streams -- race on the
+ * array and corrupt each other's results; serialise them.
+ */
+int attn_fwd_host_noalloc(const void *q, const void *k, const void *v,
+                          void *o, float *lse, int B, int H, int N, int d,
+                          int causal, float scale, attn_stream_t stream);
 
 /* Human-readable text for an error code (static string, never NULL). */
 const char *attn_strerror(int code);
