@@ -176,3 +176,19 @@ def attn_fwd_host_noalloc(q, k, v, out, lse, causal: bool, scale: float,
                        out.data_ptr(), lse.data_ptr(), B, H, N, d,
                        int(bool(causal)), float(scale), _stream_handle(stream))
     _check(rc, "attn_fwd_host_noalloc")
+
+
+def selftest_exp2(x, mode: int, stream=None):
+    """y = 2^x for a float32 CUDA tensor, evaluated as the kernel does:
+    mode 0 = FMA-pipe polynomial, mode 1 = ex2.approx (test hook)."""
+    import torch
+    f = lib().attn_selftest_exp2
+    if f.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        f.argtypes = [vp, vp, i, i, vp]
+        f.restype = i
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check(f(x.data_ptr(), y.data_ptr(), x.numel(), int(mode),
+             _stream_handle(stream)), "attn_selftest_exp2")
+    return y

@@ -194,6 +194,21 @@ int launch(DeviceState &st, int variant, const CUtensorMap *maps,
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+__global__ void exp2_selftest_kernel(const float *x, float *y, int n, int mode) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+  float y0, y1;
+  if (mode == 0) {
+    attn_b200::f32x2_split(attn_b200::exp2_poly_x2(x0, x1), y0, y1);
+  } else {
+    y0 = attn_b200::ex2_approx(x0);
+    y1 = attn_b200::ex2_approx(x1);
+  }
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -315,6 +330,19 @@ int attn_status(attn_stream_t stream) {
 }
 
 uint32_t attn_last_status_bits(void) { return g_last_bits.load(); }
+
+int attn_selftest_exp2(const float *x, float *y, int n, int mode,
+                       attn_stream_t stream) {
+  if (n < 0) return ATTN_ERR_INVALID_SIZE;
+  if (mode != 0 && mode != 1) return ATTN_ERR_INVALID_SCALE;
+  if (n == 0) return ATTN_OK;
+  if (!x || !y) return ATTN_ERR_NULL_POINTER;
+  const int pairs = (n + 1) / 2;
+  exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0,
+                         reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
 
 const char *attn_strerror(int code) {
   switch (code) {

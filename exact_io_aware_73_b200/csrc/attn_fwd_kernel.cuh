@@ -58,9 +58,20 @@ namespace attn_b200 {
 
 constexpr int kBlockM = 128;   // query rows per Q tile (= TMEM lanes)
 constexpr int kBlockN = 128;   // keys per K/V tile
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 384;  // 12 warps = 3 warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kVLoaderWarp = 10;  // warp 11 only completes warpgroup 2
+// Register split.  With 12 warps every thread is launched with 168
+// registers (an SM sub-partition holds 3 warps of the CTA); warpgroup 2 (the
+// loader / MMA / idle warps) hands registers back and the two softmax
+// warpgroups take them, so a softmax thread holds its whole score row with
+// room for the compiler to keep many exponentials in flight.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kControlRegs = 104;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P <= 2^8
 constexpr float kLn2 = 0.6931471805599453f;
@@ -72,6 +83,49 @@ constexpr uint32_t kRoleMma = 1u << 9;
 constexpr uint32_t kRoleSoftmax = 1u << 10;
 constexpr uint32_t kRoleEpilogue = 1u << 11;
 constexpr uint32_t kRoleDrain = 1u << 12;
+
+// Pairs of exponentials (out of every 8 pairs of a score row) evaluated on the
+// FMA pipe by exp2_poly_x2 instead of the MUFU unit; the rest use ex2.approx.
+// At d = 64 the MUFU carries twice the exponentials per tensor-core FLOP of
+// d = 128 and is the binding unit, so a quarter of them move to the FMA pipe;
+// at d = 128 measurement favoured the MUFU alone.
+#ifndef ATTN_EXP2_EMU_PER8
+#define ATTN_EXP2_EMU_PER8_D64 2
+#define ATTN_EXP2_EMU_PER8_D128 0
+#else
+#define ATTN_EXP2_EMU_PER8_D64 ATTN_EXP2_EMU_PER8
+#define ATTN_EXP2_EMU_PER8_D128 ATTN_EXP2_EMU_PER8
+#endif
+template <int D>
+constexpr int kEmuPer8 = (D == 128) ? ATTN_EXP2_EMU_PER8_D128 : ATTN_EXP2_EMU_PER8_D64;
+static_assert(kEmuPer8<64> >= 0 && kEmuPer8<64> <= 8 && kEmuPer8<128> >= 0 &&
+                  kEmuPer8<128> <= 8,
+              "pairs out of 8");
+
+// 2^x for two values at once on the FMA / integer pipes (x <= 8 here).
+// Cody-Waite split x = n + f, n = round-to-nearest(x) obtained by adding
+// 1.5 * 2^23 (n then sits in the low mantissa bits), f = x - n in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial with minimax relative error 7.5e-5, fitted by
+// csrc/gen_exp2_poly.py (Remez exchange); 2^n by adding n to the exponent
+// field.  x is clamped at -125 so the exponent cannot underflow (2^-125 is
+// far below what a bf16 P can add next to the row maximum's weight of >= 1).
+__device__ __forceinline__ uint64_t exp2_poly_x2(float x0, float x1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = add_f32x2(x, f32x2(kMagic, kMagic));
+  const uint64_t n = add_f32x2(t, f32x2(-kMagic, -kMagic));
+  const uint64_t f = fma_f32x2(n, f32x2(-1.f, -1.f), x);
+  uint64_t q = fma_f32x2(f32x2(0x1.c3f76p-5f, 0x1.c3f76p-5f), f,
+                         f32x2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  q = fma_f32x2(q, f, f32x2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  q = fma_f32x2(q, f, f32x2(0x1.fff692p-1f, 0x1.fff692p-1f));
+  float t0, t1, q0, q1;
+  f32x2_split(t, t0, t1);
+  f32x2_split(q, q0, q1);
+  const uint32_t r0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
+  return f32x2(__uint_as_float(r0), __uint_as_float(r1));
+}
 
 struct FwdParams {
   uint16_t *o;         // [BH, N, D] bf16
@@ -91,17 +145,24 @@ struct Smem {
   static constexpr int kSub = D / 64;                         // 64-col panels
   static constexpr uint32_t kPanelBytes = kBlockM * 128;      // 128 rows x 128 B
   static constexpr uint32_t kTileBytes = kBlockM * D * 2;     // one Q/K/V tile
-  static constexpr int kStages = (D == 128) ? 2 : 4;          // K and V ring depth
+  // Ring depths.  K_j is released as soon as both S MMAs of iteration j are
+  // issued, V_j only after both P.V MMAs, so V needs the deeper ring to be
+  // refilled a full iteration ahead.
+#ifndef ATTN_V_STAGES_D128
+#define ATTN_V_STAGES_D128 2
+#endif
+  static constexpr int kKStages = (D == 128) ? 2 : 4;
+  static constexpr int kVStages = (D == 128) ? ATTN_V_STAGES_D128 : 4;
   static constexpr uint32_t kQ = 0;                           // 2 Q tiles
   static constexpr uint32_t kK = kQ + 2 * kTileBytes;         // K ring
-  static constexpr uint32_t kV = kK + kStages * kTileBytes;   // V ring
-  static constexpr uint32_t kBars = kV + kStages * kTileBytes;
+  static constexpr uint32_t kV = kK + kKStages * kTileBytes;  // V ring
+  static constexpr uint32_t kBars = kV + kVStages * kTileBytes;
   // barrier indices
   static constexpr int Q_FULL = 0, Q_EMPTY = 2, S_FULL = 4, P_FULL = 6,
                        O_FULL = 8, O_EMPTY = 10, DRAIN = 12,
-                       K_FULL = 13, K_EMPTY = K_FULL + kStages,
-                       V_FULL = K_EMPTY + kStages, V_EMPTY = V_FULL + kStages,
-                       NUM_BARS = V_EMPTY + kStages;
+                       K_FULL = 13, K_EMPTY = K_FULL + kKStages,
+                       V_FULL = K_EMPTY + kKStages, V_EMPTY = V_FULL + kVStages,
+                       NUM_BARS = V_EMPTY + kVStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;  // tmem slot, abort
   static constexpr uint32_t kBytes = kMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for alignment
@@ -144,13 +205,18 @@ struct WaitCtx {
 
 // Bounded wait for the phase of `bar` with parity `parity`.  Returns false
 // (after flagging the CTA and the device status word) when the time limit
-// runs out, or when another thread of the CTA already gave up.
+// runs out, or when another thread of the CTA already gave up.  A waiting
+// thread sleeps inside try_wait (up to kSleepHintNs per probe) instead of
+// spinning, so it takes no issue slots from the warps sharing its SM
+// sub-partition; the abort flag and the clock are looked at between probes.
+constexpr uint32_t kSleepHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           const WaitCtx &wc, uint32_t role) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
     if (*wc.abort) return false;
     if (global_timer_ns() - t0 > wc.timeout_ns) {
       *wc.abort = 1;
@@ -160,11 +226,32 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Same contract as mbar_wait, for the single MMA-issuing thread: it polls
+// without sleeping (it is on the critical path of every tile, and a thread
+// woken from a sleeping probe resumes late), looking at the abort flag and
+// the clock every 128 probes.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                               const WaitCtx &wc, uint32_t role) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 127u) == 0) {
+      if (*wc.abort) return false;
+      if (global_timer_ns() - t0 > wc.timeout_ns) {
+        *wc.abort = 1;
+        atomicOr(wc.status, kStatusTimeout | role);
+        return false;
+      }
+    }
+  }
+}
+
 // Bounded wait used while draining after an abort: ignores the abort flag.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,
                                                 const WaitCtx &wc) {
   const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, kSleepHintNs)) {
     if (global_timer_ns() - t0 > wc.timeout_ns) {
       atomicOr(wc.status, kStatusTimeout | kRoleDrain);
       return;
@@ -183,7 +270,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr,
 
 // ------------------------------------------------------------------ loader
 
-template <int D, bool CAUSAL>
+// Two loader threads: one for Q and K, one for V, so that K (released early,
+// after the S MMAs) never waits in line behind V (released late, after the
+// P.V MMAs).
+constexpr int kLoadQK = 1, kLoadV = 2;
+
+template <int D, bool CAUSAL, int MODE>
 __device__ __forceinline__ void producer_role(uint32_t base,
                                               const CUtensorMap *tq,
                                               const CUtensorMap *tk,
@@ -195,7 +287,7 @@ __device__ __forceinline__ void producer_role(uint32_t base,
   int qocc[2] = {0, 0};     // non-empty occurrences of each Q tile so far
   int q_issued[2] = {0, 0};
   int k_issued = 0, v_issued = 0;
-  bool skip_first_q = (p.debug_flags & 1u) && blockIdx.x == 0;
+  bool skip_first_q = (MODE != kLoadV) && (p.debug_flags & 1u) && blockIdx.x == 0;
   bool ok = true;
   const uint64_t pol_kv = policy_evict_last();
   const uint64_t pol_q = policy_evict_first();
@@ -203,7 +295,7 @@ __device__ __forceinline__ void producer_role(uint32_t base,
   for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
     const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
     const int nt[2] = {w.n0, w.n1};
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; MODE != kLoadV && t < 2; ++t) {
       if (nt[t] == 0) continue;
       if (qocc[t] > 0) {
         ok = mbar_wait(bar(L::Q_EMPTY + t), (qocc[t] - 1) & 1, wc, kRoleProducer);
@@ -224,24 +316,30 @@ __device__ __forceinline__ void producer_role(uint32_t base,
     if (!ok) break;
     const int nmax = max(nt[0], nt[1]);
     for (int j = 0; j < nmax; ++j) {
-      const int st = k_issued % L::kStages;
-      const uint32_t ph = (k_issued / L::kStages) & 1;
-      ok = mbar_wait(bar(L::K_EMPTY + st), ph ^ 1, wc, kRoleProducer);
-      if (!ok) break;
-      mbar_arrive_expect_tx(bar(L::K_FULL + st), L::kTileBytes);
-      for (int s = 0; s < L::kSub; ++s)
-        tma_load_3d_hint(base + L::kK + st * L::kTileBytes + s * L::kPanelBytes,
-                         tk, bar(L::K_FULL + st), s * 64, j * kBlockN, w.bh,
-                         pol_kv);
-      ++k_issued;
-      ok = mbar_wait(bar(L::V_EMPTY + st), ph ^ 1, wc, kRoleProducer);
-      if (!ok) break;
-      mbar_arrive_expect_tx(bar(L::V_FULL + st), L::kTileBytes);
-      for (int s = 0; s < L::kSub; ++s)
-        tma_load_3d_hint(base + L::kV + st * L::kTileBytes + s * L::kPanelBytes,
-                         tv, bar(L::V_FULL + st), s * 64, j * kBlockN, w.bh,
-                         pol_kv);
-      ++v_issued;
+      if (MODE != kLoadV) {
+        const int ks = k_issued % L::kKStages;
+        ok = mbar_wait(bar(L::K_EMPTY + ks), ((k_issued / L::kKStages) & 1) ^ 1,
+                       wc, kRoleProducer);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(L::K_FULL + ks), L::kTileBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d_hint(base + L::kK + ks * L::kTileBytes + s * L::kPanelBytes,
+                           tk, bar(L::K_FULL + ks), s * 64, j * kBlockN, w.bh,
+                           pol_kv);
+        ++k_issued;
+      }
+      if (MODE != kLoadQK) {
+        const int vs = v_issued % L::kVStages;
+        ok = mbar_wait(bar(L::V_EMPTY + vs), ((v_issued / L::kVStages) & 1) ^ 1,
+                       wc, kRoleProducer);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(L::V_FULL + vs), L::kTileBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d_hint(base + L::kV + vs * L::kTileBytes + s * L::kPanelBytes,
+                           tv, bar(L::V_FULL + vs), s * 64, j * kBlockN, w.bh,
+                           pol_kv);
+        ++v_issued;
+      }
     }
   }
 
@@ -250,16 +348,16 @@ __device__ __forceinline__ void producer_role(uint32_t base,
     for (int t = 0; t < 2; ++t)
       if (q_issued[t] > 0)
         mbar_wait_drain(bar(L::Q_FULL + t), (q_issued[t] - 1) & 1, wc);
-    for (int st = 0; st < L::kStages; ++st) {
+    for (int st = 0; st < L::kKStages; ++st)
       if (k_issued > st) {
-        const int last = st + ((k_issued - 1 - st) / L::kStages) * L::kStages;
-        mbar_wait_drain(bar(L::K_FULL + st), (last / L::kStages) & 1, wc);
+        const int last = st + ((k_issued - 1 - st) / L::kKStages) * L::kKStages;
+        mbar_wait_drain(bar(L::K_FULL + st), (last / L::kKStages) & 1, wc);
       }
+    for (int st = 0; st < L::kVStages; ++st)
       if (v_issued > st) {
-        const int last = st + ((v_issued - 1 - st) / L::kStages) * L::kStages;
-        mbar_wait_drain(bar(L::V_FULL + st), (last / L::kStages) & 1, wc);
+        const int last = st + ((v_issued - 1 - st) / L::kVStages) * L::kVStages;
+        mbar_wait_drain(bar(L::V_FULL + st), (last / L::kVStages) & 1, wc);
       }
-    }
   }
 }
 
@@ -318,13 +416,13 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
     const int nmax = max(nt[0], nt[1]);
     for (int t = 0; t < 2 && ok; ++t)
       if (nt[t] > 0) {
-        ok = mbar_wait(bar(L::Q_FULL + t), qocc[t] & 1, wc, kRoleMma);
+        ok = mbar_wait_spin(bar(L::Q_FULL + t), qocc[t] & 1, wc, kRoleMma);
         ++qocc[t];
       }
     if (!ok) break;
     {  // S_0 for both tiles
-      const int ks = kcons % L::kStages;
-      ok = mbar_wait(bar(L::K_FULL + ks), (kcons / L::kStages) & 1, wc, kRoleMma);
+      const int ks = kcons % L::kKStages;
+      ok = mbar_wait_spin(bar(L::K_FULL + ks), (kcons / L::kKStages) & 1, wc, kRoleMma);
       if (!ok) break;
       tc_fence_after_sync();
       for (int t = 0; t < 2; ++t)
@@ -337,31 +435,32 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
       ++kcons;
     }
     for (int j = 0; j < nmax && ok; ++j) {
-      const int vs = vcons % L::kStages;
-      ok = mbar_wait(bar(L::V_FULL + vs), (vcons / L::kStages) & 1, wc, kRoleMma);
+      const int vs = vcons % L::kVStages;
+      ok = mbar_wait_spin(bar(L::V_FULL + vs), (vcons / L::kVStages) & 1, wc, kRoleMma);
       if (!ok) break;
-      const int ks = kcons % L::kStages;
-      bool k_next = false;
+      const int ks = kcons % L::kKStages;
+      const bool k_next = j + 1 < nmax;  // K_{j+1} exists (waited below)
+      bool k_ready = false;
       for (int t = 0; t < 2; ++t) {
         if (j >= nt[t]) continue;
-        ok = mbar_wait(bar(L::P_FULL + t), pcnt[t] & 1, wc, kRoleMma);
+        ok = mbar_wait_spin(bar(L::P_FULL + t), pcnt[t] & 1, wc, kRoleMma);
         ++pcnt[t];
         if (!ok) break;
         if (j == 0 && oocc[t] > 0) {
           // previous unit's epilogue must have read O out of TMEM
-          ok = mbar_wait(bar(L::O_EMPTY + t), (oocc[t] - 1) & 1, wc, kRoleMma);
+          ok = mbar_wait_spin(bar(L::O_EMPTY + t), (oocc[t] - 1) & 1, wc, kRoleMma);
           if (!ok) break;
         }
         tc_fence_after_sync();
         issue_pv<D>(tO[t], tS[t], base + L::kV + vs * L::kTileBytes, j > 0);
         mma_commit(bar(L::O_FULL + t));
         if (j + 1 < nt[t]) {
-          if (!k_next) {
-            ok = mbar_wait(bar(L::K_FULL + ks), (kcons / L::kStages) & 1, wc,
-                           kRoleMma);
+          if (!k_ready) {
+            ok = mbar_wait_spin(bar(L::K_FULL + ks), (kcons / L::kKStages) & 1, wc,
+                          kRoleMma);
             if (!ok) break;
             tc_fence_after_sync();
-            k_next = true;
+            k_ready = true;
           }
           // issued after this tile's P.V in the same thread: the tensor pipe
           // reads P before this MMA overwrites the S columns holding it
@@ -402,6 +501,70 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
   }
 }
 
+// Loads this thread's row of S (128 fp32 columns of TMEM) into registers;
+// on the last tile of a row applies the mask: keys c > limit are -inf
+// (causal diagonal: limit = row; ragged tail: limit = N - 1 - first key).
+__device__ __forceinline__ void load_scores(uint32_t tS, uint32_t (&s)[4][32],
+                                            bool mask, int limit) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+  tmem_wait_ld(s[0]);
+  reg_fence(s[1]);
+  reg_fence(s[2]);
+  reg_fence(s[3]);
+  if (mask) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (c > limit) s[c >> 5][c & 31] = __float_as_uint(-CUDART_INF_F);
+  }
+}
+
+// Row maximum of the raw scores: 3-input max over pairs, 8 chains.
+__device__ __forceinline__ float row_max_raw(const uint32_t (&s)[4][32]) {
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[0][i]);
+#pragma unroll
+  for (int c = 8; c < 128; c += 2)
+    mx[(c >> 1) & 7] = max3f(mx[(c >> 1) & 7], __uint_as_float(s[c >> 5][c & 31]),
+                             __uint_as_float(s[(c + 1) >> 5][(c + 1) & 31]));
+  return max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]),
+               fmaxf(mx[6], mx[7]));
+}
+
+// p = 2^(s * scale * log2 e - m) for the whole row: one packed FMA per pair,
+// the exponential on the MUFU unit or (kEmuPer8 pairs in 8) the FMA pipe,
+// packed row sums, bf16x2 packing for the P.V MMA.  Returns the row sum.
+template <int D>
+__device__ __forceinline__ float exp_row(const uint32_t (&s)[4][32], float cl2,
+                                         float m, uint32_t (&pk)[2][32]) {
+  const uint64_t c2 = f32x2(cl2, cl2);
+  const uint64_t nm2 = f32x2(-m, -m);
+  uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    const float s0 = __uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]);
+    const float s1 = __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
+    const uint64_t x2 = fma_f32x2(f32x2(s0, s1), c2, nm2);
+    float x0, x1;
+    f32x2_split(x2, x0, x1);
+    uint64_t p2;
+    if ((c & 7) < kEmuPer8<D>) {
+      p2 = exp2_poly_x2(x0, x1);
+    } else {
+      p2 = f32x2(ex2_approx(x0), ex2_approx(x1));
+    }
+    acc[c & 1] = add_f32x2(acc[c & 1], p2);
+    float p0, p1;
+    f32x2_split(p2, p0, p1);
+    pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+  }
+  float a0, a1, b0, b1;
+  f32x2_split(acc[0], a0, a1);
+  f32x2_split(acc[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
 template <int D, bool CAUSAL>
 __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
                                              const FwdParams &p,
@@ -434,62 +597,37 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
       if (!ok) break;
       tc_fence_after_sync();
 
+      const bool mask = (j == n - 1) && (CAUSAL || (p.n & (kBlockN - 1)));
+      const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
       uint32_t s[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
-      tmem_wait_ld(s[0]);
-      reg_fence(s[1]);
-      reg_fence(s[2]);
-      reg_fence(s[3]);
-
-      if (j == n - 1 && (CAUSAL || (p.n & (kBlockN - 1)))) {
-        // diagonal tile (causal: key c visible iff c <= row) or ragged tail
-        // (keys at or beyond N do not exist)
-        const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > limit) s[c >> 5][c & 31] = __float_as_uint(-CUDART_INF_F);
-      }
-
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(s[0][i]);
-#pragma unroll
-      for (int c = 8; c < 128; ++c)
-        mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c >> 5][c & 31]));
-      const float m_tile =
-          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * cl2;
-
-      // Lazy max update (warp-uniform decision, per-row values).
-      const bool update =
-          __any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold);
-      float alpha = 1.f;
-      if (update) {
-        const float m_new = fmaxf(m_run, m_tile);
-        alpha = ex2_approx(m_run - m_new);  // 0 on the first tile (m_run = -inf)
-        l_run *= alpha;
-        m_run = m_new;
-      }
-
-      const float neg_m = -m_run;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[2][32];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float x0 = __uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]);
-        const float x1 = __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
-        const float p0 = ex2_approx(fmaf(x0, cl2, neg_m));
-        const float p1 = ex2_approx(fmaf(x1, cl2, neg_m));
-        ls[c & 3] += p0 + p1;
-        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+      load_scores(tS, s, mask, limit);
+
+      // Row max and the lazy base update: the base only moves when some row
+      // of the warp gains more than 2^8 (warp-uniform decision, per-row
+      // values); P then stays below 256 and O / l is unchanged because m and
+      // l always move together.  The first tile of a row sets the base.
+      const float m_tile = row_max_raw(s) * cl2;
+      float alpha = 1.f;
+      bool update = false;
+      if (j == 0) {
+        m_run = m_tile;
+      } else {
+        update = __any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold);
+        if (update) {
+          const float m_new = fmaxf(m_run, m_tile);
+          alpha = ex2_approx(m_run - m_new);
+          l_run *= alpha;
+          m_run = m_new;
+        }
       }
+      const float row_sum = exp_row<D>(s, cl2, m_run, pk);
       tmem_st_32x32b_x32(tS + 0, pk[0]);
       tmem_st_32x32b_x32(tS + 32, pk[1]);
-      l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l_run += row_sum;
       // O holds the earlier P.V products; the S_FULL commit for this tile was
       // issued after the previous P.V, so that MMA has completed.
-      if (update && j > 0) rescale_o<D>(tO, alpha);
+      if (update) rescale_o<D>(tO, alpha);
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
@@ -561,9 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(b0 + 8 * (L::O_EMPTY + t), 4);
     }
     mbar_init(b0 + 8 * L::DRAIN, 1);
-    for (int s = 0; s < L::kStages; ++s) {
+    for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(b0 + 8 * (L::K_FULL + s), 1);
       mbar_init(b0 + 8 * (L::K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < L::kVStages; ++s) {
       mbar_init(b0 + 8 * (L::V_FULL + s), 1);
       mbar_init(b0 + 8 * (L::V_EMPTY + s), 1);
     }
@@ -586,12 +726,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
 
   if (warp < 8) {
+    setmaxnreg_inc<kSoftmaxRegs>();
     softmax_role<D, CAUSAL>(base, tmem, p, wc, warp, lane);
-  } else if (warp == kProducerWarp) {
-    if (lane == 0) producer_role<D, CAUSAL>(base, &tm_q, &tm_k, &tm_v, p, wc);
-    __syncwarp();
   } else {
-    if (lane == 0) mma_role<D, CAUSAL>(base, tmem, p, wc);
+    setmaxnreg_dec<kControlRegs>();
+    if (warp == kProducerWarp) {
+      if (lane == 0)
+        producer_role<D, CAUSAL, kLoadQK>(base, &tm_q, &tm_k, &tm_v, p, wc);
+    } else if (warp == kVLoaderWarp) {
+      if (lane == 0)
+        producer_role<D, CAUSAL, kLoadV>(base, &tm_q, &tm_k, &tm_v, p, wc);
+    } else if (warp == kMmaWarp) {
+      if (lane == 0) mma_role<D, CAUSAL>(base, tmem, p, wc);
+    }
     __syncwarp();
   }
 

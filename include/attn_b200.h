@@ -141,6 +141,18 @@ int attn_status(attn_stream_t stream);
  * (which pipeline role gave up), for diagnostics; 0 when none. */
 uint32_t attn_last_status_bits(void);
 
+/*
+ * attn_selftest_exp2 -- test hook for the kernel's exponentials.  For n
+ * device floats x, writes y[i] = 2^x[i] as the attention kernel evaluates
+ * it: mode 0 = the FMA-pipe polynomial (Cody-Waite split + degree-3 minimax,
+ * inputs below -125 clamped to -125), mode 1 = the ex2.approx instruction.
+ * x and y are 4-byte aligned device pointers of the current device; the work
+ * is queued on `stream`.  Returns ATTN_ERR_NULL_POINTER, ATTN_ERR_INVALID_SIZE
+ * (n < 0) or ATTN_ERR_INVALID_SCALE (mode not 0 or 1) before any CUDA call.
+ */
+int attn_selftest_exp2(const float *x, float *y, int n, int mode,
+                       attn_stream_t stream);
+
 /* Size of the static device scratch array behind attn_fwd_host_noalloc:
  * 256 bytes of status followed by the q, k, v, o, lse staging area. */
 #define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
