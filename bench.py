@@ -33,6 +33,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from exact_io_aware_73_b200 import replicas as R  # noqa: E402
 from exact_io_aware_73_b200 import workloads as W  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (bf16, causal/non-causal) and % of B200 dense BF16 peak"
@@ -81,63 +82,69 @@ def load_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled every 10 ms through NVML while
+    the timed region runs (read-only queries); nvidia-smi is the fallback."""
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
+               "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
-        self.t = None
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self._nvml = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-            return
-        self.t = threading.Thread(target=self._read, daemon=True)
-        self.t.start()
-        time.sleep(0.3)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(
+                h, pynvml.NVML_CLOCK_SM)
+            self._nvml = (pynvml, h)
+        except Exception:  # no NVML: fall back to one nvidia-smi query
+            self._nvml = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _query(self):
+        if self._nvml is not None:
+            pynvml, h = self._nvml
+            mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            try:
+                mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except AttributeError:
+                mask = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+            return float(mhz), int(mask)
+        out = subprocess.run(
+            ["nvidia-smi", "-i", str(self.gpu),
+             "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+             "--format=csv,noheader,nounits"], capture_output=True, text=True,
+            timeout=10).stdout.strip().split(",")
+        self.max_mhz = float(out[1])
+        return float(out[0]), int(out[2].strip(), 16)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._query())
+            except Exception:
+                return
+            self._stop.wait(0.01 if self._nvml is not None else 0.2)
 
     def stop(self):
-        if self.proc is None:
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=5)
+        if not self.samples:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        if self.t:
-            self.t.join(timeout=2)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = sorted(n for n, bit in self.REASONS.items()
+                         if any(m & bit for _, m in self.samples))
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples),
+                "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
 def cpu_baseline(w, qkv, budget_s: float, seed: int = 11):
@@ -184,7 +191,8 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     qkv = W.make_qkv(w)
-    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.2, min(args.cpu_budget_s, 20.0,
+                            150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(w, qkv, per_step / 4)
     vals = []
@@ -230,27 +238,20 @@ def main():
         return run_reference(args, w)
 
     import torch
-    import torch.distributed as dist
     from exact_io_aware_73_b200 import attn
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = R.env_ranks()
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+    R.init("nccl", world, device=dev)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        R.barrier(world)
 
     # ---- inputs (seeded per rank), resident in HBM before timing
-    seed = w.seed + 7919 * rank
+    seed = R.rank_seed(w.seed, rank)
     qkv_host = W.make_qkv(w, seed=seed)
     q, k, v = (t.to(dev) for t in qkv_host)
     o = torch.empty_like(q)
@@ -308,13 +309,10 @@ def main():
     if rc != 0:
         raise attn.AttnError(rc, "timed region")
 
-    t = torch.tensor([kernel_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = R.max_over_ranks(kernel_ms, world, dev)
     ms_per_step = max_ms / args.steps
     flops = w.flops()
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = R.job_throughput(flops, world, ms_per_step * 1e-3) / 1e12
 
     # ---- end to end through the host-buffer C entry point
     qh, kh, vh = (x.pin_memory() for x in qkv_host)
@@ -339,11 +337,8 @@ def main():
     rc = attn.status()
     if rc != 0:
         raise attn.AttnError(rc, "e2e region")
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / e2e_steps
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = R.max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    e2e_value = R.job_throughput(flops, world, e2e_ms * 1e-3) / 1e12
     h2d = 3 * qh.numel() * 2
     d2h = oh.numel() * 2 + lh.numel() * 4
 
@@ -387,8 +382,7 @@ def main():
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    R.finish(world)
     return 0
 
 
