@@ -14,6 +14,7 @@ brute force and a hand-worked fixture (``tests/golden/``).
 """
 from .oracle import (  # noqa: F401
     attention,
+    attention_backward,
     attention_blocked,
     attention_rows_bf16,
     attend_scores,

@@ -33,6 +33,15 @@
  * block).  It exists only so that the two-pass oracle can be cross-checked
  * against the pages' own algorithm; it calls none of the two-pass helpers.
  *
+ * The backward pass ([MM] "Backward pass: menghitung ulang, bukan
+ * menyimpan") is the gradient of the same definition, written out from the
+ * calculus (the pages give no formulas): for an upstream gradient dO,
+ *     dV = P^T dO,   dP = dO V^T,   D_i = sum_j P_ij dP_ij,
+ *     dS = P * (dP - D) (elementwise, D broadcast along the row),
+ *     dQ = scale * dS K,   dK = scale * dS^T Q.
+ * Masked entries have P = 0 and so dS = 0.  The oracle recomputes P from
+ * the scores with its own two-pass softmax, exactly as the forward does.
+ *
  * Layout conventions: Q, K, V, O are contiguous row-major [B, H, N, d];
  * lse is contiguous [B, H, N].  bf16 inputs are passed as their raw 16-bit
  * patterns and widened exactly to double (bf16 -> fp32 is exact, fp32 ->
@@ -310,6 +319,82 @@ int oracle_attention_blocked_f64(const double *Q, const double *K,
   }
   free(Sij); free(PV); free(mi); free(li);
   return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward pass.                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Gradients of the attention forward for one (b, h) head: Q, K, V, dO are
+ * [N, d]; dQ, dK, dV are [N, d] outputs.  P is materialised row by row with
+ * the two-pass softmax; dK and dV accumulate over the rows of the head in
+ * ascending row order. */
+static int backward_head(const double *Q, const double *K, const double *V,
+                         const double *dO, double *dQ, double *dK, double *dV,
+                         int64_t N, int64_t d, int causal, double scale) {
+  double *s = (double *)malloc(sizeof(double) * (size_t)N);
+  double *pr = (double *)malloc(sizeof(double) * (size_t)N);
+  double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+  if (!s || !pr || !dp) { free(s); free(pr); free(dp); return ORACLE_ENOMEM; }
+  for (int64_t x = 0; x < N * d; ++x) { dQ[x] = 0.0; dK[x] = 0.0; dV[x] = 0.0; }
+  for (int64_t i = 0; i < N; ++i) {
+    const int64_t n = visible_keys(i, N, causal);
+    const double *qi = Q + i * d, *doi = dO + i * d;
+    /* scores and probabilities of row i */
+    for (int64_t j = 0; j < n; ++j) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < d; ++t) acc += qi[t] * K[j * d + t];
+      s[j] = scale * acc;
+    }
+    double m = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) if (s[j] > m) m = s[j];
+    double l = 0.0;
+    for (int64_t j = 0; j < n; ++j) { pr[j] = exp(s[j] - m); l += pr[j]; }
+    for (int64_t j = 0; j < n; ++j) pr[j] /= l;
+    /* dP_ij = dO_i . V_j ; D_i = sum_j P_ij dP_ij */
+    double Di = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < d; ++t) acc += doi[t] * V[j * d + t];
+      dp[j] = acc;
+      Di += pr[j] * acc;
+    }
+    for (int64_t j = 0; j < n; ++j) {
+      const double dsij = pr[j] * (dp[j] - Di);
+      for (int64_t t = 0; t < d; ++t) {
+        dV[j * d + t] += pr[j] * doi[t];
+        dQ[i * d + t] += scale * dsij * K[j * d + t];
+        dK[j * d + t] += scale * dsij * qi[t];
+      }
+    }
+  }
+  free(s); free(pr); free(dp);
+  return ORACLE_OK;
+}
+
+/* Backward of the attention forward over fp64 [B, H, N, d] inputs.  OpenMP
+ * parallel over heads (each head's dK, dV sum over all of its rows). */
+int oracle_attention_backward_f64(const double *Q, const double *K,
+                                  const double *V, const double *dO,
+                                  double *dQ, double *dK, double *dV,
+                                  int64_t B, int64_t H, int64_t N, int64_t d,
+                                  int causal, double scale, int nthreads) {
+  if (!Q || !K || !V || !dO || !dQ || !dK || !dV || B < 0 || H < 0 ||
+      N < 0 || d < 1)
+    return ORACLE_EBADARG;
+  const int64_t heads = B * H;
+  int err = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads > 0 ? nthreads : 1)
+  for (int64_t h = 0; h < heads; ++h) {
+    const int64_t off = h * N * d;
+    int rc = backward_head(Q + off, K + off, V + off, dO + off, dQ + off,
+                           dK + off, dV + off, N, d, causal, scale);
+    if (rc != ORACLE_OK) {
+#pragma omp atomic write
+      err = rc;
+    }
+  }
+  return err;
 }
 
 /* Threads OpenMP would use by default (for reporting). */

@@ -36,6 +36,10 @@ def _load():
         lib.oracle_attention_rows_bf16.argtypes = [
             u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_int,
             ctypes.c_double, i64p, i64, dp, dp, ctypes.c_int]
+        lib.oracle_attention_backward_f64.argtypes = [
+            dp, dp, dp, dp, dp, dp, dp, i64, i64, i64, i64, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int]
+        lib.oracle_attention_backward_f64.restype = ctypes.c_int
         lib.oracle_attention_blocked_f64.argtypes = [
             dp, dp, dp, dp, dp, i64, i64, i64, i64, ctypes.c_int,
             ctypes.c_double, i64, i64]
@@ -147,3 +151,18 @@ def attention_rows_bf16(qbits, kbits, vbits, causal: bool, scale: float,
         rows.size, _dptr(O), _dptr(lse), _threads(threads)),
         "attention_rows_bf16")
     return O, lse
+
+
+def attention_backward(q, k, v, do, causal: bool, scale: float, threads=None):
+    """Gradients (dQ, dK, dV) of the forward for upstream gradient dO; fp64
+    arrays shaped [B, H, N, d]."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    dq = np.empty((B, H, N, d))
+    dk = np.empty((B, H, N, d))
+    dv = np.empty((B, H, N, d))
+    _check(_load().oracle_attention_backward_f64(
+        _dptr(q), _dptr(k), _dptr(v), _dptr(do), _dptr(dq), _dptr(dk),
+        _dptr(dv), B, H, N, d, int(bool(causal)), float(scale),
+        _threads(threads)), "attention_backward")
+    return dq, dk, dv

@@ -17,6 +17,9 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "attention_oracle.c")
 
+PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+BACKWARD_PINS = os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")
+
 MUTANTS = {
     "mask_hides_diagonal": ("return causal ? (i + 1) : N;",
                             "return causal ? (i > 0 ? i : 1) : N;"),
@@ -36,9 +39,24 @@ MUTANTS = {
     "sum_sign_flipped": ("l += e;", "l -= e;"),
 }
 
+# planted mistakes in the backward pass; each must fail a backward pin
+BACKWARD_MUTANTS = {
+    "bwd_D_unweighted": ("Di += pr[j] * acc;", "Di += acc;"),
+    "bwd_dS_sign": ("const double dsij = pr[j] * (dp[j] - Di);",
+                    "const double dsij = pr[j] * (Di - dp[j]);"),
+    "bwd_dK_no_scale": ("dK[j * d + t] += scale * dsij * qi[t];",
+                        "dK[j * d + t] += dsij * qi[t];"),
+    "bwd_dV_uses_dP": ("dV[j * d + t] += pr[j] * doi[t];",
+                       "dV[j * d + t] += dp[j] * doi[t];"),
+    "bwd_dQ_uses_V": ("dQ[i * d + t] += scale * dsij * K[j * d + t];",
+                      "dQ[i * d + t] += scale * dsij * V[j * d + t];"),
+    "bwd_mask_leak": ("const int64_t n = visible_keys(i, N, causal);\n    const double *qi = Q + i * d, *doi",
+                      "const int64_t n = causal ? (i + 1 < N ? i + 2 : N) : N;\n    const double *qi = Q + i * d, *doi"),
+}
+
 
 def _build_mutant(name, tmpdir):
-    old, new = MUTANTS[name]
+    old, new = {**MUTANTS, **BACKWARD_MUTANTS}[name]
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
     path_c = os.path.join(tmpdir, f"{name}.c")
@@ -50,21 +68,31 @@ def _build_mutant(name, tmpdir):
     return path_so
 
 
+def _run_against(mutants, pin_file, tmp):
+    procs = {}
+    for name in mutants:
+        so = _build_mutant(name, tmp)
+        env = dict(os.environ, ORACLE_LIBRARY=so)
+        procs[name] = subprocess.Popen(
+            [sys.executable, "-m", "pytest", "-q", "-x", "-p",
+             "no:cacheprovider", pin_file],
+            cwd=ROOT, env=env, stdout=subprocess.PIPE,
+            stderr=subprocess.STDOUT)
+    survivors = []
+    for name, p in procs.items():
+        p.communicate(timeout=600)
+        if p.returncode == 0:
+            survivors.append(name)
+    return survivors
+
+
 def test_every_planted_mistake_fails_a_pin():
     with tempfile.TemporaryDirectory() as tmp:
-        procs = {}
-        for name in MUTANTS:
-            so = _build_mutant(name, tmp)
-            env = dict(os.environ, ORACLE_LIBRARY=so)
-            procs[name] = subprocess.Popen(
-                [sys.executable, "-m", "pytest", "-q", "-x", "-p",
-                 "no:cacheprovider", os.path.join(ROOT, "tests",
-                                                  "test_oracle_pins.py")],
-                cwd=ROOT, env=env, stdout=subprocess.PIPE,
-                stderr=subprocess.STDOUT)
-        survivors = []
-        for name, p in procs.items():
-            out, _ = p.communicate(timeout=600)
-            if p.returncode == 0:
-                survivors.append(name)
+        survivors = _run_against(MUTANTS, PINS, tmp)
         assert not survivors, f"pins did not catch: {survivors}"
+
+
+def test_every_planted_backward_mistake_fails_a_backward_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        survivors = _run_against(BACKWARD_MUTANTS, BACKWARD_PINS, tmp)
+        assert not survivors, f"backward pins did not catch: {survivors}"
