@@ -192,3 +192,49 @@ def selftest_exp2(x, mode: int, stream=None):
     _check(f(x.data_ptr(), y.data_ptr(), x.numel(), int(mode),
              _stream_handle(stream)), "attn_selftest_exp2")
     return y
+
+
+def _bwd_fns():
+    L = lib()
+    f, g = L.attn_bwd, L.attn_bwd_workspace_bytes
+    if f.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        f.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                      i, i, i, i, i, ctypes.c_float, vp]
+        f.restype = i
+        g.argtypes = [i, i, i]
+        g.restype = ctypes.c_size_t
+    return f, g
+
+
+def bwd_workspace_bytes(B, H, N) -> int:
+    return int(_bwd_fns()[1](B, H, N))
+
+
+def attn_bwd_raw(q, k, v, o, dout, lse, dq, dk, dv, ws, ws_bytes, B, H, N, d,
+                 causal, scale, stream_handle) -> int:
+    """Direct call with integer pointers; returns the library's code."""
+    return _bwd_fns()[0](q, k, v, o, dout, lse, dq, dk, dv, ws, ws_bytes,
+                         int(B), int(H), int(N), int(d), int(bool(causal)),
+                         float(scale), stream_handle)
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal: bool = False,
+             scale: float | None = None, stream=None, workspace=None):
+    """dQ, dK, dV of attn_fwd for upstream gradient dout (bf16 CUDA tensors
+    [B, H, N, d]; o and lse are attn_fwd's outputs)."""
+    import torch
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    need = bwd_workspace_bytes(B, H, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    rc = attn_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                      dout.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                      dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                      workspace.numel(), B, H, N, d, causal, scale,
+                      _stream_handle(stream))
+    _check(rc, "attn_bwd")
+    return dq, dk, dv

@@ -14,7 +14,7 @@
 #include <mutex>
 
 #include "attn_b200.h"
-#include "attn_fwd_kernel.cuh"
+#include "attn_bwd_kernel.cuh"
 
 namespace {
 
@@ -30,6 +30,7 @@ struct DeviceState {
   int sm_count = 0;
   uint32_t *status = nullptr;  // 4-byte device status word, lazily allocated
   bool smem_attr_set[4] = {false, false, false, false};
+  bool bwd_attr_set[4] = {false, false, false, false};
 };
 
 std::mutex g_mu;
@@ -194,6 +195,55 @@ int launch(DeviceState &st, int variant, const CUtensorMap *maps,
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// fp32 vectors [bh, npad] (npad a multiple of 128) as a 2-D tensor with
+// 128-entry boxes: row stride npad * 4 bytes and every box start (x = 128 i)
+// are 512-byte multiples.
+int encode_vec_map(EncodeTiledFn enc, CUtensorMap *map, const void *ptr, int bh,
+                   int npad) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(npad), static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(npad) * 4};
+  cuuint32_t box[2] = {128, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(ptr),
+                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_TENSOR_MAP;
+}
+
+template <int D, bool CAUSAL>
+int launch_bwd(DeviceState &st, int variant, const CUtensorMap *m,
+               const attn_b200::BwdParams &p, cudaStream_t stream) {
+  using namespace attn_b200;
+  auto kdq = attn_bwd_dq_kernel<D, CAUSAL>;
+  auto kdkv = attn_bwd_dkdv_kernel<D, CAUSAL>;
+  const uint32_t smem_dq = BwdDqSmem<D>::kAlloc;
+  const uint32_t smem_dkv = BwdDkvSmem<D>::kAlloc;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!st.bwd_attr_set[variant]) {
+      if (cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_dq)) != cudaSuccess ||
+          cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_dkv)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      st.bwd_attr_set[variant] = true;
+    }
+  }
+  const int64_t prep_rows = static_cast<int64_t>(p.bh) * p.npad;
+  const int64_t prep_blocks_needed = (prep_rows + 7) / 8;
+  const int prep_blocks = static_cast<int>(
+      prep_blocks_needed < st.sm_count * 16 ? prep_blocks_needed : st.sm_count * 16);
+  attn_bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(p);
+  const int grid = p.num_units < st.sm_count ? p.num_units : st.sm_count;
+  kdq<<<grid, kBwdThreads, smem_dq, stream>>>(m[0], m[1], m[2], m[3], p);
+  kdkv<<<grid, kBwdThreads, smem_dkv, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
 __global__ void exp2_selftest_kernel(const float *x, float *y, int n, int mode) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (i >= n) return;
@@ -294,6 +344,93 @@ int attn_fwd_host(const void *q, const void *k, const void *v, void *o,
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int N) {
+  if (B < 0 || H < 0 || N < 0) return 0;
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  return 2 * round256(static_cast<size_t>(B) * H * npad * 4);
+}
+
+int attn_bwd(const void *q, const void *k, const void *v, const void *o,
+             const void *dout, const float *lse, void *dq, void *dk, void *dv,
+             void *workspace, size_t workspace_bytes, int B, int H, int N,
+             int d, int causal, float scale, attn_stream_t stream) {
+  if (B < 0 || H < 0 || N < 0) return ATTN_ERR_INVALID_SIZE;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID_SCALE;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv)
+    return ATTN_ERR_NULL_POINTER;
+  const int64_t bh64 = static_cast<int64_t>(B) * H;
+  if (N > ATTN_MAX_SEQ || bh64 > ATTN_MAX_HEADS) return ATTN_ERR_INVALID_SIZE;
+  const int64_t tiles = (N + 127) / 128;
+  if (bh64 * tiles > 0x7fffffffLL) return ATTN_ERR_INVALID_SIZE;
+  auto al = [](const void *ptr, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0;
+  };
+  if (!al(q, 16) || !al(k, 16) || !al(v, 16) || !al(o, 16) || !al(dout, 16) ||
+      !al(dq, 16) || !al(dk, 16) || !al(dv, 16) || !al(lse, 4))
+    return ATTN_ERR_MISALIGNED;
+  const size_t need = attn_bwd_workspace_bytes(B, H, N);
+  if (!workspace || workspace_bytes < need || !al(workspace, 256))
+    return ATTN_ERR_WORKSPACE;
+  const size_t tb = static_cast<size_t>(bh64) * N * d * 2;
+  const size_t lb = static_cast<size_t>(bh64) * N * 4;
+  const void *ins[6] = {q, k, v, o, dout, lse};
+  const size_t in_bytes[6] = {tb, tb, tb, tb, tb, lb};
+  void *outs[4] = {dq, dk, dv, workspace};
+  const size_t out_bytes[4] = {tb, tb, tb, need};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], out_bytes[a], ins[b], in_bytes[b])) return ATTN_ERR_ALIAS;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], out_bytes[a], outs[b], out_bytes[b])) return ATTN_ERR_ALIAS;
+  }
+  int rc, dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  const void *all[10] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
+  for (const void *ptr : all)
+    if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
+  EncodeTiledFn enc;
+  if ((rc = get_encode_fn(&enc)) != ATTN_OK) return rc;
+  const int bh = B * H;
+  const int npad = static_cast<int>(tiles * 128);
+  float *lse2 = static_cast<float *>(workspace);
+  float *dsum = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                          round256(static_cast<size_t>(bh) * npad * 4));
+  CUtensorMap maps[6];
+  if ((rc = encode_map(enc, &maps[0], q, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[1], dout, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[2], k, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[3], v, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_vec_map(enc, &maps[4], lse2, bh, npad)) != ATTN_OK) return rc;
+  if ((rc = encode_vec_map(enc, &maps[5], dsum, bh, npad)) != ATTN_OK) return rc;
+  attn_b200::BwdParams p;
+  p.o = static_cast<const uint16_t *>(o);
+  p.dout = static_cast<const uint16_t *>(dout);
+  p.lse = lse;
+  p.lse2 = lse2;
+  p.dsum = dsum;
+  p.dq = static_cast<uint16_t *>(dq);
+  p.dk = static_cast<uint16_t *>(dk);
+  p.dv = static_cast<uint16_t *>(dv);
+  p.status = st->status;
+  p.bh = bh;
+  p.n = N;
+  p.npad = npad;
+  p.tiles = static_cast<int>(tiles);
+  p.num_units = static_cast<int>(bh64 * tiles);
+  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.scale = scale;
+  p.timeout_ns = g_timeout_ns.load();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch_bwd<128, true>(*st, 0, maps, p, s)
+                  : launch_bwd<128, false>(*st, 1, maps, p, s);
+  return causal ? launch_bwd<64, true>(*st, 2, maps, p, s)
+                : launch_bwd<64, false>(*st, 3, maps, p, s);
 }
 
 int attn_status(attn_stream_t stream) {

@@ -1,0 +1,630 @@
+// attn_bwd_kernel.cuh -- backward pass of exact attention for B200 (sm_100a).
+//
+// Source cited as [MM]: the marketmaker.cc blog post (Indonesian edition)
+// "Apakah Konteks Sehari Penuh Mengalahkan Konteks Sepuluh Menit? Perhatian
+// Kilat dan Pertanyaan Panjang Urutan", section "Backward pass: menghitung
+// ulang, bukan menyimpan": the backward pass keeps only O and the softmax
+// statistics of the forward (here lse = m + ln l) and recomputes the score
+// tiles from Q and K instead of storing the N x N probabilities.
+//
+// Gradients of O = softmax(scale Q K^T [mask]) V for an upstream gradient dO
+// (the calculus of the forward definition; the pages give no formulas):
+//     P = exp(scale Q K^T - lse)   (recomputed per tile from the saved lse)
+//     dV = P^T dO      dP = dO V^T      D_i = sum_t dO_it O_it
+//     dS = P * (dP - D)             dQ = scale dS K      dK = scale dS^T Q
+//
+// Three kernels, all persistent with bounded waits like the forward:
+//   attn_bwd_prep_kernel    D_i, one warp per row (bandwidth-bound);
+//   attn_bwd_dq_kernel      one 128-row Q tile per unit, loop over K/V tiles:
+//                           S = Q K^T and dP = dO V^T (tcgen05, TMEM), the
+//                           compute warpgroup forms dS over S, dQ += dS K;
+//   attn_bwd_dkdv_kernel    one 128-key K/V tile per unit, loop over Q tiles:
+//                           S^T = K Q^T and dP^T = V dO^T, the compute
+//                           warpgroup forms P^T and dS^T (lse and D per query
+//                           column come from shared memory), dV += P^T dO,
+//                           dK += dS^T Q.
+// Each tcgen05 MMA has one of the two forms of the forward kernel: A and B
+// K-major in shared memory (N = 128), or A from TMEM and B MN-major (N = d).
+#pragma once
+
+#include "attn_fwd_kernel.cuh"
+
+namespace attn_b200 {
+
+constexpr int kBwdThreads = 192;   // warps 0-3 compute, 4 loader, 5 MMA
+constexpr int kBwdLoaderWarp = 4;
+constexpr int kBwdMmaWarp = 5;
+
+struct BwdParams {
+  const uint16_t *o;     // [BH, N, D] forward output (prep only)
+  const uint16_t *dout;  // [BH, N, D] upstream gradient (prep only)
+  const float *lse;      // [BH, N] forward log-sum-exp, natural log (prep only)
+  // Workspace, rows padded to npad = 128 * tiles so every 128-row TMA tile of
+  // these fp32 vectors starts on a 512-byte boundary; padding rows hold 0.
+  float *lse2;           // [BH, npad] lse * log2(e)
+  float *dsum;           // [BH, npad] D_i = sum_t dO_it O_it
+  uint16_t *dq, *dk, *dv;  // [BH, N, D] outputs
+  uint32_t *status;
+  int bh, n, npad, tiles, num_units;
+  float c_log2;          // scale * log2(e)
+  float scale;
+  unsigned long long timeout_ns;
+};
+
+// ------------------------------------------------------------------ prep
+
+// D_i = sum_t dO_it * O_it and lse_i * log2(e) for every row, fp32, into the
+// padded workspace vectors (0 in padding rows); one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256)
+    attn_bwd_prep_kernel(const BwdParams p) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(p.bh) * p.npad;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int64_t prow = warp; prow < rows; prow += nwarps) {
+    const int64_t bh = prow / p.npad;
+    const int n = static_cast<int>(prow - bh * p.npad);
+    float acc = 0.f, l2 = 0.f;
+    if (n < p.n) {
+      const int64_t row = bh * p.n + n;
+      const uint16_t *a = p.o + row * D + lane * (D / 32);
+      const uint16_t *b = p.dout + row * D + lane * (D / 32);
+#pragma unroll
+      for (int t = 0; t < D / 32; ++t)
+        acc += __uint_as_float(static_cast<uint32_t>(a[t]) << 16) *
+               __uint_as_float(static_cast<uint32_t>(b[t]) << 16);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      l2 = p.lse[row] * 1.4426950408889634f;
+    }
+    if (lane == 0) {
+      p.dsum[prow] = acc;
+      p.lse2[prow] = l2;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+
+template <int D>
+struct BwdDqSmem {
+  static constexpr uint32_t kTile = Smem<D>::kTileBytes;
+  static constexpr uint32_t kPanel = Smem<D>::kPanelBytes;
+  static constexpr int kSub = D / 64;
+  static constexpr int kStages = (D == 128) ? 2 : 4;  // K+V ring
+  static constexpr uint32_t kQ = 0, kDO = kTile;
+  static constexpr uint32_t kK = 2 * kTile;
+  static constexpr uint32_t kV = kK + kStages * kTile;
+  static constexpr uint32_t kBars = kV + kStages * kTile;
+  static constexpr int Q_FULL = 0, Q_EMPTY = 1, S_FULL = 2, DS_FULL = 3,
+                       ACC_FULL = 4, ACC_EMPTY = 5, DRAIN = 6, KV_FULL = 7,
+                       KV_EMPTY = KV_FULL + kStages,
+                       NUM_BARS = KV_EMPTY + kStages;
+  static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;
+  static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ void dq_unit(int u, int bh_count, int tiles,
+                                        int &bh, int &qt, int &nkv) {
+  if (CAUSAL) {  // longest rows first
+    qt = tiles - 1 - u / bh_count;
+    bh = u % bh_count;
+    nkv = qt + 1;
+  } else {
+    bh = u / tiles;
+    qt = u % tiles;
+    nkv = tiles;
+  }
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const BwdParams p) {
+  using L = BwdDqSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  auto bar = [&](int i) { return base + L::kBars + 8u * i; };
+
+  if (tid == 0) {
+    mbar_init(bar(L::Q_FULL), 1);
+    mbar_init(bar(L::Q_EMPTY), 1);
+    mbar_init(bar(L::S_FULL), 1);
+    mbar_init(bar(L::DS_FULL), 4);
+    mbar_init(bar(L::ACC_FULL), 1);
+    mbar_init(bar(L::ACC_EMPTY), 4);
+    mbar_init(bar(L::DRAIN), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::KV_FULL + s), 1);
+      mbar_init(bar(L::KV_EMPTY + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+  // TMEM: S (cols 0-127, dS written over it), dP (128-255), dQ (256-256+D)
+  const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+
+  if (warp == kBwdLoaderWarp) {
+    if (lane == 0) {
+      int uocc = 0, kv_issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        int bh, qt, nkv;
+        dq_unit<CAUSAL>(u, p.bh, p.tiles, bh, qt, nkv);
+        if (uocc > 0) {
+          ok = mbar_wait(bar(L::Q_EMPTY), (uocc - 1) & 1, wc, kRoleProducer);
+          if (!ok) break;
+        }
+        ++uocc;
+        mbar_arrive_expect_tx(bar(L::Q_FULL), 2 * L::kTile);
+        for (int s = 0; s < L::kSub; ++s) {
+          tma_load_3d(base + L::kQ + s * L::kPanel, &tm_q, bar(L::Q_FULL), s * 64,
+                      qt * kBlockM, bh);
+          tma_load_3d(base + L::kDO + s * L::kPanel, &tm_do, bar(L::Q_FULL),
+                      s * 64, qt * kBlockM, bh);
+        }
+        for (int j = 0; j < nkv; ++j) {
+          const int st = kv_issued % L::kStages;
+          ok = mbar_wait(bar(L::KV_EMPTY + st), ((kv_issued / L::kStages) & 1) ^ 1,
+                         wc, kRoleProducer);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(L::KV_FULL + st), 2 * L::kTile);
+          for (int s = 0; s < L::kSub; ++s) {
+            tma_load_3d(base + L::kK + st * L::kTile + s * L::kPanel, &tm_k,
+                        bar(L::KV_FULL + st), s * 64, j * kBlockN, bh);
+            tma_load_3d(base + L::kV + st * L::kTile + s * L::kPanel, &tm_v,
+                        bar(L::KV_FULL + st), s * 64, j * kBlockN, bh);
+          }
+          ++kv_issued;
+        }
+      }
+      if (*wc.abort) {
+        if (uocc > 0) mbar_wait_drain(bar(L::Q_FULL), (uocc - 1) & 1, wc);
+        for (int st = 0; st < L::kStages; ++st)
+          if (kv_issued > st) {
+            const int last = st + ((kv_issued - 1 - st) / L::kStages) * L::kStages;
+            mbar_wait_drain(bar(L::KV_FULL + st), (last / L::kStages) & 1, wc);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0) {
+      int uocc = 0, kv_cons = 0, ds_cnt = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        int bh, qt, nkv;
+        dq_unit<CAUSAL>(u, p.bh, p.tiles, bh, qt, nkv);
+        ok = mbar_wait_spin(bar(L::Q_FULL), uocc & 1, wc, kRoleMma);
+        if (!ok) break;
+        for (int j = 0; j < nkv; ++j) {
+          const int st = kv_cons % L::kStages;
+          ok = mbar_wait_spin(bar(L::KV_FULL + st), (kv_cons / L::kStages) & 1, wc,
+                              kRoleMma);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t k_s = base + L::kK + st * L::kTile;
+          const uint32_t v_s = base + L::kV + st * L::kTile;
+          // issued after the previous dQ MMA in this thread: it has read dS
+          // out of the S columns before they are overwritten
+          issue_qk<D>(tS, base + L::kQ, k_s);    // S  = Q  K^T
+          issue_qk<D>(tdP, base + L::kDO, v_s);  // dP = dO V^T
+          mma_commit(bar(L::S_FULL));
+          if (j == nkv - 1) mma_commit(bar(L::Q_EMPTY));  // last read of Q, dO
+          ok = mbar_wait_spin(bar(L::DS_FULL), ds_cnt & 1, wc, kRoleMma);
+          ++ds_cnt;
+          if (!ok) break;
+          if (j == 0 && uocc > 0) {
+            ok = mbar_wait_spin(bar(L::ACC_EMPTY), (uocc - 1) & 1, wc, kRoleMma);
+            if (!ok) break;
+          }
+          tc_fence_after_sync();
+          issue_pv<D>(tdQ, tS, k_s, j > 0);      // dQ += dS K
+          mma_commit(bar(L::KV_EMPTY + st));
+          ++kv_cons;
+        }
+        if (!ok) break;
+        mma_commit(bar(L::ACC_FULL));
+        ++uocc;
+      }
+      mma_commit(bar(L::DRAIN));
+      mbar_wait_drain(bar(L::DRAIN), 0, wc);
+    }
+    __syncwarp();
+  } else {
+    // compute warpgroup: thread = query row r of the tile
+    const int wq = warp;  // warps 0-3 = TMEM lane quarters 0-3
+    const int r = wq * 32 + lane;
+    const uint32_t lb = static_cast<uint32_t>(wq * 32) << 16;
+    int s_cnt = 0, uocc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      int bh, qt, nkv;
+      dq_unit<CAUSAL>(u, p.bh, p.tiles, bh, qt, nkv);
+      const int row = qt * kBlockM + r;  // < npad: padded vectors in range
+      const bool row_ok = row < p.n;
+      const int64_t grow = static_cast<int64_t>(bh) * p.n + row;
+      const int64_t prow = static_cast<int64_t>(bh) * p.npad + row;
+      const float nlse = -p.lse2[prow];
+      const float drow = p.dsum[prow];
+      for (int j = 0; j < nkv; ++j) {
+        ok = mbar_wait(bar(L::S_FULL), s_cnt & 1, wc, kRoleSoftmax);
+        ++s_cnt;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const bool mask = (j == nkv - 1) && (CAUSAL || (p.n & (kBlockN - 1)));
+        const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], dv[32];
+          tmem_ld_32x32b_x32(tS + lb + c * 32, sv);
+          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
+          tmem_wait_ld(sv);
+          reg_fence(dv);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k0 = c * 32 + 2 * i;
+            float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), p.c_log2, nlse));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), p.c_log2, nlse));
+            if (mask && k0 > limit) p0 = 0.f;
+            if (mask && k0 + 1 > limit) p1 = 0.f;
+            const float ds0 = p0 * (__uint_as_float(dv[2 * i]) - drow);
+            const float ds1 = p1 * (__uint_as_float(dv[2 * i + 1]) - drow);
+            pk[i] = pack_bf16x2(ds0, ds1);
+          }
+          tmem_st_32x32b_x16(tS + lb + c * 16, pk);  // dS over loaded S columns
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::DS_FULL));
+      }
+      if (!ok) break;
+      ok = mbar_wait(bar(L::ACC_FULL), uocc & 1, wc, kRoleEpilogue);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++uocc;
+      tc_fence_after_sync();
+      uint4 *out = reinterpret_cast<uint4 *>(p.dq + grow * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tdQ + lb + c * 32, o);
+        tmem_wait_ld(o);
+        uint32_t h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * p.scale,
+                             __uint_as_float(o[2 * i + 1]) * p.scale);
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            out[c * 4 + i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2],
+                                        h[4 * i + 3]);
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::ACC_EMPTY));
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ dK, dV
+
+template <int D>
+struct BwdDkvSmem {
+  static constexpr uint32_t kTile = Smem<D>::kTileBytes;
+  static constexpr uint32_t kPanel = Smem<D>::kPanelBytes;
+  static constexpr int kSub = D / 64;
+  static constexpr int kStages = (D == 128) ? 2 : 4;  // Q+dO+lse+D ring
+  // one stage: Q tile, dO tile, 128 lse, 128 D (fp32), 1024-aligned
+  static constexpr uint32_t kStage = 2 * kTile + 1024;
+  static constexpr uint32_t kK = 0, kV = kTile;
+  static constexpr uint32_t kRing = 2 * kTile;
+  static constexpr uint32_t kBars = kRing + kStages * kStage;
+  static constexpr int KV_FULL = 0, KV_EMPTY = 1, ST_FULL = 2, PDS_FULL = 3,
+                       ACC_FULL = 4, ACC_EMPTY = 5, DRAIN = 6, Q_FULL = 7,
+                       Q_EMPTY = Q_FULL + kStages,
+                       NUM_BARS = Q_EMPTY + kStages;
+  static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;
+  static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ void dkv_unit(int u, int bh_count, int tiles,
+                                         int &bh, int &kt, int &q_first) {
+  if (CAUSAL) {  // key tiles seen by the most queries first
+    kt = u / bh_count;
+    bh = u % bh_count;
+    q_first = kt;
+  } else {
+    bh = u / tiles;
+    kt = u % tiles;
+    q_first = 0;
+  }
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_lse,
+                         const __grid_constant__ CUtensorMap tm_dsum,
+                         const BwdParams p) {
+  using L = BwdDkvSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  auto bar = [&](int i) { return base + L::kBars + 8u * i; };
+
+  if (tid == 0) {
+    mbar_init(bar(L::KV_FULL), 1);
+    mbar_init(bar(L::KV_EMPTY), 1);
+    mbar_init(bar(L::ST_FULL), 1);
+    mbar_init(bar(L::PDS_FULL), 4);
+    mbar_init(bar(L::ACC_FULL), 1);
+    mbar_init(bar(L::ACC_EMPTY), 4);
+    mbar_init(bar(L::DRAIN), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::Q_FULL + s), 1);
+      mbar_init(bar(L::Q_EMPTY + s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+  // TMEM: S^T (0-127, P^T over it), dP^T (128-255, dS^T over it), dV, dK
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256,
+                 tdK = tmem + 256 + D;
+
+  if (warp == kBwdLoaderWarp) {
+    if (lane == 0) {
+      int uocc = 0, q_issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        int bh, kt, q0;
+        dkv_unit<CAUSAL>(u, p.bh, p.tiles, bh, kt, q0);
+        if (uocc > 0) {
+          ok = mbar_wait(bar(L::KV_EMPTY), (uocc - 1) & 1, wc, kRoleProducer);
+          if (!ok) break;
+        }
+        ++uocc;
+        mbar_arrive_expect_tx(bar(L::KV_FULL), 2 * L::kTile);
+        for (int s = 0; s < L::kSub; ++s) {
+          tma_load_3d(base + L::kK + s * L::kPanel, &tm_k, bar(L::KV_FULL), s * 64,
+                      kt * kBlockN, bh);
+          tma_load_3d(base + L::kV + s * L::kPanel, &tm_v, bar(L::KV_FULL), s * 64,
+                      kt * kBlockN, bh);
+        }
+        for (int i = q0; i < p.tiles; ++i) {
+          const int st = q_issued % L::kStages;
+          ok = mbar_wait(bar(L::Q_EMPTY + st), ((q_issued / L::kStages) & 1) ^ 1,
+                         wc, kRoleProducer);
+          if (!ok) break;
+          const uint32_t sb = base + L::kRing + st * L::kStage;
+          mbar_arrive_expect_tx(bar(L::Q_FULL + st), 2 * L::kTile + 1024);
+          for (int s = 0; s < L::kSub; ++s) {
+            tma_load_3d(sb + s * L::kPanel, &tm_q, bar(L::Q_FULL + st), s * 64,
+                        i * kBlockM, bh);
+            tma_load_3d(sb + L::kTile + s * L::kPanel, &tm_do, bar(L::Q_FULL + st),
+                        s * 64, i * kBlockM, bh);
+          }
+          tma_load_2d(sb + 2 * L::kTile, &tm_lse, bar(L::Q_FULL + st), i * kBlockM, bh);
+          tma_load_2d(sb + 2 * L::kTile + 512, &tm_dsum, bar(L::Q_FULL + st),
+                      i * kBlockM, bh);
+          ++q_issued;
+        }
+      }
+      if (*wc.abort) {
+        if (uocc > 0) mbar_wait_drain(bar(L::KV_FULL), (uocc - 1) & 1, wc);
+        for (int st = 0; st < L::kStages; ++st)
+          if (q_issued > st) {
+            const int last = st + ((q_issued - 1 - st) / L::kStages) * L::kStages;
+            mbar_wait_drain(bar(L::Q_FULL + st), (last / L::kStages) & 1, wc);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0) {
+      int uocc = 0, q_cons = 0, pds_cnt = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        int bh, kt, q0;
+        dkv_unit<CAUSAL>(u, p.bh, p.tiles, bh, kt, q0);
+        ok = mbar_wait_spin(bar(L::KV_FULL), uocc & 1, wc, kRoleMma);
+        if (!ok) break;
+        for (int i = q0; i < p.tiles; ++i) {
+          const int st = q_cons % L::kStages;
+          ok = mbar_wait_spin(bar(L::Q_FULL + st), (q_cons / L::kStages) & 1, wc,
+                              kRoleMma);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t sb = base + L::kRing + st * L::kStage;
+          // issued after the previous dV/dK MMAs in this thread: they have
+          // read P^T / dS^T before these overwrite the columns
+          issue_qk<D>(tS, base + L::kK, sb);             // S^T  = K Q^T
+          issue_qk<D>(tdP, base + L::kV, sb + L::kTile); // dP^T = V dO^T
+          mma_commit(bar(L::ST_FULL));
+          if (i == p.tiles - 1) mma_commit(bar(L::KV_EMPTY));  // last K, V read
+          ok = mbar_wait_spin(bar(L::PDS_FULL), pds_cnt & 1, wc, kRoleMma);
+          ++pds_cnt;
+          if (!ok) break;
+          if (i == q0 && uocc > 0) {
+            ok = mbar_wait_spin(bar(L::ACC_EMPTY), (uocc - 1) & 1, wc, kRoleMma);
+            if (!ok) break;
+          }
+          tc_fence_after_sync();
+          issue_pv<D>(tdV, tS, sb + L::kTile, i > q0);  // dV += P^T  dO
+          issue_pv<D>(tdK, tdP, sb, i > q0);            // dK += dS^T Q
+          mma_commit(bar(L::Q_EMPTY + st));
+          ++q_cons;
+        }
+        if (!ok) break;
+        mma_commit(bar(L::ACC_FULL));
+        ++uocc;
+      }
+      mma_commit(bar(L::DRAIN));
+      mbar_wait_drain(bar(L::DRAIN), 0, wc);
+    }
+    __syncwarp();
+  } else {
+    // compute warpgroup: thread = key row r of the tile
+    const int wq = warp;
+    const int r = wq * 32 + lane;
+    const uint32_t lb = static_cast<uint32_t>(wq * 32) << 16;
+    int s_cnt = 0, uocc = 0, q_cons = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      int bh, kt, q0;
+      dkv_unit<CAUSAL>(u, p.bh, p.tiles, bh, kt, q0);
+      for (int i = q0; i < p.tiles; ++i) {
+        const int st = q_cons % L::kStages;
+        ++q_cons;
+        ok = mbar_wait(bar(L::ST_FULL), s_cnt & 1, wc, kRoleSoftmax);
+        ++s_cnt;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after_sync();
+        // the stage's lse / D vectors were written by TMA: acquire them on
+        // the stage's own barrier (complete by now: the MMA waited on it)
+        ok = mbar_wait(bar(L::Q_FULL + st), ((q_cons - 1) / L::kStages) & 1, wc,
+                       kRoleSoftmax);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint32_t vec = base + L::kRing + st * L::kStage + 2 * L::kTile;
+        // causal: on the diagonal tile query c < key r is in the key's past
+        // of no query (P = 0); on the last tile queries >= N do not exist
+        const bool diag = CAUSAL && (i == kt);
+        const bool tail = (i == p.tiles - 1) && (p.n & (kBlockM - 1));
+        const int qlimit = p.n - 1 - i * kBlockM;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], dv[32];
+          tmem_ld_32x32b_x32(tS + lb + c * 32, sv);
+          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
+          tmem_wait_ld(sv);
+          reg_fence(dv);
+          uint32_t ppk[16], dpk[16];
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const float4 lv = ld_shared_f4(vec + (c * 32 + 4 * g) * 4);
+            const float4 dd = ld_shared_f4(vec + 512 + (c * 32 + 4 * g) * 4);
+            const float lse4[4] = {lv.x, lv.y, lv.z, lv.w};
+            const float d4[4] = {dd.x, dd.y, dd.z, dd.w};
+            float pv[4], dsv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int qc = c * 32 + 4 * g + e;  // query column in the tile
+              float pe = ex2_approx(fmaf(__uint_as_float(sv[4 * g + e]), p.c_log2,
+                                         -lse4[e]));
+              if ((diag && qc < r) || (tail && qc > qlimit)) pe = 0.f;
+              pv[e] = pe;
+              dsv[e] = pe * (__uint_as_float(dv[4 * g + e]) - d4[e]);
+            }
+            ppk[2 * g] = pack_bf16x2(pv[0], pv[1]);
+            ppk[2 * g + 1] = pack_bf16x2(pv[2], pv[3]);
+            dpk[2 * g] = pack_bf16x2(dsv[0], dsv[1]);
+            dpk[2 * g + 1] = pack_bf16x2(dsv[2], dsv[3]);
+          }
+          tmem_st_32x32b_x16(tS + lb + c * 16, ppk);   // P^T  over S^T
+          tmem_st_32x32b_x16(tdP + lb + c * 16, dpk);  // dS^T over dP^T
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::PDS_FULL));
+      }
+      if (!ok) break;
+      ok = mbar_wait(bar(L::ACC_FULL), uocc & 1, wc, kRoleEpilogue);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++uocc;
+      tc_fence_after_sync();
+      const int key = kt * kBlockN + r;
+      const bool row_ok = key < p.n;
+      const int64_t grow = static_cast<int64_t>(bh) * p.n + key;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t src = which ? tdK : tdV;
+        const float mul = which ? p.scale : 1.f;
+        uint4 *out = reinterpret_cast<uint4 *>((which ? p.dk : p.dv) + grow * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(src + lb + c * 32, o);
+          tmem_wait_ld(o);
+          uint32_t h[16];
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2)
+            h[i2] = pack_bf16x2(__uint_as_float(o[2 * i2]) * mul,
+                                __uint_as_float(o[2 * i2 + 1]) * mul);
+          if (row_ok) {
+#pragma unroll
+            for (int i2 = 0; i2 < 4; ++i2)
+              out[c * 4 + i2] = make_uint4(h[4 * i2], h[4 * i2 + 1],
+                                           h[4 * i2 + 2], h[4 * i2 + 3]);
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::ACC_EMPTY));
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace attn_b200

@@ -142,6 +142,35 @@ int attn_status(attn_stream_t stream);
 uint32_t attn_last_status_bits(void);
 
 /*
+ * attn_bwd -- backward pass of attn_fwd (gradients of O with respect to
+ * q, k, v), by recomputation: the marketmaker.cc post's section "Backward
+ * pass: menghitung ulang, bukan menyimpan" keeps only the forward's output
+ * and softmax statistics and recomputes the score tiles from Q and K.
+ *
+ *   q, k, v  the forward's inputs; o, lse its outputs (attn_fwd with the
+ *            same B, H, N, d, causal, scale); dout = dL/dO.  All bf16
+ *            [B, H, N, d] device buffers (16-byte aligned) except lse, fp32
+ *            [B, H, N] (4-byte aligned).
+ *   dq, dk, dv  outputs, bf16 [B, H, N, d] (16-byte aligned), written in
+ *            full: dq = scale * dS k, dk = scale * dS^T q, dv = P^T dout with
+ *            P = softmax(scale q k^T [mask]) and
+ *            dS = P * (dout v^T - rowsum(dout * o)).
+ *   workspace  device memory of at least attn_bwd_workspace_bytes(B, H, N)
+ *            bytes, 256-byte aligned, caller-owned, scratch for this call.
+ *
+ * Queued on `stream` like attn_fwd; device timeouts surface in attn_status.
+ * Outputs and workspace must not overlap any input or each other.
+ */
+int attn_bwd(const void *q, const void *k, const void *v, const void *o,
+             const void *dout, const float *lse, void *dq, void *dk, void *dv,
+             void *workspace, size_t workspace_bytes, int B, int H, int N,
+             int d, int causal, float scale, attn_stream_t stream);
+
+/* Workspace bytes attn_bwd needs (0 on bad sizes): two fp32 vectors of
+ * B * H * (N rounded up to 128) entries, each rounded up to 256 bytes. */
+size_t attn_bwd_workspace_bytes(int B, int H, int N);
+
+/*
  * attn_selftest_exp2 -- test hook for the kernel's exponentials.  For n
  * device floats x, writes y[i] = 2^x[i] as the attention kernel evaluates
  * it: mode 0 = the FMA-pipe polynomial (Cody-Waite split + degree-3 minimax,
