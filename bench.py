@@ -37,6 +37,7 @@ from exact_io_aware_73_b200 import replicas as R  # noqa: E402
 from exact_io_aware_73_b200 import workloads as W  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (bf16, causal/non-causal) and % of B200 dense BF16 peak"
+METRIC_BWD = "attention bwd TFLOP/s (bf16; 2.5 x forward FLOPs)"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
@@ -221,6 +222,115 @@ def run_reference(args, w):
     return 0
 
 
+def cpu_baseline_bwd(w, budget_s: float):
+    """fp64 backward oracle on a bounded slice of the workload: the first
+    2048 positions of up to (host cores) heads, one head per thread."""
+    import numpy as np
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    H = max(1, min(w.H * w.B, threads))
+    n = min(w.N, 2048)
+    sub = W.shape_case(1, H, n, w.d, w.causal, seed=w.seed)
+    q, k, v = (oracle.bf16_bits_to_f64(oracle.bf16_bits(t)) for t in W.make_qkv(sub))
+    do = np.random.default_rng(5).standard_normal(q.shape)
+    t0 = time.perf_counter()
+    oracle.attention_backward(q, k, v, do, w.causal, w.scale, threads)
+    dt = time.perf_counter() - t0
+    flops = 2.5 * sub.flops()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"fp64 backward of {H} heads x N={n}, d={w.d} "
+                      f"({'causal' if w.causal else 'non-causal'}), {dt:.1f} s"}
+
+
+def run_backward(args, w):
+    """Time attn_bwd (prep + dQ + dK/dV kernels) on the workload; one GPU."""
+    import torch
+    from exact_io_aware_73_b200 import attn
+    world, rank, local = R.env_ranks()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    R.init("nccl", world, device=dev)
+    q, k, v = (t.to(dev) for t in W.make_qkv(w, seed=R.rank_seed(w.seed, rank)))
+    g = torch.Generator().manual_seed(R.rank_seed(w.seed, rank) + 3)
+    dout = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    o, lse = attn.attn_fwd(q, k, v, causal=w.causal, scale=w.scale)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(attn.bwd_workspace_bytes(w.B, w.H, w.N), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    in_bytes = 6 * q.numel() * 2
+    flush = None if in_bytes > L2_BYTES else torch.empty(
+        2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        rc = attn.attn_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                               o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                               ws.data_ptr(), ws.numel(), w.B, w.H, w.N, w.d,
+                               w.causal, w.scale, sh)
+        if rc != 0:
+            raise attn.AttnError(rc, "attn_bwd")
+
+    for _ in range(args.warmup):
+        step()
+    if attn.status() != 0:
+        raise RuntimeError("device status after warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    evs = []
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        evs.append((a, b))
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if attn.status() != 0:
+        raise RuntimeError("device status after the timed region")
+    ms = R.max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
+    ms_per_step = ms / args.steps
+    flops = 2.5 * w.flops()
+    value = R.job_throughput(flops, world, ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    cb = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_baseline_bwd(w, args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC_BWD, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian/uniform bf16 inputs, N(0,1) dO)",
+            "config": {"workload": w.name, "pass": "bwd", "B": w.B, "H": w.H,
+                       "N": w.N, "d": w.d, "causal": w.causal,
+                       "l2": ("inputs larger than L2" if flush is None else
+                              "L2 flushed between steps (outside the events)"),
+                       "parallelism": f"{world} independent replicas"},
+            "roofline": {"bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+                         "traffic": None,
+                         "note": "FLOPs = 2.5 x forward (5 GEMMs); the kernels "
+                                 "run 7 (S and dP are recomputed in both the "
+                                 "dQ and the dK/dV kernel)"},
+            "cpu_baseline": cb, "e2e": None,
+            "gpu_launches": 3 * args.steps, "clocks": clk}), flush=True)
+    R.finish(world)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -228,6 +338,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd (default): the forward hot path; bwd: attn_bwd")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     args = ap.parse_args()
@@ -236,6 +348,8 @@ def main():
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.pass_ == "bwd":
+        return run_backward(args, w)
 
     import torch
     from exact_io_aware_73_b200 import attn
