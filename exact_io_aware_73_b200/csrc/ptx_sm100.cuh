@@ -1,6 +1,7 @@
 // ptx_sm100.cuh -- hand-written inline-PTX wrappers for sm_100a: mbarriers,
-// TMA tensor copies (no cluster multicast anywhere), bulk-async groups and
-// the tcgen05 tensor-core / tensor-memory instructions.
+// TMA tensor loads (no cluster multicast anywhere), the tcgen05 tensor-core /
+// tensor-memory instructions, register reallocation and a few packed-math
+// and conversion instructions.
 //
 // Only instructions are wrapped here; the attention kernel decides what to
 // do with them.  Each wrapper is a single PTX instruction (or a predicate
@@ -118,40 +119,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-
-// 3-D tiled store shared -> global; rows outside the tensor are clipped.
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map,
-                                             uint32_t src, int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, "
-      "%4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until the source shared memory of all committed bulk stores is read.
-__device__ __forceinline__ void bulk_wait_group_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// Wait until all committed bulk stores are complete.
-__device__ __forceinline__ void bulk_wait_group_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// Make generic-proxy shared-memory writes visible to the async proxy (TMA).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_barrier_sync(uint32_t id,
-                                                   uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -382,14 +349,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t d;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a,
-                                             uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a),
-               "r"(b), "r"(c), "r"(d)
-               : "memory");
 }
 
 }  // namespace attn_b200
