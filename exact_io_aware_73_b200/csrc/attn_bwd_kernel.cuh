@@ -99,8 +99,8 @@ struct BwdDqSmem {
   static constexpr uint32_t kV = kK + kStages * kTile;
   static constexpr uint32_t kBars = kV + kStages * kTile;
   static constexpr int Q_FULL = 0, Q_EMPTY = 1, S_FULL = 2, DS_FULL = 3,
-                       ACC_FULL = 4, ACC_EMPTY = 5, DRAIN = 6, KV_FULL = 7,
-                       KV_EMPTY = KV_FULL + kStages,
+                       ACC_FULL = 4, ACC_EMPTY = 5, DRAIN = 6, DP_FULL = 7,
+                       S_FREE = 8, KV_FULL = 9, KV_EMPTY = KV_FULL + kStages,
                        NUM_BARS = KV_EMPTY + kStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;
   static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
@@ -142,6 +142,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(L::Q_FULL), 1);
     mbar_init(bar(L::Q_EMPTY), 1);
     mbar_init(bar(L::S_FULL), 1);
+    mbar_init(bar(L::DP_FULL), 1);
+    mbar_init(bar(L::S_FREE), 4);
     mbar_init(bar(L::DS_FULL), 4);
     mbar_init(bar(L::ACC_FULL), 1);
     mbar_init(bar(L::ACC_EMPTY), 4);
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
-  // TMEM: S (cols 0-127, dS written over it), dP (128-255), dQ (256-256+D)
+  // TMEM: S (cols 0-127), dP (128-255, dS written over it), dQ (256-256+D)
   const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
 
   if (warp == kBwdLoaderWarp) {
@@ -211,40 +213,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == kBwdMmaWarp) {
     if (lane == 0) {
-      int uocc = 0, kv_cons = 0, ds_cnt = 0;
+      // Per K/V tile j: S_j and dP_j; the compute warps read S_j (P phase),
+      // release it (S_FREE) and form dS_j over dP_j (dS phase).  S_{j+1} is
+      // issued as soon as S_j is free, so it runs during the dS phase; dQ_j
+      // and dP_{j+1} run during the next P phase.
+      int uocc = 0, kv_cons = 0, jcnt = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         int bh, qt, nkv;
         dq_unit<CAUSAL>(u, p.bh, p.tiles, bh, qt, nkv);
         ok = mbar_wait_spin(bar(L::Q_FULL), uocc & 1, wc, kRoleMma);
         if (!ok) break;
+        auto stage_of = [&](int idx) { return idx % L::kStages; };
+        auto k_tile = [&](int idx) { return base + L::kK + stage_of(idx) * L::kTile; };
+        auto v_tile = [&](int idx) { return base + L::kV + stage_of(idx) * L::kTile; };
+        // prologue: S_0, dP_0
+        ok = mbar_wait_spin(bar(L::KV_FULL + stage_of(kv_cons)),
+                            (kv_cons / L::kStages) & 1, wc, kRoleMma);
+        if (!ok) break;
+        tc_fence_after_sync();
+        issue_qk<D>(tS, base + L::kQ, k_tile(kv_cons));     // S  = Q  K^T
+        mma_commit(bar(L::S_FULL));
+        issue_qk<D>(tdP, base + L::kDO, v_tile(kv_cons));   // dP = dO V^T
+        mma_commit(bar(L::DP_FULL));
+        if (nkv == 1) mma_commit(bar(L::Q_EMPTY));  // last read of Q, dO
         for (int j = 0; j < nkv; ++j) {
-          const int st = kv_cons % L::kStages;
-          ok = mbar_wait_spin(bar(L::KV_FULL + st), (kv_cons / L::kStages) & 1, wc,
-                              kRoleMma);
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint32_t k_s = base + L::kK + st * L::kTile;
-          const uint32_t v_s = base + L::kV + st * L::kTile;
-          // issued after the previous dQ MMA in this thread: it has read dS
-          // out of the S columns before they are overwritten
-          issue_qk<D>(tS, base + L::kQ, k_s);    // S  = Q  K^T
-          issue_qk<D>(tdP, base + L::kDO, v_s);  // dP = dO V^T
-          mma_commit(bar(L::S_FULL));
-          if (j == nkv - 1) mma_commit(bar(L::Q_EMPTY));  // last read of Q, dO
-          ok = mbar_wait_spin(bar(L::DS_FULL), ds_cnt & 1, wc, kRoleMma);
-          ++ds_cnt;
+          const int cur = kv_cons + j;
+          const int nxt = cur + 1;
+          if (j + 1 < nkv) {
+            ok = mbar_wait_spin(bar(L::KV_FULL + stage_of(nxt)),
+                                (nxt / L::kStages) & 1, wc, kRoleMma);
+            if (!ok) break;
+            ok = mbar_wait_spin(bar(L::S_FREE), (jcnt + j) & 1, wc, kRoleMma);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_qk<D>(tS, base + L::kQ, k_tile(nxt));
+            mma_commit(bar(L::S_FULL));
+          }
+          ok = mbar_wait_spin(bar(L::DS_FULL), (jcnt + j) & 1, wc, kRoleMma);
           if (!ok) break;
           if (j == 0 && uocc > 0) {
             ok = mbar_wait_spin(bar(L::ACC_EMPTY), (uocc - 1) & 1, wc, kRoleMma);
             if (!ok) break;
           }
           tc_fence_after_sync();
-          issue_pv<D>(tdQ, tS, k_s, j > 0);      // dQ += dS K
-          mma_commit(bar(L::KV_EMPTY + st));
-          ++kv_cons;
+          issue_pv<D>(tdQ, tdP, k_tile(cur), j > 0);   // dQ += dS K
+          mma_commit(bar(L::KV_EMPTY + stage_of(cur)));
+          if (j + 1 < nkv) {
+            // after dQ_j in this thread: dS_j has been read from these columns
+            issue_qk<D>(tdP, base + L::kDO, v_tile(nxt));
+            mma_commit(bar(L::DP_FULL));
+            if (j + 2 == nkv) mma_commit(bar(L::Q_EMPTY));  // last read of Q, dO
+          }
         }
         if (!ok) break;
+        kv_cons += nkv;
+        jcnt += nkv;
         mma_commit(bar(L::ACC_FULL));
         ++uocc;
       }
@@ -269,33 +293,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float nlse = -p.lse2[prow];
       const float drow = p.dsum[prow];
       for (int j = 0; j < nkv; ++j) {
+        // ---- P phase: P_j from S_j, kept in registers; S released
         ok = mbar_wait(bar(L::S_FULL), s_cnt & 1, wc, kRoleSoftmax);
-        ++s_cnt;
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after_sync();
         const bool mask = (j == nkv - 1) && (CAUSAL || (p.n & (kBlockN - 1)));
         const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
+        float pr[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32], dv[32];
+          uint32_t sv[32];
           tmem_ld_32x32b_x32(tS + lb + c * 32, sv);
-          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
           tmem_wait_ld(sv);
-          reg_fence(dv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float e = ex2_approx(fmaf(__uint_as_float(sv[i]), p.c_log2, nlse));
+            pr[c * 32 + i] = (mask && c * 32 + i > limit) ? 0.f : e;
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::S_FREE));
+        // ---- dS phase: dS_j = P_j (dP_j - D) written over dP_j
+        ok = mbar_wait(bar(L::DP_FULL), s_cnt & 1, wc, kRoleSoftmax);
+        ++s_cnt;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dv[32];
+          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
+          tmem_wait_ld(dv);
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int k0 = c * 32 + 2 * i;
-            float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), p.c_log2, nlse));
-            float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), p.c_log2, nlse));
-            if (mask && k0 > limit) p0 = 0.f;
-            if (mask && k0 + 1 > limit) p1 = 0.f;
-            const float ds0 = p0 * (__uint_as_float(dv[2 * i]) - drow);
-            const float ds1 = p1 * (__uint_as_float(dv[2 * i + 1]) - drow);
-            pk[i] = pack_bf16x2(ds0, ds1);
-          }
-          tmem_st_32x32b_x16(tS + lb + c * 16, pk);  // dS over loaded S columns
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(pr[c * 32 + 2 * i] * (__uint_as_float(dv[2 * i]) - drow),
+                                pr[c * 32 + 2 * i + 1] *
+                                    (__uint_as_float(dv[2 * i + 1]) - drow));
+          tmem_st_32x32b_x16(tdP + lb + c * 16, pk);  // over loaded dP columns
         }
         tmem_wait_st();
         tc_fence_before_sync();
@@ -353,9 +390,9 @@ struct BwdDkvSmem {
   static constexpr uint32_t kK = 0, kV = kTile;
   static constexpr uint32_t kRing = 2 * kTile;
   static constexpr uint32_t kBars = kRing + kStages * kStage;
-  static constexpr int KV_FULL = 0, KV_EMPTY = 1, ST_FULL = 2, PDS_FULL = 3,
-                       ACC_FULL = 4, ACC_EMPTY = 5, DRAIN = 6, Q_FULL = 7,
-                       Q_EMPTY = Q_FULL + kStages,
+  static constexpr int KV_FULL = 0, KV_EMPTY = 1, S_FULL = 2, DP_FULL = 3,
+                       P_READY = 4, DS_READY = 5, ACC_FULL = 6, ACC_EMPTY = 7,
+                       DRAIN = 8, Q_FULL = 9, Q_EMPTY = Q_FULL + kStages,
                        NUM_BARS = Q_EMPTY + kStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;
   static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
@@ -398,8 +435,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (tid == 0) {
     mbar_init(bar(L::KV_FULL), 1);
     mbar_init(bar(L::KV_EMPTY), 1);
-    mbar_init(bar(L::ST_FULL), 1);
-    mbar_init(bar(L::PDS_FULL), 4);
+    mbar_init(bar(L::S_FULL), 1);
+    mbar_init(bar(L::DP_FULL), 1);
+    mbar_init(bar(L::P_READY), 4);
+    mbar_init(bar(L::DS_READY), 4);
     mbar_init(bar(L::ACC_FULL), 1);
     mbar_init(bar(L::ACC_EMPTY), 4);
     mbar_init(bar(L::DRAIN), 1);
@@ -473,40 +512,65 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == kBwdMmaWarp) {
     if (lane == 0) {
-      int uocc = 0, q_cons = 0, pds_cnt = 0;
+      // Per Q tile i: S^T_i and dP^T_i; the compute warps form P^T_i over
+      // S^T_i (P phase, P_READY), then dS^T_i over dP^T_i (dS phase,
+      // DS_READY).  dV_i and S^T_{i+1} run during the dS phase, dK_i and
+      // dP^T_{i+1} during the next P phase.  Each MMA that overwrites S^T or
+      // dP^T is issued after the one reading P^T or dS^T from those columns.
+      int uocc = 0, q_cons = 0, tcnt = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         int bh, kt, q0;
         dkv_unit<CAUSAL>(u, p.bh, p.tiles, bh, kt, q0);
         ok = mbar_wait_spin(bar(L::KV_FULL), uocc & 1, wc, kRoleMma);
         if (!ok) break;
+        auto ring = [&](int idx) {
+          return base + L::kRing + (idx % L::kStages) * L::kStage;
+        };
+        // prologue: S^T and dP^T of the first Q tile
+        ok = mbar_wait_spin(bar(L::Q_FULL + q_cons % L::kStages),
+                            (q_cons / L::kStages) & 1, wc, kRoleMma);
+        if (!ok) break;
+        tc_fence_after_sync();
+        issue_qk<D>(tS, base + L::kK, ring(q_cons));               // S^T  = K Q^T
+        mma_commit(bar(L::S_FULL));
+        issue_qk<D>(tdP, base + L::kV, ring(q_cons) + L::kTile);   // dP^T = V dO^T
+        mma_commit(bar(L::DP_FULL));
+        if (q0 == p.tiles - 1) mma_commit(bar(L::KV_EMPTY));  // last K, V read
         for (int i = q0; i < p.tiles; ++i) {
-          const int st = q_cons % L::kStages;
-          ok = mbar_wait_spin(bar(L::Q_FULL + st), (q_cons / L::kStages) & 1, wc,
-                              kRoleMma);
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint32_t sb = base + L::kRing + st * L::kStage;
-          // issued after the previous dV/dK MMAs in this thread: they have
-          // read P^T / dS^T before these overwrite the columns
-          issue_qk<D>(tS, base + L::kK, sb);             // S^T  = K Q^T
-          issue_qk<D>(tdP, base + L::kV, sb + L::kTile); // dP^T = V dO^T
-          mma_commit(bar(L::ST_FULL));
-          if (i == p.tiles - 1) mma_commit(bar(L::KV_EMPTY));  // last K, V read
-          ok = mbar_wait_spin(bar(L::PDS_FULL), pds_cnt & 1, wc, kRoleMma);
-          ++pds_cnt;
+          const int cur = q_cons + (i - q0);
+          const int nxt = cur + 1;
+          const int t = tcnt + (i - q0);
+          ok = mbar_wait_spin(bar(L::P_READY), t & 1, wc, kRoleMma);
           if (!ok) break;
           if (i == q0 && uocc > 0) {
             ok = mbar_wait_spin(bar(L::ACC_EMPTY), (uocc - 1) & 1, wc, kRoleMma);
             if (!ok) break;
           }
           tc_fence_after_sync();
-          issue_pv<D>(tdV, tS, sb + L::kTile, i > q0);  // dV += P^T  dO
-          issue_pv<D>(tdK, tdP, sb, i > q0);            // dK += dS^T Q
-          mma_commit(bar(L::Q_EMPTY + st));
-          ++q_cons;
+          issue_pv<D>(tdV, tS, ring(cur) + L::kTile, i > q0);  // dV += P^T dO
+          if (i + 1 < p.tiles) {
+            ok = mbar_wait_spin(bar(L::Q_FULL + nxt % L::kStages),
+                                (nxt / L::kStages) & 1, wc, kRoleMma);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_qk<D>(tS, base + L::kK, ring(nxt));
+            mma_commit(bar(L::S_FULL));
+          }
+          ok = mbar_wait_spin(bar(L::DS_READY), t & 1, wc, kRoleMma);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_pv<D>(tdK, tdP, ring(cur), i > q0);            // dK += dS^T Q
+          mma_commit(bar(L::Q_EMPTY + cur % L::kStages));
+          if (i + 1 < p.tiles) {
+            issue_qk<D>(tdP, base + L::kV, ring(nxt) + L::kTile);
+            mma_commit(bar(L::DP_FULL));
+            if (i + 2 == p.tiles) mma_commit(bar(L::KV_EMPTY));  // last K, V read
+          }
         }
         if (!ok) break;
+        q_cons += p.tiles - q0;
+        tcnt += p.tiles - q0;
         mma_commit(bar(L::ACC_FULL));
         ++uocc;
       }
@@ -527,8 +591,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int i = q0; i < p.tiles; ++i) {
         const int st = q_cons % L::kStages;
         ++q_cons;
-        ok = mbar_wait(bar(L::ST_FULL), s_cnt & 1, wc, kRoleSoftmax);
-        ++s_cnt;
+        // ---- P phase: P^T_i from S^T_i, kept in fp32 registers, and bf16
+        // P^T written over the S^T columns already read
+        ok = mbar_wait(bar(L::S_FULL), s_cnt & 1, wc, kRoleSoftmax);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after_sync();
@@ -544,42 +609,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool diag = CAUSAL && (i == kt);
         const bool tail = (i == p.tiles - 1) && (p.n & (kBlockM - 1));
         const int qlimit = p.n - 1 - i * kBlockM;
+        float pr[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32], dv[32];
+          uint32_t sv[32];
           tmem_ld_32x32b_x32(tS + lb + c * 32, sv);
-          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
           tmem_wait_ld(sv);
-          reg_fence(dv);
-          uint32_t ppk[16], dpk[16];
+          uint32_t ppk[16];
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
             const float4 lv = ld_shared_f4(vec + (c * 32 + 4 * g) * 4);
-            const float4 dd = ld_shared_f4(vec + 512 + (c * 32 + 4 * g) * 4);
             const float lse4[4] = {lv.x, lv.y, lv.z, lv.w};
-            const float d4[4] = {dd.x, dd.y, dd.z, dd.w};
-            float pv[4], dsv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int qc = c * 32 + 4 * g + e;  // query column in the tile
               float pe = ex2_approx(fmaf(__uint_as_float(sv[4 * g + e]), p.c_log2,
                                          -lse4[e]));
               if ((diag && qc < r) || (tail && qc > qlimit)) pe = 0.f;
-              pv[e] = pe;
-              dsv[e] = pe * (__uint_as_float(dv[4 * g + e]) - d4[e]);
+              pr[qc] = pe;
             }
-            ppk[2 * g] = pack_bf16x2(pv[0], pv[1]);
-            ppk[2 * g + 1] = pack_bf16x2(pv[2], pv[3]);
-            dpk[2 * g] = pack_bf16x2(dsv[0], dsv[1]);
-            dpk[2 * g + 1] = pack_bf16x2(dsv[2], dsv[3]);
+            ppk[2 * g] = pack_bf16x2(pr[c * 32 + 4 * g], pr[c * 32 + 4 * g + 1]);
+            ppk[2 * g + 1] = pack_bf16x2(pr[c * 32 + 4 * g + 2], pr[c * 32 + 4 * g + 3]);
           }
-          tmem_st_32x32b_x16(tS + lb + c * 16, ppk);   // P^T  over S^T
+          tmem_st_32x32b_x16(tS + lb + c * 16, ppk);   // P^T over S^T
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::P_READY));
+        // ---- dS phase: dS^T_i = P^T_i (dP^T_i - D) written over dP^T_i
+        ok = mbar_wait(bar(L::DP_FULL), s_cnt & 1, wc, kRoleSoftmax);
+        ++s_cnt;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dv[32];
+          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
+          tmem_wait_ld(dv);
+          uint32_t dpk[16];
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const float4 dd = ld_shared_f4(vec + 512 + (c * 32 + 4 * g) * 4);
+            const int q4 = c * 32 + 4 * g;
+            dpk[2 * g] = pack_bf16x2(pr[q4] * (__uint_as_float(dv[4 * g]) - dd.x),
+                                     pr[q4 + 1] * (__uint_as_float(dv[4 * g + 1]) - dd.y));
+            dpk[2 * g + 1] =
+                pack_bf16x2(pr[q4 + 2] * (__uint_as_float(dv[4 * g + 2]) - dd.z),
+                            pr[q4 + 3] * (__uint_as_float(dv[4 * g + 3]) - dd.w));
+          }
           tmem_st_32x32b_x16(tdP + lb + c * 16, dpk);  // dS^T over dP^T
         }
         tmem_wait_st();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::PDS_FULL));
+        if (lane == 0) mbar_arrive(bar(L::DS_READY));
       }
       if (!ok) break;
       ok = mbar_wait(bar(L::ACC_FULL), uocc & 1, wc, kRoleEpilogue);
