@@ -132,3 +132,28 @@ def sample_rows(w: Workload, count: int, seed: int = 7):
     r = torch.randint(0, total, (max(0, count - len(picks)),), generator=g)
     picks.update(int(x) for x in r)
     return sorted(picks)
+
+
+# ------------------------------------------------------------ FP8 inputs
+
+def make_signs(seed: int, d: int) -> torch.Tensor:
+    """The random signs of the randomized Hadamard rotation: d entries of
+    +-1 (int8), drawn from a seeded generator.  They are an input of the FP8
+    path (both sides receive the same draw)."""
+    bits = torch.randint(0, 2, (d,), generator=_gen(seed), dtype=torch.int64)
+    return (1 - 2 * bits).to(torch.int8)
+
+
+def add_channel_outliers(x: torch.Tensor, channels, factor: float) -> torch.Tensor:
+    """Outlier features: the given coordinates of every row multiplied by
+    ``factor`` (in fp32, then rounded to bf16 again).  Large, persistent
+    per-channel magnitudes are the pattern that spoils plain FP8
+    quantization of Q and K."""
+    y = x.float()
+    y[..., list(channels)] *= float(factor)
+    return y.to(torch.bfloat16)
+
+
+def outlier_channels(seed: int, d: int, count: int):
+    """``count`` distinct coordinates in [0, d), drawn from a seeded generator."""
+    return sorted(int(c) for c in torch.randperm(d, generator=_gen(seed))[:count])

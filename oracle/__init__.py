@@ -23,4 +23,11 @@ from .oracle import (  # noqa: F401
     bf16_bits_to_f64,
     max_threads,
     library_path,
+    e4m3_encode,
+    e4m3_decode,
+    hadamard_rotate,
+    fp8_quantize,
+    attention_fp8,
+    attention_fp8_rows,
+    quantize_qkv_fp8,
 )

@@ -43,6 +43,22 @@ def _load():
         lib.oracle_attention_blocked_f64.argtypes = [
             dp, dp, dp, dp, dp, i64, i64, i64, i64, ctypes.c_int,
             ctypes.c_double, i64, i64]
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        i8p = ctypes.POINTER(ctypes.c_int8)
+        fp = ctypes.POINTER(ctypes.c_float)
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode_array.argtypes = [fp, i64, u8p]
+        lib.oracle_hadamard_rotate.argtypes = [dp, i64, i64, i8p, dp]
+        lib.oracle_fp8_quantize.argtypes = [u16p, i64, i64, i64, ctypes.c_int,
+                                            i8p, i64, u8p, dp]
+        lib.oracle_attention_fp8_rows.argtypes = [
+            u8p, dp, u8p, dp, u8p, dp, i64, i64, i64, ctypes.c_int,
+            ctypes.c_double, i64, i64, i64, i64p, i64, dp, dp, ctypes.c_double,
+            dp, ctypes.c_int]
+        for f in (lib.oracle_e4m3_encode_array, lib.oracle_hadamard_rotate,
+                  lib.oracle_fp8_quantize, lib.oracle_attention_fp8_rows):
+            f.restype = ctypes.c_int
         for f in (lib.oracle_softmax_row, lib.oracle_attend_scores,
                   lib.oracle_attention_f64, lib.oracle_attention_rows_bf16,
                   lib.oracle_attention_blocked_f64, lib.oracle_max_threads):
@@ -166,3 +182,118 @@ def attention_backward(q, k, v, do, causal: bool, scale: float, threads=None):
         _dptr(dv), B, H, N, d, int(bool(causal)), float(scale),
         _threads(threads)), "attention_backward")
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- FP8 path
+# FP8 attention with incoherent processing (fp8_oracle.c): E4M3 codes,
+# randomized Hadamard rotation of Q and K, power-of-two block scales, and the
+# blocked online softmax with E4M3 probabilities.
+
+def _u8ptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 codes (round to nearest even, saturating) of float32 values."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    _check(_load().oracle_e4m3_encode_array(
+        x.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), x.size, _u8ptr(out)),
+        "e4m3_encode")
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values (float64) of E4M3 codes."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    table = np.array([_load().oracle_e4m3_decode(c) for c in range(256)])
+    return table[codes]
+
+
+def _signs(signs, d):
+    signs = np.ascontiguousarray(signs, dtype=np.int8)
+    if signs.shape != (d,) or not np.all(np.abs(signs) == 1):
+        raise ValueError("signs must be d entries of +-1")
+    return signs
+
+
+def hadamard_rotate(x, signs) -> np.ndarray:
+    """x diag(signs) H (unscaled Sylvester Hadamard) for rows of x [..., d]."""
+    x = _f64(x)
+    d = x.shape[-1]
+    signs = _signs(signs, d)
+    y = np.empty_like(x)
+    _check(_load().oracle_hadamard_rotate(
+        _dptr(x), x.size // d, d,
+        signs.ctypes.data_as(ctypes.POINTER(ctypes.c_int8)), _dptr(y)),
+        "hadamard_rotate")
+    return y
+
+
+def fp8_quantize(bits, rotate: bool, signs=None, block_rows: int = 128):
+    """Block quantization of bf16 bit patterns [B, H, N, d] (or [BH, N, d]):
+    returns (codes uint8 same shape, scales float64 [BH, ceil(N/block_rows)])."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    N, d = bits.shape[-2], bits.shape[-1]
+    BH = bits.size // (N * d)
+    nblk = -(-N // int(block_rows))
+    codes = np.empty(bits.shape, dtype=np.uint8)
+    scales = np.empty((BH, nblk))
+    sp = None
+    if rotate:
+        signs = _signs(signs, d)
+        sp = signs.ctypes.data_as(ctypes.POINTER(ctypes.c_int8))
+    _check(_load().oracle_fp8_quantize(
+        bits.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)), BH, N, d,
+        int(bool(rotate)), sp, int(block_rows), _u8ptr(codes), _dptr(scales)),
+        "fp8_quantize")
+    return codes, scales
+
+
+def attention_fp8_rows(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
+                       scale: float, rows, block: int = 128, flip_delta=0.0,
+                       threads=None):
+    """FP8 attention on codes [.., N, d] for flat rows (bh * N + i); Q and K
+    scales per `block` rows, V one scale per head.  Returns (O, lse,
+    flip_bound) with flip_bound None unless flip_delta > 0."""
+    q8, k8, v8 = (np.ascontiguousarray(a, dtype=np.uint8) for a in (q8, k8, v8))
+    N, d = q8.shape[-2], q8.shape[-1]
+    BH = q8.size // (N * d)
+    qs, ks, vs = (_f64(a).reshape(BH, -1) for a in (q_scale, k_scale, v_scale))
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    O = np.empty((rows.size, d))
+    lse = np.empty(rows.size)
+    fb = np.empty(rows.size) if flip_delta > 0 else None
+    _check(_load().oracle_attention_fp8_rows(
+        _u8ptr(q8), _dptr(qs), _u8ptr(k8), _dptr(ks), _u8ptr(v8), _dptr(vs),
+        BH, N, d, int(bool(causal)), float(scale), int(block), int(block), 128,
+        rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.size,
+        _dptr(O), _dptr(lse), float(flip_delta),
+        _dptr(fb) if fb is not None else None, _threads(threads)),
+        "attention_fp8_rows")
+    return O, lse, fb
+
+
+def attention_fp8(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
+                  scale: float, block: int = 128, flip_delta=0.0, threads=None):
+    """attention_fp8_rows over every row; O shaped like the codes."""
+    shape = q8.shape
+    N, d = shape[-2], shape[-1]
+    rows = np.arange(q8.size // d, dtype=np.int64)
+    O, lse, fb = attention_fp8_rows(q8, q_scale, k8, k_scale, v8, v_scale,
+                                    causal, scale, rows, block, flip_delta,
+                                    threads)
+    return (O.reshape(shape), lse.reshape(shape[:-1]),
+            None if fb is None else fb.reshape(shape[:-1]))
+
+
+def quantize_qkv_fp8(qbits, kbits, vbits, rotate: bool, signs=None):
+    """The method's quantization of one problem: Q and K rotated (if asked)
+    and quantized per 128-row tile, V per head.  Returns a dict of codes and
+    scales plus the softmax-scale multiplier of the rotated problem."""
+    d = qbits.shape[-1]
+    q8, qs = fp8_quantize(qbits, rotate, signs, 128)
+    k8, ks = fp8_quantize(kbits, rotate, signs, 128)
+    v8, vs = fp8_quantize(vbits, False, None, vbits.shape[-2])
+    return dict(q8=q8, qs=qs, k8=k8, ks=ks, v8=v8, vs=vs,
+                gain=(1.0 / d) if rotate else 1.0)

@@ -1,8 +1,10 @@
 """The oracle's pins must catch plausible mistakes.
 
-Each case copies ``oracle/attention_oracle.c``, plants one mistake (a dropped
-term, a wrong sign or index, a swapped operand, a misplaced mask boundary),
-compiles the copy on the CPU and runs ``tests/test_oracle_pins.py`` against
+Each case copies one oracle source (``oracle/attention_oracle.c`` or
+``oracle/fp8_oracle.c``), plants one mistake (a dropped term, a wrong sign or
+index, a swapped operand, a misplaced mask boundary, a wrong rounding rule),
+compiles it with the other source unchanged on the CPU and runs the matching
+pin file (``tests/test_oracle_pins.py``, the backward or the FP8 pins) against
 it.  The pins pass on the real oracle (that file's own run) and must fail on
 every mutant.  Mistakes are chosen so that every memory access stays in
 bounds.
@@ -16,9 +18,11 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "attention_oracle.c")
+FP8_SRC = os.path.join(ROOT, "oracle", "fp8_oracle.c")
 
 PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 BACKWARD_PINS = os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")
+FP8_PINS = os.path.join(ROOT, "tests", "test_oracle_fp8_pins.py")
 
 MUTANTS = {
     "mask_hides_diagonal": ("return causal ? (i + 1) : N;",
@@ -54,17 +58,45 @@ BACKWARD_MUTANTS = {
                       "const int64_t n = causal ? (i + 1 < N ? i + 2 : N) : N;\n    const double *qi = Q + i * d, *doi"),
 }
 
+# planted mistakes in the FP8 oracle; each must fail an FP8 pin
+FP8_MUTANTS = {
+    "fp8_ties_away_from_even": ("else pick = (lo & 1) ? hi : lo;",
+                                "else pick = hi;"),
+    "fp8_subnormal_scale": ("v = ldexp((double)man, -9);",
+                            "v = ldexp((double)man, -10);"),
+    "fp8_signs_ignored": ("acc += x[a] * (double)s[a] * hadamard_entry(a, t);",
+                          "acc += x[a] * hadamard_entry(a, t);"),
+    "fp8_hadamard_or": ("(popcount_u32((uint32_t)(a & t)) & 1)",
+                        "(popcount_u32((uint32_t)(a | t)) & 1)"),
+    "fp8_scale_half_range": ("while (ldexp(amax, e) > E4M3_MAX) --e;",
+                             "while (ldexp(amax, e) > E4M3_MAX / 2) --e;"),
+    "fp8_no_probability_offset": ("const double p = 256.0 * exp(s[c - k0] - m);",
+                                  "const double p = exp(s[c - k0] - m);"),
+    "fp8_sum_of_rounded_p": ("      l += p;\n",
+                             "      l += oracle_e4m3_decode(oracle_e4m3_encode((float)p));\n"),
+    "fp8_no_output_rescale": ("for (int64_t t = 0; t < d; ++t) acc[t] *= alpha;", ""),
+    "fp8_mask_leak": ("const int64_t kend = causal ? i + 1 : N;",
+                      "const int64_t kend = causal ? (i + 2 < N ? i + 2 : N) : N;"),
+    "fp8_first_q_scale_only": ("q_scale[bh * qblocks + i / q_block]",
+                               "q_scale[bh * qblocks]"),
+}
+
 
 def _build_mutant(name, tmpdir):
-    old, new = {**MUTANTS, **BACKWARD_MUTANTS}[name]
-    src = open(SRC).read()
+    if name in FP8_MUTANTS:
+        old, new = FP8_MUTANTS[name]
+        target, other = FP8_SRC, SRC
+    else:
+        old, new = {**MUTANTS, **BACKWARD_MUTANTS}[name]
+        target, other = SRC, FP8_SRC
+    src = open(target).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
     path_c = os.path.join(tmpdir, f"{name}.c")
     path_so = os.path.join(tmpdir, f"{name}.so")
     with open(path_c, "w") as f:
         f.write(src.replace(old, new))
     subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
-                    path_c, "-o", path_so, "-lm"], check=True)
+                    path_c, other, "-o", path_so, "-lm"], check=True)
     return path_so
 
 
@@ -96,3 +128,9 @@ def test_every_planted_backward_mistake_fails_a_backward_pin():
     with tempfile.TemporaryDirectory() as tmp:
         survivors = _run_against(BACKWARD_MUTANTS, BACKWARD_PINS, tmp)
         assert not survivors, f"backward pins did not catch: {survivors}"
+
+
+def test_every_planted_fp8_mistake_fails_an_fp8_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        survivors = _run_against(FP8_MUTANTS, FP8_PINS, tmp)
+        assert not survivors, f"FP8 pins did not catch: {survivors}"
