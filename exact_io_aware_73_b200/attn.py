@@ -238,3 +238,124 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False,
                       _stream_handle(stream))
     _check(rc, "attn_bwd")
     return dq, dk, dv
+
+
+# ------------------------------------------------------------------ FP8 path
+
+def _fp8_fns():
+    L = lib()
+    if L.attn_fwd_fp8.argtypes is None:
+        vp, i, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
+        L.attn_fp8_quantize.argtypes = [vp, vp, vp, vp, i, i, i, i, i, u64, u64,
+                                        i, vp]
+        L.attn_fp8_quantize.restype = i
+        L.attn_fwd_fp8_quantized.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i,
+                                             i, i, i, i, ctypes.c_float, vp]
+        L.attn_fwd_fp8_quantized.restype = i
+        L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i,
+                                   ctypes.c_float, i, u64, u64, vp,
+                                   ctypes.c_size_t, vp]
+        L.attn_fwd_fp8.restype = i
+        L.attn_fwd_fp8_workspace_bytes.argtypes = [i, i, i, i]
+        L.attn_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
+    return L
+
+
+def sign_mask(signs) -> tuple[int, int]:
+    """(sign_lo, sign_hi) bit masks of a +-1 sequence of length <= 128:
+    bit t set where signs[t] == -1."""
+    lo = hi = 0
+    for t, s in enumerate(int(x) for x in signs):
+        if s not in (1, -1):
+            raise ValueError("signs must be +-1")
+        if s < 0:
+            if t < 64:
+                lo |= 1 << t
+            else:
+                hi |= 1 << (t - 64)
+    return lo, hi
+
+
+def fp8_workspace_bytes(B, H, N, d) -> int:
+    return int(_fp8_fns().attn_fwd_fp8_workspace_bytes(B, H, N, d))
+
+
+def fp8_quantize_raw(x, x8, scales, tile_amax, B, H, N, d, rotate, sign_lo,
+                     sign_hi, per_head, stream_handle) -> int:
+    return _fp8_fns().attn_fp8_quantize(x, x8, scales, tile_amax, int(B), int(H),
+                                        int(N), int(d), int(bool(rotate)),
+                                        int(sign_lo), int(sign_hi),
+                                        int(bool(per_head)), stream_handle)
+
+
+def fp8_quantize(x, rotate: bool, signs=None, per_head: bool = False,
+                 stream=None):
+    """E4M3 codes (uint8, same shape) and fp32 scales of a bf16 CUDA tensor
+    [B, H, N, 128]: per 128-row tile ([B, H, ceil(N/128)]) or per head
+    ([B, H]); Q and K rotated with the signs when `rotate`."""
+    import torch
+    B, H, N, d = x.shape
+    lo, hi = sign_mask(signs) if rotate else (0, 0)
+    tiles = -(-N // 128)
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty((B, H) if per_head else (B, H, tiles),
+                         dtype=torch.float32, device=x.device)
+    amax = (torch.empty((B, H, tiles), dtype=torch.float32, device=x.device)
+            if per_head else None)
+    rc = fp8_quantize_raw(x.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                          amax.data_ptr() if amax is not None else None,
+                          B, H, N, d, rotate, lo, hi, per_head,
+                          _stream_handle(stream))
+    _check(rc, "attn_fp8_quantize")
+    return codes, scales
+
+
+def attn_fwd_fp8_quantized(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
+                           scale: float, stream=None):
+    """O (bf16), lse of the FP8 attention on quantized operands; `scale` is
+    the softmax scale of the problem the codes encode."""
+    import torch
+    B, H, N, d = q8.shape
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    rc = _fp8_fns().attn_fwd_fp8_quantized(
+        q8.data_ptr(), q_scale.data_ptr(), k8.data_ptr(), k_scale.data_ptr(),
+        v8.data_ptr(), v_scale.data_ptr(), o.data_ptr(), lse.data_ptr(),
+        B, H, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
+    _check(rc, "attn_fwd_fp8_quantized")
+    return o, lse
+
+
+def attn_fwd_fp8_raw(q, k, v, o, lse, B, H, N, d, causal, scale, rotate,
+                     sign_lo, sign_hi, ws, ws_bytes, stream_handle) -> int:
+    return _fp8_fns().attn_fwd_fp8(q, k, v, o, lse, int(B), int(H), int(N),
+                                   int(d), int(bool(causal)), float(scale),
+                                   int(bool(rotate)), int(sign_lo),
+                                   int(sign_hi), ws, ws_bytes, stream_handle)
+
+
+def attn_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None,
+                 signs=None, workspace=None, out=None, lse=None, stream=None):
+    """FP8 attention forward of bf16 CUDA tensors [B, H, N, 128]: Q and K
+    rotated with `signs` (+-1, length 128; None = no rotation, naive FP8)
+    and block-quantized to E4M3 with V, then the FP8 kernel.  Returns
+    (O bf16, lse fp32)."""
+    import torch
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    lo, hi = sign_mask(signs) if signs is not None else (0, 0)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    need = fp8_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    rc = attn_fwd_fp8_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                          out.data_ptr(), lse.data_ptr(), B, H, N, d, causal,
+                          scale, signs is not None, lo, hi,
+                          workspace.data_ptr(), workspace.numel(),
+                          _stream_handle(stream))
+    _check(rc, "attn_fwd_fp8")
+    return out, lse

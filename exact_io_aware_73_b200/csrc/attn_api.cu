@@ -15,6 +15,7 @@
 
 #include "attn_b200.h"
 #include "attn_bwd_kernel.cuh"
+#include "fp8_quant_kernel.cuh"
 
 namespace {
 
@@ -29,7 +30,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   uint32_t *status = nullptr;  // 4-byte device status word, lazily allocated
-  bool smem_attr_set[4] = {false, false, false, false};
+  bool smem_attr_set[6] = {false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
 };
 
@@ -171,11 +172,28 @@ int encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *ptr, int bh,
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_TENSOR_MAP;
 }
 
-template <int D, bool CAUSAL>
+// E4M3 codes [B*H, N, d] as a 3-D byte tensor; boxes of 128 x 128 rows
+// (one 128-byte swizzle panel per row at d = 128).
+int encode_map_u8(EncodeTiledFn enc, CUtensorMap *map, const void *ptr, int bh,
+                  int N, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                           static_cast<cuuint64_t>(N) * d};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr),
+                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_TENSOR_MAP;
+}
+
+template <int D, bool CAUSAL, bool FP8 = false>
 int launch(DeviceState &st, int variant, const CUtensorMap *maps,
            const FwdParams &p, cudaStream_t stream) {
-  auto kern = attn_b200::attn_fwd_sm100_kernel<D, CAUSAL>;
-  const uint32_t smem = Smem<D>::kAlloc;
+  auto kern = attn_b200::attn_fwd_sm100_kernel<D, CAUSAL, FP8>;
+  const uint32_t smem = Smem<D, FP8>::kAlloc;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!st.smem_attr_set[variant]) {
@@ -242,6 +260,32 @@ int launch_bwd(DeviceState &st, int variant, const CUtensorMap *m,
   kdkv<<<grid, kBwdThreads, smem_dkv, stream>>>(m[0], m[1], m[2], m[3], m[4], m[5], p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
+}
+
+// One fp8_quant_kernel launch over every 128-row tile of every head: one
+// persistent CTA per SM (or per tile, when there are fewer tiles).
+int launch_quant(DeviceState &st, const attn_b200::QuantParams &p, int mode,
+                 cudaStream_t stream) {
+  const int64_t tiles = static_cast<int64_t>(p.bh) * p.tiles;
+  const int grid = static_cast<int>(tiles < st.sm_count ? tiles : st.sm_count);
+  attn_b200::fp8_quant_kernel<128><<<grid, attn_b200::kQuantThreads, 0, stream>>>(p, mode);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+// Size checks shared by the FP8 entries (no CUDA calls).
+int check_fp8_sizes(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0) return ATTN_ERR_INVALID_SIZE;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  if (N > ATTN_MAX_SEQ || bh > ATTN_MAX_HEADS) return ATTN_ERR_INVALID_SIZE;
+  if (bh * ((N + 255) / 256) > 0x7fffffffLL || bh * ((N + 127) / 128) > 0x7fffffffLL)
+    return ATTN_ERR_INVALID_SIZE;
+  return ATTN_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
 
 __global__ void exp2_selftest_kernel(const float *x, float *y, int n, int mode) {
@@ -431,6 +475,152 @@ int attn_bwd(const void *q, const void *k, const void *v, const void *o,
                   : launch_bwd<128, false>(*st, 1, maps, p, s);
   return causal ? launch_bwd<64, true>(*st, 2, maps, p, s)
                 : launch_bwd<64, false>(*st, 3, maps, p, s);
+}
+
+int attn_fp8_quantize(const void *x, void *x8, float *scales, float *tile_amax,
+                      int B, int H, int N, int d, int rotate, uint64_t sign_lo,
+                      uint64_t sign_hi, int per_head, attn_stream_t stream) {
+  int rc = check_fp8_sizes(B, H, N, d);
+  if (rc != ATTN_OK || B == 0 || H == 0 || N == 0) return rc;
+  if (!x || !x8 || !scales || (per_head && !tile_amax)) return ATTN_ERR_NULL_POINTER;
+  if (!aligned(x, 16) || !aligned(x8, 16) || !aligned(scales, 4) ||
+      (tile_amax && !aligned(tile_amax, 4)))
+    return ATTN_ERR_MISALIGNED;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  const int tiles = (N + 127) / 128;
+  const size_t xb = static_cast<size_t>(bh) * N * d * 2, cb = xb / 2;
+  const size_t sb = static_cast<size_t>(per_head ? bh : bh * tiles) * 4;
+  const size_t ab = static_cast<size_t>(bh) * tiles * 4;
+  if (overlaps(x8, cb, x, xb) || overlaps(scales, sb, x, xb) ||
+      overlaps(scales, sb, x8, cb) ||
+      (per_head && (overlaps(tile_amax, ab, x, xb) || overlaps(tile_amax, ab, x8, cb) ||
+                    overlaps(tile_amax, ab, scales, sb))))
+    return ATTN_ERR_ALIAS;
+  int dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  if (!is_device_memory_of(x, dev) || !is_device_memory_of(x8, dev) ||
+      !is_device_memory_of(scales, dev) ||
+      (per_head && !is_device_memory_of(tile_amax, dev)))
+    return ATTN_ERR_NOT_DEVICE_MEMORY;
+  attn_b200::QuantParams p;
+  p.x = static_cast<const uint16_t *>(x);
+  p.codes = static_cast<uint8_t *>(x8);
+  p.scales = scales;
+  p.tile_amax = tile_amax;
+  p.sign_lo = sign_lo;
+  p.sign_hi = sign_hi;
+  p.bh = static_cast<int>(bh);
+  p.n = N;
+  p.tiles = tiles;
+  p.rotate = rotate ? 1 : 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!per_head) return launch_quant(*st, p, attn_b200::kQuantPerTile, s);
+  if ((rc = launch_quant(*st, p, attn_b200::kQuantAmaxOnly, s)) != ATTN_OK) return rc;
+  return launch_quant(*st, p, attn_b200::kQuantPerHead, s);
+}
+
+int attn_fwd_fp8_quantized(const void *q8, const float *q_scale,
+                           const void *k8, const float *k_scale,
+                           const void *v8, const float *v_scale, void *o,
+                           float *lse, int B, int H, int N, int d, int causal,
+                           float scale, attn_stream_t stream) {
+  int rc = check_fp8_sizes(B, H, N, d);
+  if (rc != ATTN_OK) return rc;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID_SCALE;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!q8 || !q_scale || !k8 || !k_scale || !v8 || !v_scale || !o || !lse)
+    return ATTN_ERR_NULL_POINTER;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(q_scale, 4) || !aligned(k_scale, 4) ||
+      !aligned(v_scale, 4))
+    return ATTN_ERR_MISALIGNED;
+  const int64_t bh64 = static_cast<int64_t>(B) * H;
+  const int tiles = (N + 127) / 128;
+  const size_t cb = static_cast<size_t>(bh64) * N * d;
+  const size_t ob = cb * 2, lb = static_cast<size_t>(bh64) * N * 4;
+  const size_t tsb = static_cast<size_t>(bh64) * tiles * 4, vsb = bh64 * 4;
+  const void *ins[6] = {q8, k8, v8, q_scale, k_scale, v_scale};
+  const size_t in_bytes[6] = {cb, cb, cb, tsb, tsb, vsb};
+  for (int a = 0; a < 6; ++a)
+    if (overlaps(o, ob, ins[a], in_bytes[a]) || overlaps(lse, lb, ins[a], in_bytes[a]))
+      return ATTN_ERR_ALIAS;
+  if (overlaps(o, ob, lse, lb)) return ATTN_ERR_ALIAS;
+  int dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  const void *all[8] = {q8, k8, v8, q_scale, k_scale, v_scale, o, lse};
+  for (const void *ptr : all)
+    if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
+  EncodeTiledFn enc;
+  if ((rc = get_encode_fn(&enc)) != ATTN_OK) return rc;
+  const int bh = B * H;
+  CUtensorMap maps[3];
+  if ((rc = encode_map_u8(enc, &maps[0], q8, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map_u8(enc, &maps[1], k8, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map_u8(enc, &maps[2], v8, bh, N, d)) != ATTN_OK) return rc;
+  FwdParams p;
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.status = st->status;
+  p.bh = bh;
+  p.n = N;
+  p.num_units = bh * ((N + 255) / 256);
+  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.timeout_ns = g_timeout_ns.load();
+  p.debug_flags = 0;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.tiles = tiles;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return causal ? launch<128, true, true>(*st, 4, maps, p, s)
+                : launch<128, false, true>(*st, 5, maps, p, s);
+}
+
+size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d) {
+  if (check_fp8_sizes(B, H, N, d) != ATTN_OK) return 0;
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t tiles = (static_cast<size_t>(N) + 127) / 128;
+  return 3 * round256(bh * N * d) + 3 * round256(bh * tiles * 4) + round256(bh * 4);
+}
+
+int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
+                 float *lse, int B, int H, int N, int d, int causal,
+                 float scale, int rotate, uint64_t sign_lo, uint64_t sign_hi,
+                 void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+  int rc = check_fp8_sizes(B, H, N, d);
+  if (rc != ATTN_OK) return rc;
+  if ((rc = check_args(q, k, v, o, lse, B, H, N, d, scale, true)) != ATTN_OK) return rc;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  const size_t need = attn_fwd_fp8_workspace_bytes(B, H, N, d);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+    return ATTN_ERR_WORKSPACE;
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t tb = bh * N * d * 2, lb = bh * N * 4;
+  const void *bufs[5] = {q, k, v, o, lse};
+  const size_t bytes[5] = {tb, tb, tb, tb, lb};
+  for (int a = 0; a < 5; ++a)
+    if (overlaps(workspace, need, bufs[a], bytes[a])) return ATTN_ERR_ALIAS;
+  const size_t tiles = (static_cast<size_t>(N) + 127) / 128;
+  const size_t cbr = round256(bh * N * d), tsr = round256(bh * tiles * 4);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint8_t *q8 = ws, *k8 = ws + cbr, *v8 = ws + 2 * cbr;
+  float *qs = reinterpret_cast<float *>(ws + 3 * cbr);
+  float *ks = reinterpret_cast<float *>(ws + 3 * cbr + tsr);
+  float *vamax = reinterpret_cast<float *>(ws + 3 * cbr + 2 * tsr);
+  float *vs = reinterpret_cast<float *>(ws + 3 * cbr + 3 * tsr);
+  if ((rc = attn_fp8_quantize(q, q8, qs, nullptr, B, H, N, d, rotate, sign_lo,
+                              sign_hi, 0, stream)) != ATTN_OK ||
+      (rc = attn_fp8_quantize(k, k8, ks, nullptr, B, H, N, d, rotate, sign_lo,
+                              sign_hi, 0, stream)) != ATTN_OK ||
+      (rc = attn_fp8_quantize(v, v8, vs, vamax, B, H, N, d, 0, 0, 0, 1, stream)) !=
+          ATTN_OK)
+    return rc;
+  // unscaled Hadamard: (Q D H)(K D H)^T = d Q K^T
+  const float scale_qk = rotate ? scale / static_cast<float>(d) : scale;
+  return attn_fwd_fp8_quantized(q8, qs, k8, ks, v8, vs, o, lse, B, H, N, d, causal,
+                                scale_qk, stream);
 }
 
 int attn_status(attn_stream_t stream) {

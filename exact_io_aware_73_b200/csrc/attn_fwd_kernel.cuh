@@ -46,6 +46,17 @@
 //   * every wait is bounded in time; a wait that runs out records it in a
 //     device status word, the CTA drains its in-flight copies, frees its
 //     tensor memory and exits.
+//
+// FP8 variant (template flag FP8; [MM] "FA3: Mekanika hopper" item 3): Q, K,
+// V arrive as E4M3 codes with power-of-two block scales (one per 128-row Q /
+// K tile, one per head for V).  Both GEMMs run as tcgen05.mma kind::f8f6f4
+// (K = 32 per instruction, 128-byte rows = one swizzle panel at d = 128).  The
+// score multiplier scale * log2(e) * q_scale * k_scale changes per K tile;
+// the running max is exact (every increase rescales O), and P is carried as
+// 2^(x - m + 8) <= 256 so that E4M3's smallest code still reaches 2^-17 of
+// the row maximum; P goes to TMEM as four E4M3 bytes per column.  The row
+// sum adds the unrounded P; V's per-head scale multiplies the output in the
+// epilogue and lse subtracts the 2^8 again.
 #pragma once
 
 #include <cstdint>
@@ -137,22 +148,36 @@ struct FwdParams {
   float c_log2;        // scale * log2(e)
   unsigned long long timeout_ns;
   uint32_t debug_flags;  // bit 0: first CTA skips its first Q copy
+  // FP8 variant only: dequantization scales (powers of two)
+  const float *q_scale;  // [BH, tiles] one per 128-row Q tile
+  const float *k_scale;  // [BH, tiles] one per 128-row K tile
+  const float *v_scale;  // [BH] one per head
+  int tiles;             // ceil(n / 128)
 };
 
-// Shared-memory map (offsets from a 1024-byte aligned base).
-template <int D>
+// Pairs of FP8 exponentials (out of 8) evaluated on the FMA pipe.
+#ifndef ATTN_EXP2_EMU_PER8_FP8
+#define ATTN_EXP2_EMU_PER8_FP8 0
+#endif
+
+// Shared-memory map (offsets from a 1024-byte aligned base).  Tiles are
+// 128 rows of D elements (2 bytes, or 1 for FP8), in 128-byte-wide panels.
+template <int D, bool FP8 = false>
 struct Smem {
-  static constexpr int kSub = D / 64;                         // 64-col panels
+  static constexpr int kElem = FP8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kElem;
+  static constexpr int kSub = kRowBytes / 128;                // 128-byte panels
+  static constexpr int kPanelElems = 128 / kElem;             // elements per panel row
   static constexpr uint32_t kPanelBytes = kBlockM * 128;      // 128 rows x 128 B
-  static constexpr uint32_t kTileBytes = kBlockM * D * 2;     // one Q/K/V tile
+  static constexpr uint32_t kTileBytes = kBlockM * kRowBytes; // one Q/K/V tile
   // Ring depths.  K_j is released as soon as both S MMAs of iteration j are
   // issued, V_j only after both P.V MMAs, so V needs the deeper ring to be
   // refilled a full iteration ahead.
 #ifndef ATTN_V_STAGES_D128
 #define ATTN_V_STAGES_D128 2
 #endif
-  static constexpr int kKStages = (D == 128) ? 2 : 4;
-  static constexpr int kVStages = (D == 128) ? ATTN_V_STAGES_D128 : 4;
+  static constexpr int kKStages = (kRowBytes == 256) ? 2 : 4;
+  static constexpr int kVStages = (kRowBytes == 256) ? ATTN_V_STAGES_D128 : 4;
   static constexpr uint32_t kQ = 0;                           // 2 Q tiles
   static constexpr uint32_t kK = kQ + 2 * kTileBytes;         // K ring
   static constexpr uint32_t kV = kK + kKStages * kTileBytes;  // V ring
@@ -275,14 +300,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr,
 // P.V MMAs).
 constexpr int kLoadQK = 1, kLoadV = 2;
 
-template <int D, bool CAUSAL, int MODE>
+template <int D, bool CAUSAL, int MODE, bool FP8>
 __device__ __forceinline__ void producer_role(uint32_t base,
                                               const CUtensorMap *tq,
                                               const CUtensorMap *tk,
                                               const CUtensorMap *tv,
                                               const FwdParams &p,
                                               const WaitCtx &wc) {
-  using L = Smem<D>;
+  using L = Smem<D, FP8>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   int qocc[2] = {0, 0};     // non-empty occurrences of each Q tile so far
   int q_issued[2] = {0, 0};
@@ -309,7 +334,8 @@ __device__ __forceinline__ void producer_role(uint32_t base,
       mbar_arrive_expect_tx(bar(L::Q_FULL + t), L::kTileBytes);
       for (int s = 0; s < L::kSub; ++s)
         tma_load_3d_hint(base + L::kQ + t * L::kTileBytes + s * L::kPanelBytes,
-                         tq, bar(L::Q_FULL + t), s * 64, w.q0 + kBlockM * t,
+                         tq, bar(L::Q_FULL + t), s * L::kPanelElems,
+                         w.q0 + kBlockM * t,
                          w.bh, pol_q);
       ++q_issued[t];
     }
@@ -324,7 +350,8 @@ __device__ __forceinline__ void producer_role(uint32_t base,
         mbar_arrive_expect_tx(bar(L::K_FULL + ks), L::kTileBytes);
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d_hint(base + L::kK + ks * L::kTileBytes + s * L::kPanelBytes,
-                           tk, bar(L::K_FULL + ks), s * 64, j * kBlockN, w.bh,
+                           tk, bar(L::K_FULL + ks), s * L::kPanelElems,
+                           j * kBlockN, w.bh,
                            pol_kv);
         ++k_issued;
       }
@@ -336,7 +363,8 @@ __device__ __forceinline__ void producer_role(uint32_t base,
         mbar_arrive_expect_tx(bar(L::V_FULL + vs), L::kTileBytes);
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d_hint(base + L::kV + vs * L::kTileBytes + s * L::kPanelBytes,
-                           tv, bar(L::V_FULL + vs), s * 64, j * kBlockN, w.bh,
+                           tv, bar(L::V_FULL + vs), s * L::kPanelElems,
+                           j * kBlockN, w.bh,
                            pol_kv);
         ++v_issued;
       }
@@ -363,45 +391,57 @@ __device__ __forceinline__ void producer_role(uint32_t base,
 
 // ------------------------------------------------------------------ MMA
 
-template <int D>
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem,
                                          uint32_t k_smem) {
-  // S[128 x 128] = Q[128 x D] K[128 x D]^T; both K-major, 128B swizzle.
-  constexpr uint32_t idesc = (1u << 4)              // D: f32
-                             | (1u << 7)            // A: bf16
-                             | (1u << 10)           // B: bf16
+  // S[128 x 128] = Q[128 x D] K[128 x D]^T; both K-major, 128B swizzle.  One
+  // instruction covers 32 bytes of K (16 bf16 or 32 E4M3 elements).
+  constexpr uint32_t idesc = (1u << 4)                           // D: f32
+                             | ((FP8 ? 0u : 1u) << 7)            // A: bf16 | e4m3
+                             | ((FP8 ? 0u : 1u) << 10)           // B: bf16 | e4m3
                              | ((uint32_t)(kBlockN >> 3) << 17)  // N
                              | ((uint32_t)(kBlockM >> 4) << 24); // M
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * Smem<D>::kPanelBytes + (kk & 3) * 32;
-    mma_bf16_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024),
+  for (int kk = 0; kk < Smem<D, FP8>::kRowBytes / 32; ++kk) {
+    const uint32_t off = (kk >> 2) * Smem<D, FP8>::kPanelBytes + (kk & 3) * 32;
+    if constexpr (FP8)
+      mma_f8_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024),
                 smem_desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
+    else
+      mma_bf16_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024),
+                  smem_desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
   }
 }
 
-template <int D>
+template <int D, bool FP8 = false>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
                                          uint32_t v_smem, bool accumulate) {
-  // O[128 x D] (+)= P[128 x 128] V[128 x D]; P in TMEM (K-major, bf16
-  // packed two per column), V MN-major (D contiguous) with 128B swizzle:
-  // 64-wide D panels are kPanelBytes apart (LBO), 8-key groups 1024 B (SBO).
-  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10)
+  // O[128 x D] (+)= P[128 x 128] V[128 x D]; P in TMEM (K-major: bf16 two per
+  // column, or E4M3 four per column), V MN-major (D contiguous) with 128B
+  // swizzle: 128-byte-wide D panels are kPanelBytes apart (LBO), 8-key
+  // groups 1024 B (SBO).  One instruction covers 16 keys (bf16) or 32 (E4M3):
+  // 8 TMEM columns of P and 16 or 32 rows of V.
+  constexpr uint32_t idesc = (1u << 4) | ((FP8 ? 0u : 1u) << 7) |
+                             ((FP8 ? 0u : 1u) << 10)
                              | (1u << 16)           // B: MN-major
                              | ((uint32_t)(D >> 3) << 17)
                              | ((uint32_t)(kBlockM >> 4) << 24);
+  constexpr int kKeys = FP8 ? 32 : 16;
 #pragma unroll
-  for (int kk = 0; kk < kBlockN / 16; ++kk) {
-    mma_bf16_ts(d_tmem, p_tmem + kk * 8,
-                smem_desc_sw128(v_smem + kk * 2048, Smem<D>::kPanelBytes, 1024),
-                idesc, (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < kBlockN / kKeys; ++kk) {
+    const uint64_t bdesc =
+        smem_desc_sw128(v_smem + kk * kKeys * 128, Smem<D, FP8>::kPanelBytes, 1024);
+    if constexpr (FP8)
+      mma_f8_ts(d_tmem, p_tmem + kk * 8, bdesc, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    else
+      mma_bf16_ts(d_tmem, p_tmem + kk * 8, bdesc, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8>
 __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
                                          const FwdParams &p, const WaitCtx &wc) {
-  using L = Smem<D>;
+  using L = Smem<D, FP8>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   const uint32_t tS[2] = {tmem + 0, tmem + 128};
   const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
@@ -427,7 +467,7 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
       tc_fence_after_sync();
       for (int t = 0; t < 2; ++t)
         if (nt[t] > 0) {
-          issue_qk<D>(tS[t], sQ[t], base + L::kK + ks * L::kTileBytes);
+          issue_qk<D, FP8>(tS[t], sQ[t], base + L::kK + ks * L::kTileBytes);
           mma_commit(bar(L::S_FULL + t));
           if (nt[t] == 1) mma_commit(bar(L::Q_EMPTY + t));  // last read of Q_t
         }
@@ -452,7 +492,7 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
           if (!ok) break;
         }
         tc_fence_after_sync();
-        issue_pv<D>(tO[t], tS[t], base + L::kV + vs * L::kTileBytes, j > 0);
+        issue_pv<D, FP8>(tO[t], tS[t], base + L::kV + vs * L::kTileBytes, j > 0);
         mma_commit(bar(L::O_FULL + t));
         if (j + 1 < nt[t]) {
           if (!k_ready) {
@@ -464,7 +504,7 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
           }
           // issued after this tile's P.V in the same thread: the tensor pipe
           // reads P before this MMA overwrites the S columns holding it
-          issue_qk<D>(tS[t], sQ[t], base + L::kK + ks * L::kTileBytes);
+          issue_qk<D, FP8>(tS[t], sQ[t], base + L::kK + ks * L::kTileBytes);
           mma_commit(bar(L::S_FULL + t));
           if (j + 2 == nt[t]) mma_commit(bar(L::Q_EMPTY + t));  // last read of Q_t
         }
@@ -565,12 +605,47 @@ __device__ __forceinline__ float exp_row(const uint32_t (&s)[4][32], float cl2,
   return (a0 + a1) + (b0 + b1);
 }
 
-template <int D, bool CAUSAL>
+// FP8 version of exp_row: p = 2^(s * c - m) (m already lowered by 8, so
+// p <= 256), row sum of the unrounded p, and four E4M3 codes per 32-bit
+// column for the P.V MMA (key 4c in the lowest byte of column c).
+__device__ __forceinline__ float exp_row_fp8(const uint32_t (&s)[4][32], float c,
+                                             float m, uint32_t (&pk)[32]) {
+  const uint64_t c2 = f32x2(c, c);
+  const uint64_t nm2 = f32x2(-m, -m);
+  uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    float pv[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int e0 = 4 * q + 2 * h;
+      const float s0 = __uint_as_float(s[e0 >> 5][e0 & 31]);
+      const float s1 = __uint_as_float(s[(e0 + 1) >> 5][(e0 + 1) & 31]);
+      const uint64_t x2 = fma_f32x2(f32x2(s0, s1), c2, nm2);
+      float x0, x1;
+      f32x2_split(x2, x0, x1);
+      uint64_t p2;
+      if (((2 * q + h) & 7) < ATTN_EXP2_EMU_PER8_FP8)
+        p2 = exp2_poly_x2(x0, x1);
+      else
+        p2 = f32x2(ex2_approx(x0), ex2_approx(x1));
+      acc[h] = add_f32x2(acc[h], p2);
+      f32x2_split(p2, pv[2 * h], pv[2 * h + 1]);
+    }
+    pk[q] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
+  }
+  float a0, a1, b0, b1;
+  f32x2_split(acc[0], a0, a1);
+  f32x2_split(acc[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+template <int D, bool CAUSAL, bool FP8>
 __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
                                              const FwdParams &p,
                                              const WaitCtx &wc, int warp,
                                              int lane) {
-  using L = Smem<D>;
+  using L = Smem<D, FP8>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   const int t = warp >> 2;          // which Q tile of the unit
   const int wq = warp & 3;          // TMEM lane quarter of this warp
@@ -589,8 +664,18 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     const int qs = w.q0 + kBlockM * t;
     float m_run = -CUDART_INF_F;  // running max, log2 units (x = s * scale * log2 e)
     float l_run = 0.f;            // running sum of exp2(x - m_run)
+    // FP8: the Q tile's scale joins the score multiplier; V's is applied at
+    // the end (both are powers of two, so these products are exact)
+    float cq = cl2, v_mul = 1.f;
+    if constexpr (FP8) {
+      cq = cl2 * __ldg(p.q_scale + static_cast<int64_t>(w.bh) * p.tiles + (qs >> 7));
+      v_mul = __ldg(p.v_scale + w.bh);
+    }
+    const float* ksc = FP8 ? p.k_scale + static_cast<int64_t>(w.bh) * p.tiles : nullptr;
 
     for (int j = 0; j < n; ++j) {
+      // K tile j's score multiplier, read before the wait hides its latency
+      const float c = FP8 ? cq * __ldg(ksc + j) : cl2;
       ok = mbar_wait(bar(L::S_FULL + t), scnt & 1, wc, kRoleSoftmax);
       ++scnt;
       ok = __all_sync(0xffffffffu, ok);
@@ -600,20 +685,22 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
       const bool mask = (j == n - 1) && (CAUSAL || (p.n & (kBlockN - 1)));
       const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
       uint32_t s[4][32];
-      uint32_t pk[2][32];
       load_scores(tS, s, mask, limit);
 
       // Row max and the lazy base update: the base only moves when some row
       // of the warp gains more than 2^8 (warp-uniform decision, per-row
       // values); P then stays below 256 and O / l is unchanged because m and
       // l always move together.  The first tile of a row sets the base.
-      const float m_tile = row_max_raw(s) * cl2;
+      // FP8 keeps the exact running max (threshold 0): with P in E4M3 the
+      // base fixes which probabilities fall below the smallest code.
+      const float m_tile = row_max_raw(s) * c;
       float alpha = 1.f;
       bool update = false;
       if (j == 0) {
         m_run = m_tile;
       } else {
-        update = __any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold);
+        update = __any_sync(0xffffffffu,
+                            m_tile > m_run + (FP8 ? 0.f : kRescaleThreshold));
         if (update) {
           const float m_new = fmaxf(m_run, m_tile);
           alpha = ex2_approx(m_run - m_new);
@@ -621,9 +708,17 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
           m_run = m_new;
         }
       }
-      const float row_sum = exp_row<D>(s, cl2, m_run, pk);
-      tmem_st_32x32b_x32(tS + 0, pk[0]);
-      tmem_st_32x32b_x32(tS + 32, pk[1]);
+      float row_sum;
+      if constexpr (FP8) {
+        uint32_t pk[32];
+        row_sum = exp_row_fp8(s, c, m_run - 8.f, pk);
+        tmem_st_32x32b_x32(tS + 0, pk);
+      } else {
+        uint32_t pk[2][32];
+        row_sum = exp_row<D>(s, c, m_run, pk);
+        tmem_st_32x32b_x32(tS + 0, pk[0]);
+        tmem_st_32x32b_x32(tS + 32, pk[1]);
+      }
       l_run += row_sum;
       // O holds the earlier P.V products; the S_FULL commit for this tile was
       // issued after the previous P.V, so that MMA has completed.
@@ -641,7 +736,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     tc_fence_after_sync();
-    const float inv_l = __frcp_rn(l_run);
+    const float inv_l = __frcp_rn(l_run) * v_mul;
     const bool row_ok = qs + r < p.n;
     uint4 *orow = reinterpret_cast<uint4 *>(
         p.o + (static_cast<int64_t>(w.bh) * p.n + qs + r) * D);
@@ -667,19 +762,19 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     if (lane == 0) mbar_arrive(bar(L::O_EMPTY + t));  // O columns reusable
     if (row_ok)
       p.lse[static_cast<int64_t>(w.bh) * p.n + qs + r] =
-          (m_run + lg2_approx(l_run)) * kLn2;
+          (m_run - (FP8 ? 8.f : 0.f) + lg2_approx(l_run)) * kLn2;
   }
 }
 
 // ------------------------------------------------------------------ kernel
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const FwdParams p) {
-  using L = Smem<D>;
+  using L = Smem<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -727,17 +822,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role<D, CAUSAL>(base, tmem, p, wc, warp, lane);
+    softmax_role<D, CAUSAL, FP8>(base, tmem, p, wc, warp, lane);
   } else {
     setmaxnreg_dec<kControlRegs>();
     if (warp == kProducerWarp) {
       if (lane == 0)
-        producer_role<D, CAUSAL, kLoadQK>(base, &tm_q, &tm_k, &tm_v, p, wc);
+        producer_role<D, CAUSAL, kLoadQK, FP8>(base, &tm_q, &tm_k, &tm_v, p, wc);
     } else if (warp == kVLoaderWarp) {
       if (lane == 0)
-        producer_role<D, CAUSAL, kLoadV>(base, &tm_q, &tm_k, &tm_v, p, wc);
+        producer_role<D, CAUSAL, kLoadV, FP8>(base, &tm_q, &tm_k, &tm_v, p, wc);
     } else if (warp == kMmaWarp) {
-      if (lane == 0) mma_role<D, CAUSAL>(base, tmem, p, wc);
+      if (lane == 0) mma_role<D, CAUSAL, FP8>(base, tmem, p, wc);
     }
     __syncwarp();
   }

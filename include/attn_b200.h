@@ -225,6 +225,92 @@ int attn_fwd_host_noalloc(const void *q, const void *k, const void *v,
                           void *o, float *lse, int B, int H, int N, int d,
                           int causal, float scale, attn_stream_t stream);
 
+/*
+ * FP8 forward with incoherent processing -- the marketmaker.cc post's
+ * section "FA3: Mekanika hopper", item 3: naive FP8 attention is spoiled by
+ * outliers, so Q and K are rotated at random before block quantization,
+ * spreading an outlier's magnitude over all coordinates.
+ *
+ * Definitions used by the three entries below:
+ *   E4M3       OCP FP8 E4M3 ("fn": largest finite 448, no infinities),
+ *              round to nearest even, saturating.
+ *   rotation   x -> x diag(s) H for every row x of length d: s_t = -1 where
+ *              bit t of the 128-bit sign mask (sign_lo bits 0-63, sign_hi
+ *              bits 64-127) is set, else +1; H the unscaled d x d Sylvester
+ *              Hadamard matrix, H[a][t] = (-1)^popcount(a & t), H H^T = d I.
+ *              Computed in fp64 (exact for bf16 rows), then rounded to fp32.
+ *   block      one scale per block of rows: the largest 2^e (e <= 126) with
+ *              amax * 2^e <= 448, amax = the block's largest |value| after
+ *              rotation; codes = E4M3(value * 2^e); stored scale = 2^-e (the
+ *              dequantization multiplier).  Q and K: blocks of 128 rows
+ *              (scales [B, H, ceil(N/128)]); V: one block per head (scales
+ *              [B, H]).
+ *   attention  O = softmax(scale_qk * Qhat Khat^T [causal mask]) Vhat on the
+ *              dequantized operands (Qhat = codes * scale, ...), computed as
+ *              the blocked online softmax in 128-key blocks with an exact
+ *              running maximum m (log2 units): P = 2^(x - m + 8) <= 256 is
+ *              rounded to E4M3 for the P.V product, the row sum adds the
+ *              unrounded P, and lse = ln(sum_j exp(scale_qk Qhat_i . Khat_j))
+ *              (fp32, natural log) -- independent of the rounding of P.
+ * The three entries exist for head dimension d = 128 only (at d = 64 the
+ * exponentials, not the tensor cores, bound the forward, and FP8 buys
+ * nothing); other d give ATTN_ERR_UNSUPPORTED_HEAD_DIM.
+ */
+
+/*
+ * attn_fp8_quantize -- block-quantize one bf16 tensor x [B, H, N, 128] to
+ * E4M3 codes x8 [B, H, N, 128] (1 byte each) and fp32 scales.
+ *   rotate     nonzero: rotate every row with the sign mask first (Q, K).
+ *   per_head   0: one scale per 128-row tile, scales [B, H, ceil(N/128)];
+ *              nonzero: one per head, scales [B, H], and tile_amax must
+ *              point to B * H * ceil(N/128) floats of device scratch (the
+ *              first of the two launches stores each tile's amax there).
+ *              tile_amax may be NULL when per_head is 0.
+ * x and x8 16-byte aligned, scales and tile_amax 4-byte aligned, all device
+ * memory of the current device; x8, scales and tile_amax must not overlap x
+ * or each other.  Queued on `stream`.
+ */
+int attn_fp8_quantize(const void *x, void *x8, float *scales, float *tile_amax,
+                      int B, int H, int N, int d, int rotate, uint64_t sign_lo,
+                      uint64_t sign_hi, int per_head, attn_stream_t stream);
+
+/*
+ * attn_fwd_fp8_quantized -- the FP8 attention on quantized operands.
+ *   q8, k8, v8     E4M3 codes [B, H, N, 128], 16-byte aligned.
+ *   q_scale, k_scale  fp32 [B, H, ceil(N/128)] per-tile scales;
+ *   v_scale        fp32 [B, H] per-head scales.  Scales must be powers of
+ *                  two (as attn_fp8_quantize writes them).
+ *   scale          scale_qk of the definition above: the softmax scale of
+ *                  the problem the codes encode (for rotated Q and K that is
+ *                  the original scale / d, because H is unscaled).
+ *   o, lse         outputs as attn_fwd's: bf16 [B, H, N, 128], fp32 [B, H, N].
+ * Same launch, error and status behaviour as attn_fwd.
+ */
+int attn_fwd_fp8_quantized(const void *q8, const float *q_scale,
+                           const void *k8, const float *k_scale,
+                           const void *v8, const float *v_scale, void *o,
+                           float *lse, int B, int H, int N, int d, int causal,
+                           float scale, attn_stream_t stream);
+
+/*
+ * attn_fwd_fp8 -- the whole FP8 path from bf16 inputs: quantize Q and K
+ * (rotated when `rotate` is nonzero, per 128-row tile) and V (per head)
+ * into `workspace`, then attn_fwd_fp8_quantized with scale / d (rotated) or
+ * scale (not rotated).  q, k, v, o, lse as attn_fwd (d = 128); workspace:
+ * device memory of at least attn_fwd_fp8_workspace_bytes(B, H, N, d) bytes,
+ * 256-byte aligned, caller-owned scratch for this call, not overlapping any
+ * other argument.  Four kernels are queued on `stream` (two for V).
+ */
+int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
+                 float *lse, int B, int H, int N, int d, int causal,
+                 float scale, int rotate, uint64_t sign_lo, uint64_t sign_hi,
+                 void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/* Workspace bytes attn_fwd_fp8 needs (0 on bad sizes or d != 128): three
+ * code tensors of B*H*N*d bytes and four fp32 vectors of scales and tile
+ * maxima, each rounded up to 256 bytes. */
+size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
+
 /* Human-readable text for an error code (static string, never NULL). */
 const char *attn_strerror(int code);
 

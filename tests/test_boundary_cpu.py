@@ -134,3 +134,41 @@ def test_python_binding_has_no_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(a, "_lib", None)
     with pytest.raises(ImportError):
         a.lib()
+
+
+def test_fp8_entries_refuse_bad_arguments_without_a_device(attn):
+    far = 1 << 40
+    # d other than 128
+    assert attn.fp8_quantize_raw(far, 2 * far, 3 * far, None, 1, 1, 16, 64, 1,
+                                 0, 0, 0, None) == 3
+    # per-head quantization needs the tile-amax scratch
+    assert attn.fp8_quantize_raw(far, 2 * far, 3 * far, None, 1, 1, 16, 128, 0,
+                                 0, 0, 1, None) == 1
+    assert attn.fp8_quantize_raw(far + 8, 2 * far, 3 * far, None, 1, 1, 16, 128,
+                                 0, 0, 0, 0, None) == 4
+    # codes overlapping the input
+    assert attn.fp8_quantize_raw(far, far + 64, 3 * far, None, 1, 1, 16, 128, 0,
+                                 0, 0, 0, None) == 6
+    # whole path: workspace missing or too small
+    args = [far, 2 * far, 3 * far, 4 * far, 5 * far, 1, 1, 16, 128, 0, 0.125, 1,
+            0, 0]
+    assert attn.attn_fwd_fp8_raw(*args, None, 0, None) == 11
+    assert attn.attn_fwd_fp8_raw(*args, 6 * far, 16, None) == 11
+    assert attn.attn_fwd_fp8_raw(*(args[:8] + [64] + args[9:]), 6 * far,
+                                 1 << 30, None) == 3
+    # empty problems are no-ops
+    assert attn.attn_fwd_fp8_raw(None, None, None, None, None, 0, 1, 16, 128, 0,
+                                 0.125, 1, 0, 0, None, 0, None) == 0
+
+
+def test_fp8_workspace_and_sign_mask(attn):
+    B, H, N = 2, 3, 300
+    r = lambda x: (x + 255) // 256 * 256
+    tiles = -(-N // 128)
+    assert attn.fp8_workspace_bytes(B, H, N, 128) == \
+        3 * r(B * H * N * 128) + 3 * r(B * H * tiles * 4) + r(B * H * 4)
+    assert attn.fp8_workspace_bytes(B, H, N, 64) == 0
+    lo, hi = attn.sign_mask([1, -1] + [1] * 62 + [-1] + [1] * 63)
+    assert lo == 2 and hi == 1
+    with pytest.raises(ValueError):
+        attn.sign_mask([1, 0, 1])
