@@ -1,7 +1,8 @@
 """Benchmark of the B200 exact attention forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--no-cpu-baseline]
+                    [--impl ours|reference] [--pass fwd|bwd|fp8]
+                    [--no-cpu-baseline]
 
 A step is one attention forward pass over the whole workload (default: the
 non-causal B=1, H=32, N=16384, d=128 case the throughput target is set on),
@@ -68,10 +69,10 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def load_traffic(workload: str):
+def load_traffic(workload: str, prefix: str = "traffic_"):
     """DRAM bytes per launch from a committed ncu capture of this workload,
     or None when there is none or the kernel changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    path = os.path.join(ROOT, "profiles", f"{prefix}{workload}.json")
     try:
         with open(path) as f:
             t = json.load(f)
@@ -331,6 +332,198 @@ def run_backward(args, w):
     return 0
 
 
+METRIC_FP8 = ("attention fwd TFLOP/s, FP8 (E4M3) operands with incoherent "
+              "processing (rotation + block quantization inside the step)")
+FP8_SIGN_SEED = 77
+
+
+def cpu_baseline_fp8(w, qkv, signs, budget_s: float, seed: int = 13):
+    """The FP8 oracle (as it stands) on head (0, 0) of the workload: its Q,
+    K, V quantized (time amortised over the rows timed), then random query
+    rows through the blocked E4M3 softmax, all host cores."""
+    import numpy as np
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    bits = [oracle.bf16_bits(t[:1, :1].contiguous()) for t in qkv]
+    t0 = time.perf_counter()
+    z = oracle.quantize_qkv_fp8(*bits, True, np.asarray(signs, dtype=np.int8))
+    t_quant = time.perf_counter() - t0
+    scale_qk = float(np.float32(w.scale)) * z["gain"]
+    rng = np.random.default_rng(seed)
+    rows_done, flops, elapsed = 0, 0.0, 0.0
+    batch = max(threads, 8)
+    while elapsed < budget_s:
+        rows = rng.integers(0, w.N, size=batch)
+        t1 = time.perf_counter()
+        oracle.attention_fp8_rows(z["q8"], z["qs"], z["k8"], z["ks"], z["v8"],
+                                  z["vs"], w.causal, scale_qk, rows,
+                                  threads=threads)
+        dt = time.perf_counter() - t1
+        elapsed += dt
+        rows_done += batch
+        keys = (rows + 1) if w.causal else np.full_like(rows, w.N)
+        flops += float(np.sum(4.0 * keys * w.d))
+        rate = batch / max(dt, 1e-6)
+        batch = int(min(max(threads, rate * (budget_s - elapsed) * 0.9), w.N))
+        if budget_s - elapsed < 0.5:
+            break
+    total = elapsed + t_quant * rows_done / w.N
+    return {"value": flops / total / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"head (0,0) of {w.name}: quantized in {t_quant:.1f} s "
+                      f"(amortised over the rows), {rows_done} random query "
+                      f"rows through the FP8 oracle in {elapsed:.1f} s"}
+
+
+def run_fp8(args, w):
+    """Time the FP8 path: attn_fwd_fp8 = quantize Q, K (rotated, per tile)
+    and V (per head: two launches), then the E4M3 attention kernel."""
+    import torch
+    from exact_io_aware_73_b200 import attn
+    if w.d != 128:
+        raise SystemExit("the FP8 path exists for d = 128 only")
+    world, rank, local = R.env_ranks()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    R.init("nccl", world, device=dev)
+    qkv_host = W.make_qkv(w, seed=R.rank_seed(w.seed, rank))
+    q, k, v = (t.to(dev) for t in qkv_host)
+    signs = W.make_signs(FP8_SIGN_SEED, w.d).tolist()
+    lo, hi = attn.sign_mask(signs)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.fp8_workspace_bytes(w.B, w.H, w.N, w.d),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    in_bytes = 3 * q.numel() * 2
+    flush = None if in_bytes > L2_BYTES else torch.empty(
+        2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(qq=q, kk=k, vv=v, oo=o, ll=lse):
+        rc = attn.attn_fwd_fp8_raw(qq.data_ptr(), kk.data_ptr(), vv.data_ptr(),
+                                   oo.data_ptr(), ll.data_ptr(), w.B, w.H, w.N,
+                                   w.d, w.causal, w.scale, 1, lo, hi,
+                                   ws.data_ptr(), ws.numel(), sh)
+        if rc != 0:
+            raise attn.AttnError(rc, "attn_fwd_fp8")
+
+    # the attention kernel alone, on codes made by the same path
+    q8, qs = attn.fp8_quantize(q, True, signs)
+    k8, ks = attn.fp8_quantize(k, True, signs)
+    v8, vs = attn.fp8_quantize(v, False, per_head=True)
+    fp8_fns = attn._fp8_fns()
+
+    def kernel_only():
+        rc = fp8_fns.attn_fwd_fp8_quantized(
+            q8.data_ptr(), qs.data_ptr(), k8.data_ptr(), ks.data_ptr(),
+            v8.data_ptr(), vs.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B,
+            w.H, w.N, w.d, int(w.causal), float(w.scale / w.d), sh)
+        if rc != 0:
+            raise attn.AttnError(rc, "attn_fwd_fp8_quantized")
+
+    def timed(fn, steps):
+        evs = []
+        for _ in range(steps):
+            if flush is not None:
+                flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            evs.append((a, b))
+        R.barrier(world)
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    for _ in range(args.warmup):
+        step()
+        kernel_only()
+    if attn.status() != 0:
+        raise RuntimeError("device status after warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    step_ms = timed(step, args.steps)
+    kern_ms = timed(kernel_only, args.steps)
+    clk = clocks.stop()
+    if attn.status() != 0:
+        raise RuntimeError("device status after the timed region")
+    ms_per_step = R.max_over_ranks(step_ms, world, dev) / args.steps
+    kern_ms_per = R.max_over_ranks(kern_ms, world, dev) / args.steps
+    flops = w.flops()
+    value = R.job_throughput(flops, world, ms_per_step * 1e-3) / 1e12
+
+    # end to end: pinned host Q, K, V copied in, O and lse copied out, every
+    # step, around the same public call
+    qh, kh, vh = (x.pin_memory() for x in qkv_host)
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for dst, src in ((q, qh), (k, kh), (v, vh)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    if attn.status() != 0:
+        raise RuntimeError("device status after the e2e region")
+    e2e_ms = R.max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    e2e_value = R.job_throughput(flops, world, e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak = 2.0 * peaks["bf16_tflops"]
+    achieved = flops / (kern_ms_per * 1e-3) / 1e12
+    cb = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_baseline_fp8(w, qkv_host, signs, args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC_FP8, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic (seeded Gaussian bf16 inputs; seeded rotation signs)",
+            "config": {"workload": w.name, "pass": "fp8", "B": w.B, "H": w.H,
+                       "N": w.N, "d": w.d, "causal": w.causal,
+                       "l2": ("inputs larger than L2" if flush is None else
+                              "L2 flushed between steps (outside the events)"),
+                       "parallelism": f"{world} independent replicas"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16 burst (cuBLAS) x 2, "
+                                        "the nominal E4M3 / bf16 ratio",
+                         "traffic": load_traffic(w.name, "traffic_fp8_"),
+                         "kernel": "attn_fwd_sm100_kernel<128,*,FP8>",
+                         "kernel_ms": kern_ms_per,
+                         "quantize_ms": ms_per_step - kern_ms_per},
+            "cpu_baseline": cb,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": 3 * qh.numel() * 2,
+                    "d2h_bytes_per_step": oh.numel() * 2 + lh.numel() * 4,
+                    "ms_per_step": e2e_ms, "steps": e2e_steps,
+                    "api": "attn.attn_fwd_fp8 around torch copies of pinned buffers"},
+            "gpu_launches": 5 * args.steps, "clocks": clk}), flush=True)
+    R.finish(world)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -338,8 +531,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
-                    help="fwd (default): the forward hot path; bwd: attn_bwd")
+    ap.add_argument("--pass", dest="pass_", default="fwd",
+                    choices=["fwd", "bwd", "fp8"],
+                    help="fwd (default): the forward hot path; bwd: attn_bwd; "
+                         "fp8: the FP8 forward with incoherent processing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     args = ap.parse_args()
@@ -350,6 +545,8 @@ def main():
         return run_reference(args, w)
     if args.pass_ == "bwd":
         return run_backward(args, w)
+    if args.pass_ == "fp8":
+        return run_fp8(args, w)
 
     import torch
     from exact_io_aware_73_b200 import attn
