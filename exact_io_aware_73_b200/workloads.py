@@ -157,3 +157,69 @@ def add_channel_outliers(x: torch.Tensor, channels, factor: float) -> torch.Tens
 def outlier_channels(seed: int, d: int, count: int):
     """``count`` distinct coordinates in [0, d), drawn from a seeded generator."""
     return sorted(int(c) for c in torch.randperm(d, generator=_gen(seed))[:count])
+
+
+# ------------------------------------------------------------ decode inputs
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Nq new queries (the last Nq positions) against an Nk-long key/value
+    sequence per (batch, head)."""
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """The two GEMMs over visible keys: 4 d per (query, key) pair."""
+        if self.causal:
+            keys = sum(self.Nk - self.Nq + i + 1 for i in range(self.Nq))
+        else:
+            keys = self.Nq * self.Nk
+        return 4.0 * self.B * self.H * keys * self.d
+
+    def kv_bytes(self) -> int:
+        """K and V read once: the bytes a decode step must stream."""
+        return 2 * self.B * self.H * self.Nk * self.d * 2
+
+
+DECODE_WORKLOADS = {
+    # few heads, very long context: a grid over (batch, head) alone would
+    # occupy 8 of 148 SMs
+    "decode_b1h8nq1nk262144d128": DecodeWorkload(
+        "decode_b1h8nq1nk262144d128", 1, 8, 1, 262144, 128, True, seed=2001),
+    # a batch of sequences, one new token each
+    "decode_b8h32nq1nk32768d128": DecodeWorkload(
+        "decode_b8h32nq1nk32768d128", 8, 32, 1, 32768, 128, True, seed=2002),
+    # one trading day of one-second steps as context, 12 heads of 64,
+    # four new steps at once
+    "decode_tradingday_b16h12nq4nk23400d64": DecodeWorkload(
+        "decode_tradingday_b16h12nq4nk23400d64", 16, 12, 4, 23400, 64, True,
+        seed=2003),
+}
+
+DECODE_HEADLINE = "decode_b1h8nq1nk262144d128"
+
+
+def make_decode_qkv(w: DecodeWorkload, seed: int | None = None):
+    """(q [B, H, Nq, d], k, v [B, H, Nk, d]) bf16 CPU tensors, N(0, 1),
+    seeds seed, seed + 1, seed + 2 (default: the workload's seed)."""
+    s = w.seed if seed is None else int(seed)
+    q = _normal((w.B, w.H, w.Nq, w.d), 1.0, s)
+    k = _normal((w.B, w.H, w.Nk, w.d), 1.0, s + 1)
+    v = _normal((w.B, w.H, w.Nk, w.d), 1.0, s + 2)
+    return q, k, v
+
+
+def decode_case(B, H, Nq, Nk, d, causal, seed) -> DecodeWorkload:
+    return DecodeWorkload(f"decode_case_b{B}h{H}nq{Nq}nk{Nk}d{d}"
+                          f"{'_causal' if causal else ''}", B, H, Nq, Nk, d,
+                          causal, seed)

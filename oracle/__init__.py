@@ -30,4 +30,6 @@ from .oracle import (  # noqa: F401
     attention_fp8,
     attention_fp8_rows,
     quantize_qkv_fp8,
+    attention_decode,
+    attention_decode_rows_bf16,
 )

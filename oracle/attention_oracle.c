@@ -42,6 +42,12 @@
  * Masked entries have P = 0 and so dS = 0.  The oracle recomputes P from
  * the scores with its own two-pass softmax, exactly as the forward does.
  *
+ * Decode (few new queries against a long key/value sequence; the
+ * briefgpt.xyz summary page of FlashAttention-2, arXiv 2307.08691, entry
+ * "LeanAttention": the decode phase of long contexts): the queries are
+ * the last Nq positions of an Nk-long sequence, so with the causal mask
+ * query i sees keys 0 .. Nk - Nq + i.  Same definition otherwise.
+ *
  * Layout conventions: Q, K, V, O are contiguous row-major [B, H, N, d];
  * lse is contiguous [B, H, N].  bf16 inputs are passed as their raw 16-bit
  * patterns and widened exactly to double (bf16 -> fp32 is exact, fp32 ->
@@ -174,6 +180,105 @@ int oracle_attention_f64(const double *Q, const double *K, const double *V,
       attend_row(s, n, Vh, d, O + r * d, lse + r, NULL);
     }
     free(s);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode: few queries against a long key/value sequence.                   */
+/* ------------------------------------------------------------------------ */
+
+/* Keys visible to query i of Nq new queries appended to a sequence whose
+ * keys are 0..Nk-1 (the queries are the last Nq positions, Nq <= Nk):
+ * query i sits at position Nk - Nq + i and, with the causal mask, sees keys
+ * 0 .. Nk - Nq + i ([MM] "Causal masking ...": no key in a query's future;
+ * the "bottom-right" alignment, the only one under which the new tokens are
+ * the latest positions).  Without the mask every key is visible. */
+static int64_t decode_visible_keys(int64_t i, int64_t Nq, int64_t Nk, int causal) {
+  return causal ? (Nk - Nq + i + 1) : Nk;
+}
+
+/* Decode attention over fp64 inputs: Q [BH, Nq, d], K and V [BH, Nk, d],
+ * O [BH, Nq, d], lse [BH, Nq]; the same definition as oracle_attention_f64
+ * (whole score row, two softmax passes) with the visibility rule above.
+ * OpenMP over rows. */
+int oracle_attention_decode_f64(const double *Q, const double *K,
+                                const double *V, double *O, double *lse,
+                                int64_t BH, int64_t Nq, int64_t Nk, int64_t d,
+                                int causal, double scale, int nthreads) {
+  if (!Q || !K || !V || !O || !lse || BH < 0 || Nq < 0 || Nk < 1 || d < 1 ||
+      (causal && Nq > Nk))
+    return ORACLE_EBADARG;
+  const int64_t rows = BH * Nq;
+  if (rows == 0) return ORACLE_OK;
+  int err = ORACLE_OK;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)Nk);
+    if (!s) {
+#pragma omp atomic write
+      err = ORACLE_ENOMEM;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+      if (!s) continue;
+      const int64_t bh = r / Nq, i = r % Nq;
+      const double *Kh = K + bh * Nk * d, *Vh = V + bh * Nk * d;
+      const double *qi = Q + r * d;
+      const int64_t n = decode_visible_keys(i, Nq, Nk, causal);
+      for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < d; ++t) acc += qi[t] * Kh[j * d + t];
+        s[j] = scale * acc;
+      }
+      attend_row(s, n, Vh, d, O + r * d, lse + r, NULL);
+    }
+    free(s);
+  }
+  return err;
+}
+
+/* The same on bf16 bit patterns for selected rows (flat index bh * Nq + i),
+ * widening key and value rows on the fly (full-size checks without an fp64
+ * copy of the key/value sequence).  O_out [nrows, d], lse_out [nrows]. */
+int oracle_attention_decode_rows_bf16(const uint16_t *Q, const uint16_t *K,
+                                      const uint16_t *V, int64_t BH, int64_t Nq,
+                                      int64_t Nk, int64_t d, int causal,
+                                      double scale, const int64_t *rows,
+                                      int64_t nrows, double *O_out,
+                                      double *lse_out, int nthreads) {
+  if (!Q || !K || !V || !rows || !O_out || !lse_out || BH < 1 || Nq < 1 ||
+      Nk < 1 || d < 1 || (causal && Nq > Nk))
+    return ORACLE_EBADARG;
+  for (int64_t k = 0; k < nrows; ++k)
+    if (rows[k] < 0 || rows[k] >= BH * Nq) return ORACLE_EBADARG;
+  int err = ORACLE_OK;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)Nk);
+    double *vv = (double *)malloc(sizeof(double) * (size_t)(Nk * d));
+    double *qi = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!s || !vv || !qi) {
+#pragma omp atomic write
+      err = ORACLE_ENOMEM;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t k = 0; k < nrows; ++k) {
+      if (!s || !vv || !qi) continue;
+      const int64_t r = rows[k], bh = r / Nq, i = r % Nq;
+      const uint16_t *Kh = K + bh * Nk * d, *Vh = V + bh * Nk * d;
+      for (int64_t t = 0; t < d; ++t) qi[t] = bf16_bits_to_double(Q[r * d + t]);
+      const int64_t n = decode_visible_keys(i, Nq, Nk, causal);
+      for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < d; ++t)
+          acc += qi[t] * bf16_bits_to_double(Kh[j * d + t]);
+        s[j] = scale * acc;
+        for (int64_t t = 0; t < d; ++t) vv[j * d + t] = bf16_bits_to_double(Vh[j * d + t]);
+      }
+      attend_row(s, n, vv, d, O_out + k * d, lse_out + k, NULL);
+    }
+    free(s); free(vv); free(qi);
   }
   return err;
 }

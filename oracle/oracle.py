@@ -43,6 +43,15 @@ def _load():
         lib.oracle_attention_blocked_f64.argtypes = [
             dp, dp, dp, dp, dp, i64, i64, i64, i64, ctypes.c_int,
             ctypes.c_double, i64, i64]
+        lib.oracle_attention_decode_f64.argtypes = [
+            dp, dp, dp, dp, dp, i64, i64, i64, i64, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int]
+        lib.oracle_attention_decode_rows_bf16.argtypes = [
+            u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_int, ctypes.c_double,
+            i64p, i64, dp, dp, ctypes.c_int]
+        for f in (lib.oracle_attention_decode_f64,
+                  lib.oracle_attention_decode_rows_bf16):
+            f.restype = ctypes.c_int
         u8p = ctypes.POINTER(ctypes.c_uint8)
         i8p = ctypes.POINTER(ctypes.c_int8)
         fp = ctypes.POINTER(ctypes.c_float)
@@ -182,6 +191,44 @@ def attention_backward(q, k, v, do, causal: bool, scale: float, threads=None):
         _dptr(dv), B, H, N, d, int(bool(causal)), float(scale),
         _threads(threads)), "attention_backward")
     return dq, dk, dv
+
+
+def attention_decode(q, k, v, causal: bool, scale: float, threads=None):
+    """Decode attention on fp64 arrays: q [..., Nq, d], k and v [..., Nk, d]
+    (same leading dims); the queries are the last Nq positions, so the
+    causal mask lets query i see keys 0 .. Nk - Nq + i.  Returns (O, lse)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    Nq, d = q.shape[-2], q.shape[-1]
+    Nk = k.shape[-2]
+    BH = q.size // (Nq * d) if Nq else int(np.prod(q.shape[:-2]))
+    O = np.empty(q.shape)
+    lse = np.empty(q.shape[:-1])
+    _check(_load().oracle_attention_decode_f64(
+        _dptr(q), _dptr(k), _dptr(v), _dptr(O), _dptr(lse), BH, Nq, Nk, d,
+        int(bool(causal)), float(scale), _threads(threads)), "attention_decode")
+    return O, lse
+
+
+def attention_decode_rows_bf16(qbits, kbits, vbits, causal: bool, scale: float,
+                               rows, threads=None):
+    """Decode attention on bf16 bit patterns for flat rows bh * Nq + i;
+    returns (O [len(rows), d], lse [len(rows)])."""
+    qbits, kbits, vbits = (np.ascontiguousarray(a, dtype=np.uint16)
+                           for a in (qbits, kbits, vbits))
+    Nq, d = qbits.shape[-2], qbits.shape[-1]
+    Nk = kbits.shape[-2]
+    BH = qbits.size // (Nq * d)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    O = np.empty((rows.size, d))
+    lse = np.empty(rows.size)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    _check(_load().oracle_attention_decode_rows_bf16(
+        qbits.ctypes.data_as(u16p), kbits.ctypes.data_as(u16p),
+        vbits.ctypes.data_as(u16p), BH, Nq, Nk, d, int(bool(causal)),
+        float(scale), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        rows.size, _dptr(O), _dptr(lse), _threads(threads)),
+        "attention_decode_rows_bf16")
+    return O, lse
 
 
 # ---------------------------------------------------------------- FP8 path

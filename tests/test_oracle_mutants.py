@@ -23,6 +23,7 @@ FP8_SRC = os.path.join(ROOT, "oracle", "fp8_oracle.c")
 PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 BACKWARD_PINS = os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")
 FP8_PINS = os.path.join(ROOT, "tests", "test_oracle_fp8_pins.py")
+DECODE_PINS = os.path.join(ROOT, "tests", "test_oracle_decode_pins.py")
 
 MUTANTS = {
     "mask_hides_diagonal": ("return causal ? (i + 1) : N;",
@@ -81,13 +82,25 @@ FP8_MUTANTS = {
                                "q_scale[bh * qblocks]"),
 }
 
+# planted mistakes in the decode oracle; each must fail a decode pin
+DECODE_MUTANTS = {
+    "decode_top_left_mask": ("return causal ? (Nk - Nq + i + 1) : Nk;",
+                             "return causal ? (i + 1) : Nk;"),
+    "decode_mask_one_short": ("return causal ? (Nk - Nq + i + 1) : Nk;",
+                              "return causal ? (Nk - Nq + i) : Nk;"),
+    "decode_keys_stride_q": ("const double *Kh = K + bh * Nk * d, *Vh = V + bh * Nk * d;\n      const double *qi = Q + r * d;\n      const int64_t n = decode_visible_keys",
+                             "const double *Kh = K + bh * Nq * d, *Vh = V + bh * Nk * d;\n      const double *qi = Q + r * d;\n      const int64_t n = decode_visible_keys"),
+    "decode_rows_values_from_keys": ("for (int64_t t = 0; t < d; ++t) vv[j * d + t] = bf16_bits_to_double(Vh[j * d + t]);",
+                                     "for (int64_t t = 0; t < d; ++t) vv[j * d + t] = bf16_bits_to_double(Kh[j * d + t]);"),
+}
+
 
 def _build_mutant(name, tmpdir):
     if name in FP8_MUTANTS:
         old, new = FP8_MUTANTS[name]
         target, other = FP8_SRC, SRC
     else:
-        old, new = {**MUTANTS, **BACKWARD_MUTANTS}[name]
+        old, new = {**MUTANTS, **BACKWARD_MUTANTS, **DECODE_MUTANTS}[name]
         target, other = SRC, FP8_SRC
     src = open(target).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
@@ -134,3 +147,9 @@ def test_every_planted_fp8_mistake_fails_an_fp8_pin():
     with tempfile.TemporaryDirectory() as tmp:
         survivors = _run_against(FP8_MUTANTS, FP8_PINS, tmp)
         assert not survivors, f"FP8 pins did not catch: {survivors}"
+
+
+def test_every_planted_decode_mistake_fails_a_decode_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        survivors = _run_against(DECODE_MUTANTS, DECODE_PINS, tmp)
+        assert not survivors, f"decode pins did not catch: {survivors}"
