@@ -359,3 +359,64 @@ def attn_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None,
                           _stream_handle(stream))
     _check(rc, "attn_fwd_fp8")
     return out, lse
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_fns():
+    L = lib()
+    if L.attn_decode.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        L.attn_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                  ctypes.c_float, vp, ctypes.c_size_t, vp]
+        L.attn_decode.restype = i
+        L.attn_decode_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.attn_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.attn_set_decode_max_ctas.argtypes = [i]
+        L.attn_set_decode_max_ctas.restype = None
+    return L
+
+
+DECODE_MAX_Q = 16
+
+
+def decode_workspace_bytes(B, H, Nq, Nk, d) -> int:
+    return int(_decode_fns().attn_decode_workspace_bytes(B, H, Nq, Nk, d))
+
+
+def set_decode_max_ctas(n: int) -> None:
+    """Test hook: cap attn_decode's CTA count (0 restores two per SM)."""
+    _decode_fns().attn_set_decode_max_ctas(int(n))
+
+
+def attn_decode_raw(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, ws,
+                    ws_bytes, stream_handle) -> int:
+    return _decode_fns().attn_decode(q, k, v, o, lse, int(B), int(H), int(Nq),
+                                     int(Nk), int(d), int(bool(causal)),
+                                     float(scale), ws, ws_bytes, stream_handle)
+
+
+def attn_decode(q, k, v, causal: bool = True, scale: float | None = None,
+                workspace=None, out=None, lse=None, stream=None):
+    """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16)
+    against k, v bf16 [B, H, Nk, d]; returns (O bf16, lse fp32 [B, H, Nq])."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if k.shape != (B, H, Nk, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H, d")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, H, Nq, Nk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    rc = attn_decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                         out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
+                         causal, scale, workspace.data_ptr(), workspace.numel(),
+                         _stream_handle(stream))
+    _check(rc, "attn_decode")
+    return out, lse

@@ -16,6 +16,7 @@
 #include "attn_b200.h"
 #include "attn_bwd_kernel.cuh"
 #include "fp8_quant_kernel.cuh"
+#include "attn_decode_kernel.cuh"
 
 namespace {
 
@@ -32,6 +33,7 @@ struct DeviceState {
   uint32_t *status = nullptr;  // 4-byte device status word, lazily allocated
   bool smem_attr_set[6] = {false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
+  bool dec_attr_set[2] = {false, false};
 };
 
 std::mutex g_mu;
@@ -39,6 +41,7 @@ DeviceState g_dev[kMaxDevices];
 std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<uint32_t> g_inject{0};
 std::atomic<uint32_t> g_last_bits{0};
+std::atomic<int> g_decode_max_ctas{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
                                   void *, const cuuint64_t *, const cuuint64_t *,
@@ -269,6 +272,39 @@ int launch_quant(DeviceState &st, const attn_b200::QuantParams &p, int mode,
   const int64_t tiles = static_cast<int64_t>(p.bh) * p.tiles;
   const int grid = static_cast<int>(tiles < st.sm_count ? tiles : st.sm_count);
   attn_b200::fp8_quant_kernel<128><<<grid, attn_b200::kQuantThreads, 0, stream>>>(p, mode);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+template <int D>
+int launch_decode(DeviceState &st, int variant, attn_b200::DecodeParams &p,
+                  cudaStream_t stream) {
+  using L = attn_b200::DecSmem<D>;
+  auto kern = attn_b200::attn_decode_kernel<D>;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!st.dec_attr_set[variant]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(L::kBytes)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      st.dec_attr_set[variant] = true;
+    }
+  }
+  // stream-K: an equal share of the key tiles per CTA, two CTAs per SM
+  int ctas = g_decode_max_ctas.load();
+  if (ctas <= 0) ctas = 2 * st.sm_count;
+  if (ctas > attn_b200::kDecMaxCtas) ctas = attn_b200::kDecMaxCtas;
+  const int grid0 = p.total < ctas ? p.total : ctas;
+  p.per_cta = (p.total + grid0 - 1) / grid0;
+  const int grid = (p.total + p.per_cta - 1) / p.per_cta;
+  if (cudaMemsetAsync(p.counters, 0, sizeof(int) * static_cast<size_t>(p.bh), stream) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  kern<<<grid, attn_b200::kDecThreads, L::kBytes, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
@@ -622,6 +658,82 @@ int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
   return attn_fwd_fp8_quantized(q8, qs, k8, ks, v8, vs, o, lse, B, H, N, d, causal,
                                 scale_qk, stream);
 }
+
+size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
+  if (B < 0 || H < 0 || Nq < 0 || Nq > ATTN_DECODE_MAX_Q || Nk < 0 ||
+      (d != 64 && d != 128))
+    return 0;
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t slots = bh + attn_b200::kDecMaxCtas;
+  return round256(slots * Nq * d * 4) + round256(slots * Nq * 4) + round256(bh * 4);
+}
+
+int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                void *workspace, size_t workspace_bytes, attn_stream_t stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_SIZE;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  if (!(std::isfinite(scale) && scale > 0.f)) return ATTN_ERR_INVALID_SCALE;
+  if (Nq > ATTN_DECODE_MAX_Q || (Nq > 0 && Nk == 0) || (causal && Nq > Nk))
+    return ATTN_ERR_INVALID_SIZE;
+  if (B == 0 || H == 0 || Nq == 0) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL_POINTER;
+  const int64_t bh64 = static_cast<int64_t>(B) * H;
+  if (Nk > ATTN_MAX_DECODE_KEYS || bh64 > ATTN_MAX_HEADS) return ATTN_ERR_INVALID_SIZE;
+  const int64_t ntiles = (Nk + attn_b200::kDecTileKeys - 1) / attn_b200::kDecTileKeys;
+  if (bh64 * ntiles > 0x7fffffffLL) return ATTN_ERR_INVALID_SIZE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4))
+    return ATTN_ERR_MISALIGNED;
+  const size_t need = attn_decode_workspace_bytes(B, H, Nq, Nk, d);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+    return ATTN_ERR_WORKSPACE;
+  const size_t qb = static_cast<size_t>(bh64) * Nq * d * 2;
+  const size_t kb = static_cast<size_t>(bh64) * Nk * d * 2;
+  const size_t lb = static_cast<size_t>(bh64) * Nq * 4;
+  const void *ins[3] = {q, k, v};
+  const size_t in_bytes[3] = {qb, kb, kb};
+  void *outs[3] = {o, lse, workspace};
+  const size_t out_bytes[3] = {qb, lb, need};
+  for (int a = 0; a < 3; ++a) {
+    for (int b = 0; b < 3; ++b)
+      if (overlaps(outs[a], out_bytes[a], ins[b], in_bytes[b])) return ATTN_ERR_ALIAS;
+    for (int b = a + 1; b < 3; ++b)
+      if (overlaps(outs[a], out_bytes[a], outs[b], out_bytes[b])) return ATTN_ERR_ALIAS;
+  }
+  int rc, dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  const void *all[6] = {q, k, v, o, lse, workspace};
+  for (const void *ptr : all)
+    if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
+  const size_t slots = static_cast<size_t>(bh64) + attn_b200::kDecMaxCtas;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  attn_b200::DecodeParams p;
+  p.q = static_cast<const uint16_t *>(q);
+  p.k = static_cast<const uint16_t *>(k);
+  p.v = static_cast<const uint16_t *>(v);
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.part_o = reinterpret_cast<float *>(ws);
+  p.part_lse = reinterpret_cast<float *>(ws + round256(slots * Nq * d * 4));
+  p.counters = reinterpret_cast<int *>(ws + round256(slots * Nq * d * 4) +
+                                       round256(slots * Nq * 4));
+  p.status = st->status;
+  p.bh = static_cast<int>(bh64);
+  p.nq = Nq;
+  p.nk = Nk;
+  p.ntiles = static_cast<int>(ntiles);
+  p.total = static_cast<int>(bh64 * ntiles);
+  p.per_cta = 1;
+  p.causal = causal ? 1 : 0;
+  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.timeout_ns = g_timeout_ns.load();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_decode<128>(*st, 0, p, s) : launch_decode<64>(*st, 1, p, s);
+}
+
+void attn_set_decode_max_ctas(int n) { g_decode_max_ctas.store(n > 0 ? n : 0); }
 
 int attn_status(attn_stream_t stream) {
   int dev = -1;

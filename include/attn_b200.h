@@ -311,6 +311,45 @@ int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
  * maxima, each rounded up to 256 bytes. */
 size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
 
+/*
+ * attn_decode -- split-KV decode attention: Nq new queries against Nk keys
+ * per (batch, head), after the briefgpt.xyz summary page of FlashAttention-2
+ * (arXiv 2307.08691), entry "LeanAttention" (the decode phase of long
+ * contexts, computed in parallel over the key/value sequence).
+ *
+ *   q      bf16 [B, H, Nq, d], the queries of the last Nq positions;
+ *   k, v   bf16 [B, H, Nk, d], the whole key/value sequence;
+ *   o      bf16 [B, H, Nq, d]; lse fp32 [B, H, Nq] (natural log);
+ *   O = softmax(scale q k^T [mask]) v exactly; with causal != 0 query i
+ *   sees keys 0 .. Nk - Nq + i (the queries are the latest positions).
+ * Limits: 1 <= Nq <= ATTN_DECODE_MAX_Q (Nq = 0 is a no-op), Nk >= 1,
+ * Nq <= Nk when causal, d in {64, 128}, Nk <= ATTN_MAX_DECODE_KEYS.
+ * q, k, v, o 16-byte aligned, lse 4-byte aligned, all device memory of the
+ * current device.  workspace: at least attn_decode_workspace_bytes(...)
+ * bytes, 256-byte aligned, caller-owned scratch for this call (partial
+ * outputs of split heads and one counter per head, zeroed by the call).
+ * Outputs and workspace must not overlap the inputs or each other.
+ *
+ * The key tiles of all heads are split into equal contiguous shares, one per
+ * CTA (two CTAs per SM); a head split over several CTAs is combined exactly
+ * by the CTA that finishes its last share.  Queued on `stream`; a wait that
+ * runs out of time shows in attn_status (outputs are then invalid).
+ */
+#define ATTN_DECODE_MAX_Q 16
+#define ATTN_MAX_DECODE_KEYS (1 << 26)
+int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/* Workspace bytes attn_decode needs (0 on bad sizes): partial outputs and
+ * log-sum-exps for B*H + 1024 parts, and B*H counters, each rounded up to
+ * 256 bytes. */
+size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d);
+
+/* Test hook: cap the number of CTAs attn_decode launches (0 = two per SM),
+ * so that small problems can be split over many CTAs.  Process-wide. */
+void attn_set_decode_max_ctas(int n);
+
 /* Human-readable text for an error code (static string, never NULL). */
 const char *attn_strerror(int code);
 

@@ -172,3 +172,29 @@ def test_fp8_workspace_and_sign_mask(attn):
     assert lo == 2 and hi == 1
     with pytest.raises(ValueError):
         attn.sign_mask([1, 0, 1])
+
+
+def test_decode_entry_refuses_bad_arguments_without_a_device(attn):
+    far = 1 << 40
+    ws = 6 * far
+    base = [far, 2 * far, 3 * far, 4 * far, 5 * far]
+    def call(B=1, H=1, Nq=1, Nk=256, d=128, causal=1, scale=0.125, ptrs=None,
+             wsp=ws, wsb=1 << 30):
+        return attn.attn_decode_raw(*(ptrs or base), B, H, Nq, Nk, d, causal,
+                                    scale, wsp, wsb, None)
+    assert call(Nq=17) == 2                      # more than 16 queries
+    assert call(Nq=5, Nk=4) == 2                 # causal needs Nq <= Nk
+    assert call(d=96) == 3
+    assert call(scale=0.0) == 5
+    assert call(ptrs=[None] + base[1:]) == 1
+    assert call(ptrs=[far + 8] + base[1:]) == 4
+    assert call(wsp=None) == 11
+    assert call(wsb=16) == 11
+    assert call(ptrs=base[:3] + [far + 64, base[4]]) == 6   # o overlaps q
+    assert call(Nq=0, ptrs=[None] * 5, wsp=None) == 0       # empty: no-op
+    assert attn.decode_workspace_bytes(1, 1, 17, 10, 128) == 0
+    B, H, Nq, d = 2, 3, 4, 64
+    r = lambda x: (x + 255) // 256 * 256
+    slots = B * H + 1024
+    assert attn.decode_workspace_bytes(B, H, Nq, 1000, d) == \
+        r(slots * Nq * d * 4) + r(slots * Nq * 4) + r(B * H * 4)
