@@ -1,7 +1,7 @@
 """Benchmark of the B200 exact attention forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--pass fwd|bwd|fp8]
+                    [--impl ours|reference] [--pass fwd|bwd|fp8|decode]
                     [--no-cpu-baseline]
 
 A step is one attention forward pass over the whole workload (default: the
@@ -524,22 +524,184 @@ def run_fp8(args, w):
     return 0
 
 
+METRIC_DECODE = ("attention decode: K/V bytes streamed per second (GB/s; "
+                 "split-KV, HBM-bound)")
+
+
+def cpu_baseline_decode(w, qkv, budget_s: float):
+    """The fp64 oracle on query rows of the decode workload (every row of as
+    many heads as the budget allows), all host cores; GB/s of K/V covered."""
+    import numpy as np
+    import oracle
+    q, k, v = qkv
+    bits = [oracle.bf16_bits(t) for t in (q, k, v)]
+    threads = len(os.sched_getaffinity(0))
+    rows_total = w.B * w.H * w.Nq
+    done, elapsed, batch = 0, 0.0, max(1, min(threads, rows_total))
+    while elapsed < budget_s and done < rows_total:
+        rows = np.arange(done, min(rows_total, done + batch))
+        t0 = time.perf_counter()
+        oracle.attention_decode_rows_bf16(*bits, w.causal, w.scale, rows, threads)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        done += rows.size
+        if budget_s - elapsed < 0.5:
+            break
+    heads = done / w.Nq
+    kv = heads * 2 * w.Nk * w.d * 2
+    return {"value": kv / elapsed / 1e9, "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{done} of {rows_total} query rows of {w.name} "
+                      f"(fp64 oracle, {elapsed:.1f} s)"}
+
+
+def run_decode(args):
+    """Time attn_decode on a decode workload (Nq new queries against an
+    Nk-long key/value sequence per head); one launch per step."""
+    import torch
+    from exact_io_aware_73_b200 import attn
+    name = args.workload if args.workload in W.DECODE_WORKLOADS else W.DECODE_HEADLINE
+    w = W.DECODE_WORKLOADS[name]
+    world, rank, local = R.env_ranks()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    R.init("nccl", world, device=dev)
+    qkv_host = W.make_decode_qkv(w, seed=R.rank_seed(w.seed, rank))
+    q, k, v = (t.to(dev) for t in qkv_host)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    flush = None if w.kv_bytes() > L2_BYTES else torch.empty(
+        2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        rc = attn.attn_decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                  o.data_ptr(), lse.data_ptr(), w.B, w.H, w.Nq,
+                                  w.Nk, w.d, w.causal, w.scale, ws.data_ptr(),
+                                  ws.numel(), sh)
+        if rc != 0:
+            raise attn.AttnError(rc, "attn_decode")
+
+    for _ in range(args.warmup):
+        step()
+    if attn.status() != 0:
+        raise RuntimeError("device status after warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    evs = []
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        evs.append((a, b))
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if attn.status() != 0:
+        raise RuntimeError("device status after the timed region")
+    ms = R.max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
+    ms_per_step = ms / args.steps
+    kv = w.kv_bytes()
+    value = R.job_throughput(kv, world, ms_per_step * 1e-3) / 1e9
+    # end to end: the step's new queries copied in from pinned host memory,
+    # O and lse copied out; the key/value cache stays resident on the device
+    qh = qkv_host[0].pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    if attn.status() != 0:
+        raise RuntimeError("device status after the e2e region")
+    e2e_ms = R.max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    peaks, peak_src = load_peaks()
+    achieved = kv / (ms_per_step * 1e-3) / 1e9
+    algo_bytes = kv + 2 * q.numel() * 2 + lse.numel() * 4
+    cb = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_baseline_decode(w, qkv_host, args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC_DECODE, "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian bf16 inputs)",
+            "config": {"workload": w.name, "pass": "decode", "B": w.B, "H": w.H,
+                       "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal,
+                       "l2": ("K/V larger than L2" if flush is None else
+                              "L2 flushed between steps (outside the events)"),
+                       "parallelism": f"{world} independent replicas"},
+            "tflops": w.flops() / (ms_per_step * 1e-3) / 1e12,
+            "roofline": {"bound": "hbm", "achieved": achieved,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} HBM copy bandwidth",
+                         "traffic": load_traffic(w.name, "traffic_decode_"),
+                         "algorithmic_bytes_per_launch": algo_bytes,
+                         "kernel": f"attn_decode_kernel<{w.d}>"},
+            "cpu_baseline": cb,
+            "e2e": {"value": kv / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
+                    "h2d_bytes_per_step": qh.numel() * 2,
+                    "d2h_bytes_per_step": oh.numel() * 2 + lh.numel() * 4,
+                    "ms_per_step": e2e_ms, "steps": e2e_steps,
+                    "api": "attn.attn_decode with the new queries copied in and "
+                           "O / lse copied out; the K/V cache stays on the device"},
+            "gpu_launches": args.steps, "clocks": clk}), flush=True)
+    R.finish(world)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default=W.HEADLINE,
+                    choices=sorted(W.WORKLOADS) + sorted(W.DECODE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--pass", dest="pass_", default="fwd",
-                    choices=["fwd", "bwd", "fp8"],
+                    choices=["fwd", "bwd", "fp8", "decode"],
                     help="fwd (default): the forward hot path; bwd: attn_bwd; "
-                         "fp8: the FP8 forward with incoherent processing")
+                         "fp8: the FP8 forward with incoherent processing; "
+                         "decode: split-KV decode (decode_* workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.pass_ == "decode":
+        if args.impl == "reference":
+            ap.error("the reference arm times the forward oracle")
+        return run_decode(args)
+    if args.workload not in W.WORKLOADS:
+        ap.error(f"{args.workload} is a decode workload: use --pass decode")
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

@@ -33,7 +33,7 @@ struct DeviceState {
   uint32_t *status = nullptr;  // 4-byte device status word, lazily allocated
   bool smem_attr_set[6] = {false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
-  bool dec_attr_set[2] = {false, false};
+  bool dec_attr_set[4] = {false, false, false, false};
 };
 
 std::mutex g_mu;
@@ -276,11 +276,11 @@ int launch_quant(DeviceState &st, const attn_b200::QuantParams &p, int mode,
   return ATTN_OK;
 }
 
-template <int D>
+template <int D, int QMAX>
 int launch_decode(DeviceState &st, int variant, attn_b200::DecodeParams &p,
                   cudaStream_t stream) {
   using L = attn_b200::DecSmem<D>;
-  auto kern = attn_b200::attn_decode_kernel<D>;
+  auto kern = attn_b200::attn_decode_kernel<D, QMAX>;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!st.dec_attr_set[variant]) {
@@ -292,9 +292,10 @@ int launch_decode(DeviceState &st, int variant, attn_b200::DecodeParams &p,
       st.dec_attr_set[variant] = true;
     }
   }
-  // stream-K: an equal share of the key tiles per CTA, two CTAs per SM
+  // stream-K: an equal share of the key tiles per CTA, two CTAs per SM (one
+  // for the 16-query variant, whose registers allow one)
   int ctas = g_decode_max_ctas.load();
-  if (ctas <= 0) ctas = 2 * st.sm_count;
+  if (ctas <= 0) ctas = (QMAX <= 4 ? 2 : 1) * st.sm_count;
   if (ctas > attn_b200::kDecMaxCtas) ctas = attn_b200::kDecMaxCtas;
   const int grid0 = p.total < ctas ? p.total : ctas;
   p.per_cta = (p.total + grid0 - 1) / grid0;
@@ -730,7 +731,9 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
   p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns.load();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return d == 128 ? launch_decode<128>(*st, 0, p, s) : launch_decode<64>(*st, 1, p, s);
+  if (d == 128)
+    return Nq <= 4 ? launch_decode<128, 4>(*st, 0, p, s) : launch_decode<128, 16>(*st, 1, p, s);
+  return Nq <= 4 ? launch_decode<64, 4>(*st, 2, p, s) : launch_decode<64, 16>(*st, 3, p, s);
 }
 
 void attn_set_decode_max_ctas(int n) { g_decode_max_ctas.store(n > 0 ? n : 0); }

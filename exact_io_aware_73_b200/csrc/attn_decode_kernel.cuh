@@ -16,20 +16,25 @@
 //     B*H is;
 //   * per CTA: one producer warp (one elected lane) fills a ring of K/V
 //     stages (cp.async.bulk, one copy per 64-key K or V tile, completion on
-//     an mbarrier); eight compute warps, per tile:
+//     an mbarrier); eight compute warps each own an 8-key slice of every
+//     tile and run their own online softmax over it -- no communication
+//     between warps inside a tile:
 //       1. scores s[q][key] = (q . k) * scale * log2(e): four lanes per key,
 //          each a quarter of the dimensions, reduced by two shuffles;
-//       2. online softmax, one warp per query: tile max, running max m,
-//          p = 2^(s - m), running sum l, rescale factor alpha;
-//       3. O[q] = alpha O[q] + sum_key p v_key: one thread per (query group,
-//          pair of dimensions);
+//       2. the slice's max per query (three shuffles), the warp's running
+//          max m, p = 2^(s - m), running sum l, rescale of the warp's O;
+//       3. O[q] += sum over the 8 keys of p v_key, each lane D/32 dimensions
+//          (p broadcast from the key's lanes by shuffle);
+//     at the end of a head's share the eight warps' (m, l, O) are combined
+//     through shared memory (O in rounds of a few queries);
 //   * merge: a CTA that finished part of a head writes the part's (O_s,
 //     lse_s); the CTA that completes the head's last part (an atomic counter
 //     after a memory fence) combines them exactly,
 //     lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s.  No CTA
 //     waits for another; a head covered by one CTA is written directly.
 // Waits on the ring are bounded like the forward's; a timeout sets the
-// device status word and every compute warp leaves together.
+// device status word, and the compute warps agree at the end of the share
+// (a barrier with an AND reduction) to leave without writing.
 #pragma once
 
 #include <cstdint>
@@ -53,14 +58,14 @@ struct DecSmem {
   static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kStages * kTileBytes;
-  static constexpr uint32_t kQ = kV + kStages * kTileBytes;       // fp32 [16][D]
-  // scores, then probabilities, of the current tile: fp32 [16][64].  One
-  // buffer suffices: the barrier that opens a tile is reached only after
-  // every thread finished the previous tile's P.V step.
-  static constexpr uint32_t kS = kQ + kDecMaxQ * D * 4;
-  static constexpr uint32_t kAlpha = kS + kDecMaxQ * kDecTileKeys * 4;  // [16]
-  static constexpr uint32_t kStat = kAlpha + kDecMaxQ * 4;        // m, l [16][2]
-  static constexpr uint32_t kBars = kStat + kDecMaxQ * 8;
+  // the head's queries (fp32 [16][D], pre-scaled) while a share runs; at its
+  // end the same bytes hold the warps' O for a round of kRedQ queries
+  static constexpr uint32_t kRedBytes = 12 * 1024;
+  static constexpr int kRedQ = kRedBytes / (kDecComputeWarps * D * 4);  // 3 or 6
+  static_assert(kDecMaxQ * D * 4 <= kRedBytes, "queries fit the shared region");
+  static constexpr uint32_t kQ = kV + kStages * kTileBytes;
+  static constexpr uint32_t kStat = kQ + kRedBytes;  // m, l per warp [8][16][2]
+  static constexpr uint32_t kBars = kStat + kDecComputeWarps * kDecMaxQ * 8;
   static constexpr int FULL = 0, EMPTY = kStages, NUM_BARS = 2 * kStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;         // abort flag, last flag
   static constexpr uint32_t kBytes = kMisc + 16;
@@ -165,237 +170,230 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 
 // ------------------------------------------------------------------ compute
 
-// One head's part: write it (whole head in this CTA) or record it and, if it
-// is the last part to finish, merge all of the head's parts.
-template <int D>
-__device__ __forceinline__ void dec_finish_head(uint8_t *smem, const DecodeParams &p,
-                                                int h, int tid,
-                                                const float (&acc)[kDecMaxQ / (kDecComputeThreads / (D / 2))][2]) {
-  using L = DecSmem<D>;
-  constexpr int kPairs = D / 2;
-  constexpr int kGroups = kDecComputeThreads / kPairs;
-  constexpr int kQPer = kDecMaxQ / kGroups;
-  const float *stat = reinterpret_cast<const float *>(smem + L::kStat);
-  volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
-  const int pair = tid % kPairs, grp = tid / kPairs;
-  const int first = dec_first_cta(h, p), last = dec_last_cta(h, p);
-  const int64_t row0 = static_cast<int64_t>(h) * p.nq;
-  if (first == last) {
-#pragma unroll
-    for (int i = 0; i < kQPer; ++i) {
-      const int q = grp + i * kGroups;
-      if (q >= p.nq) continue;
-      const float m = stat[2 * q], l = stat[2 * q + 1];
-      const float inv = __frcp_rn(l);
-      reinterpret_cast<uint32_t *>(p.o + (row0 + q) * D)[pair] =
-          pack_bf16x2(acc[i][0] * inv, acc[i][1] * inv);
-      if (pair == 0) p.lse[row0 + q] = (m + lg2_approx(l)) * kLn2;
-    }
-    return;
-  }
-  const int slot = h + static_cast<int>(blockIdx.x);
-#pragma unroll
-  for (int i = 0; i < kQPer; ++i) {
-    const int q = grp + i * kGroups;
-    if (q >= p.nq) continue;
-    const float m = stat[2 * q], l = stat[2 * q + 1];
-    const bool any = l > 0.f;  // a part may see no key of a causal row
-    const float inv = any ? __frcp_rn(l) : 0.f;
-    float2 *dst = reinterpret_cast<float2 *>(p.part_o + (static_cast<int64_t>(slot) * p.nq + q) * D);
-    dst[pair] = make_float2(acc[i][0] * inv, acc[i][1] * inv);
-    if (pair == 0)
-      p.part_lse[static_cast<int64_t>(slot) * p.nq + q] =
-          any ? (m + lg2_approx(l)) * kLn2 : -CUDART_INF_F;
-  }
-  __threadfence();  // the part is visible device-wide before it is counted
-  dec_bar();
-  if (tid == 0) *last_flag = (atomicAdd(p.counters + h, 1) == last - first);
-  dec_bar();
-  if (!*last_flag) return;
-  __threadfence();
-  const int nseg = last - first + 1;
-#pragma unroll
-  for (int i = 0; i < kQPer; ++i) {
-    const int q = grp + i * kGroups;
-    if (q >= p.nq) continue;
-    float M = -CUDART_INF_F;
-    for (int s = 0; s < nseg; ++s)
-      M = fmaxf(M, __ldcg(p.part_lse + static_cast<int64_t>(h + first + s) * p.nq + q));
-    float sum = 0.f, o0 = 0.f, o1 = 0.f;
-    for (int s = 0; s < nseg; ++s) {
-      const int64_t r = static_cast<int64_t>(h + first + s) * p.nq + q;
-      const float ls = __ldcg(p.part_lse + r);
-      const float w = (ls == -CUDART_INF_F) ? 0.f : ex2_approx((ls - M) * 1.4426950408889634f);
-      const float2 po = __ldcg(reinterpret_cast<const float2 *>(p.part_o + r * D) + pair);
-      sum += w;
-      o0 = fmaf(w, po.x, o0);
-      o1 = fmaf(w, po.y, o1);
-    }
-    const float inv = __frcp_rn(sum);
-    reinterpret_cast<uint32_t *>(p.o + (row0 + q) * D)[pair] = pack_bf16x2(o0 * inv, o1 * inv);
-    if (pair == 0) p.lse[row0 + q] = M + lg2_approx(sum) * kLn2;
-  }
-  if (tid == 0) p.counters[h] = 0;  // ready for the next launch
-}
-
-template <int D>
+// One CTA's share of key tiles, head part by head part.  QMAX (4 or 16)
+// bounds the queries so that a lane's per-query state stays in registers.
+template <int D, int QMAX>
 __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
                                             const DecodeParams &p, const WaitCtx &wc,
                                             int g0, int g1, int warp, int lane) {
   using L = DecSmem<D>;
-  constexpr int kPairs = D / 2;
-  constexpr int kGroups = kDecComputeThreads / kPairs;  // 4 (d = 128) or 8
-  constexpr int kQPer = kDecMaxQ / kGroups;             // queries per thread
-  constexpr int kChunks = D / 8;                        // 16-byte chunks per row
+  constexpr int E = D / 32;        // output dimensions per lane
+  constexpr int kChunks = D / 8;   // 16-byte chunks per row
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   const int tid = warp * 32 + lane;
-  const int pair = tid % kPairs, grp = tid / kPairs;
+  const int kl = lane >> 2, q4 = lane & 3;  // key of the warp's slice, quarter
   float *qf = reinterpret_cast<float *>(smem + L::kQ);
-  float *sbuf = reinterpret_cast<float *>(smem + L::kS);
-  float *alpha_s = reinterpret_cast<float *>(smem + L::kAlpha);
+  float *red = qf;  // the same bytes once the share's last tile is done
   float *stat = reinterpret_cast<float *>(smem + L::kStat);
+  volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
   int cons = 0;
-  bool ok = true;
-  for (int g = g0; ok && g < g1;) {
+  for (int g = g0; g < g1;) {
     const int h = g / p.ntiles;
     const int gend = min(g1, (h + 1) * p.ntiles);
-    // this head's queries, scaled into log2 units
-    dec_bar();  // the previous part's readers of qf / stat are done
+    dec_bar();  // the previous part's readers of the shared region are done
     const uint16_t *qsrc = p.q + static_cast<int64_t>(h) * p.nq * D;
     for (int i = tid; i < p.nq * D; i += kDecComputeThreads)
       qf[i] = __uint_as_float(static_cast<uint32_t>(qsrc[i]) << 16) * p.c_log2;
-    float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_run[2] = {0.f, 0.f};
-    float acc[kQPer][2];
-#pragma unroll
-    for (int i = 0; i < kQPer; ++i) acc[i][0] = acc[i][1] = 0.f;
     dec_bar();
+    float m_w[QMAX], l_w[QMAX], acc[QMAX][E];
+#pragma unroll
+    for (int q = 0; q < QMAX; ++q) {
+      m_w[q] = -CUDART_INF_F;
+      l_w[q] = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[q][e] = 0.f;
+    }
+    bool ok = true;
     for (int gg = g; gg < gend; ++gg, ++cons) {
       const int j = gg - h * p.ntiles;
       const int st = cons % L::kStages;
-      const bool got = mbar_wait(bar(L::FULL + st), (cons / L::kStages) & 1, wc,
-                                 kRoleSoftmax);
-      ok = dec_bar_and(got);  // every compute thread takes the same branch
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::FULL + st), (cons / L::kStages) & 1,
+                                             wc, kRoleSoftmax));
       if (!ok) break;
       const int rows = min(kDecTileKeys, p.nk - j * kDecTileKeys);
-      const int kb = j * kDecTileKeys;
+      const int key = warp * 8 + kl;  // this lane's key within the tile
+      const bool kvalid = key < rows;
+      const int kabs = j * kDecTileKeys + key;
       const uint8_t *kt = smem + L::kK + st * L::kTileBytes;
       const uint8_t *vt = smem + L::kV + st * L::kTileBytes;
-      float *S = sbuf;
-      float *al = alpha_s;
-
-      // 1. scores: lane quarter q4 of key `key` takes chunks q4, q4 + 4, ...
-      {
-        const int key = warp * 8 + (lane >> 2), q4 = lane & 3;
-        float part[kDecMaxQ];
+      // 1. scores of the slice's 8 keys
+      float s[QMAX];
 #pragma unroll
-        for (int q = 0; q < kDecMaxQ; ++q) part[q] = 0.f;
-        if (key < rows) {
+      for (int q = 0; q < QMAX; ++q) s[q] = 0.f;
+      if (kvalid) {
 #pragma unroll
-          for (int c = 0; c < kChunks / 4; ++c) {
-            const int ch = q4 + 4 * c;
-            const uint4 raw = *reinterpret_cast<const uint4 *>(kt + key * D * 2 + ch * 16);
-            const float kf[8] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y),
-                                 bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w)};
+        for (int c = 0; c < kChunks / 4; ++c) {
+          const int ch = q4 + 4 * c;
+          const uint4 raw = *reinterpret_cast<const uint4 *>(kt + key * D * 2 + ch * 16);
+          const float kf[8] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y),
+                               bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w)};
 #pragma unroll
-            for (int q = 0; q < kDecMaxQ; ++q) {
-              if (q >= p.nq) break;
-              const float4 a = *reinterpret_cast<const float4 *>(qf + q * D + ch * 8);
-              const float4 b = *reinterpret_cast<const float4 *>(qf + q * D + ch * 8 + 4);
-              part[q] = fmaf(a.x, kf[0], fmaf(a.y, kf[1], fmaf(a.z, kf[2], fmaf(a.w, kf[3],
-                        fmaf(b.x, kf[4], fmaf(b.y, kf[5], fmaf(b.z, kf[6], fmaf(b.w, kf[7], part[q]))))))));
-            }
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < kDecMaxQ; ++q) {
-          if (q >= p.nq) break;  // uniform across the warp
-          part[q] += __shfl_xor_sync(0xffffffffu, part[q], 1);
-          part[q] += __shfl_xor_sync(0xffffffffu, part[q], 2);
-          if ((q & 3) == q4) {
-            const bool vis = key < rows && (!p.causal || kb + key <= p.nk - p.nq + q);
-            S[q * kDecTileKeys + key] = vis ? part[q] : -CUDART_INF_F;
+          for (int q = 0; q < QMAX; ++q) {
+            if (q >= p.nq) break;
+            const float4 a = *reinterpret_cast<const float4 *>(qf + q * D + ch * 8);
+            const float4 b = *reinterpret_cast<const float4 *>(qf + q * D + ch * 8 + 4);
+            s[q] = fmaf(a.x, kf[0], fmaf(a.y, kf[1], fmaf(a.z, kf[2], fmaf(a.w, kf[3],
+                   fmaf(b.x, kf[4], fmaf(b.y, kf[5], fmaf(b.z, kf[6], fmaf(b.w, kf[7], s[q]))))))));
           }
         }
       }
-      dec_bar();
-      // 2. online softmax: warp w owns queries w and w + 8
+      // 2. the warp's online softmax over its slice (all lanes of a key
+      //    hold its score; lanes 4k .. 4k+3 belong to key k)
 #pragma unroll
-      for (int qi = 0; qi < 2; ++qi) {
-        const int q = warp + 8 * qi;
-        if (q >= p.nq) continue;  // uniform across the warp
-        const float s0 = S[q * kDecTileKeys + lane], s1 = S[q * kDecTileKeys + lane + 32];
-        float tm = fmaxf(s0, s1);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, off));
-        const float mn = fmaxf(m_run[qi], tm);
-        float a = 1.f, p0 = 0.f, p1 = 0.f;
-        if (mn != -CUDART_INF_F) {  // some key of the row visible so far
-          a = ex2_approx(m_run[qi] - mn);  // 0 while nothing was visible
-          p0 = ex2_approx(s0 - mn);
-          p1 = ex2_approx(s1 - mn);
+      for (int q = 0; q < QMAX; ++q) {
+        if (q >= p.nq) break;  // uniform across the warp
+        s[q] += __shfl_xor_sync(0xffffffffu, s[q], 1);
+        s[q] += __shfl_xor_sync(0xffffffffu, s[q], 2);
+        if (!(kvalid && (!p.causal || kabs <= p.nk - p.nq + q))) s[q] = -CUDART_INF_F;
+        float tm = s[q];
+        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+        const float mn = fmaxf(m_w[q], tm);
+        float alpha = 1.f, pk = 0.f;
+        if (mn != -CUDART_INF_F) {  // a key of this slice visible so far
+          alpha = ex2_approx(m_w[q] - mn);  // 0 while none was
+          pk = ex2_approx(s[q] - mn);
         }
-        float ps = p0 + p1;
+        float ts = pk;
+        ts += __shfl_xor_sync(0xffffffffu, ts, 4);
+        ts += __shfl_xor_sync(0xffffffffu, ts, 8);
+        ts += __shfl_xor_sync(0xffffffffu, ts, 16);
+        l_w[q] = fmaf(l_w[q], alpha, ts);
+        m_w[q] = mn;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-        l_run[qi] = fmaf(l_run[qi], a, ps);
-        m_run[qi] = mn;
-        S[q * kDecTileKeys + lane] = p0;
-        S[q * kDecTileKeys + lane + 32] = p1;
-        if (lane == 0) al[q] = a;
+        for (int e = 0; e < E; ++e) acc[q][e] *= alpha;
+        s[q] = pk;
       }
-      dec_bar();
-      // 3. O[q] = alpha O[q] + sum_key p[q][key] v[key] for this thread's
-      //    pair of dimensions and queries grp, grp + kGroups, ...
+      // 3. O += p v over the slice's keys, E dimensions per lane
 #pragma unroll
-      for (int i = 0; i < kQPer; ++i) {
-        const int q = grp + i * kGroups;
-        if (q < p.nq) {
-          const float a = al[q];
-          acc[i][0] *= a;
-          acc[i][1] *= a;
+      for (int k = 0; k < 8; ++k) {
+        const int krow = warp * 8 + k;
+        if (krow >= rows) break;  // uniform across the warp
+        float vv[E];
+        if constexpr (E == 4) {
+          const uint2 w2 = *reinterpret_cast<const uint2 *>(vt + krow * D * 2 + lane * 8);
+          vv[0] = bf16lo(w2.x); vv[1] = bf16hi(w2.x); vv[2] = bf16lo(w2.y); vv[3] = bf16hi(w2.y);
+        } else {
+          const uint32_t w1 = *reinterpret_cast<const uint32_t *>(vt + krow * D * 2 + lane * 4);
+          vv[0] = bf16lo(w1); vv[1] = bf16hi(w1);
         }
-      }
-      if (grp < p.nq) {
-#pragma unroll 8
-        for (int key = 0; key < rows; ++key) {
-          const uint32_t v2 = *reinterpret_cast<const uint32_t *>(vt + key * D * 2 + pair * 4);
-          const float v0 = bf16lo(v2), v1 = bf16hi(v2);
 #pragma unroll
-          for (int i = 0; i < kQPer; ++i) {
-            const int q = grp + i * kGroups;
-            if (q < p.nq) {
-              const float pk = S[q * kDecTileKeys + key];
-              acc[i][0] = fmaf(pk, v0, acc[i][0]);
-              acc[i][1] = fmaf(pk, v1, acc[i][1]);
-            }
-          }
+        for (int q = 0; q < QMAX; ++q) {
+          if (q >= p.nq) break;
+          const float pq = __shfl_sync(0xffffffffu, s[q], 4 * k);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[q][e] = fmaf(pq, vv[e], acc[q][e]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::EMPTY + st));  // K and V of this stage read
     }
-    if (!ok) break;
-    // the part's statistics, from the softmax warps to every thread
+    if (!dec_bar_and(ok)) return;  // a wait ran out: every compute thread leaves
+
+    // ---- the eight warps' (m, l, O) combined, then written (whole head) or
+    // recorded as a part; O goes through the shared region kRedQ queries at
+    // a time.
     if (lane == 0) {
 #pragma unroll
-      for (int qi = 0; qi < 2; ++qi) {
-        const int q = warp + 8 * qi;
+      for (int q = 0; q < QMAX; ++q)
         if (q < p.nq) {
-          stat[2 * q] = m_run[qi];
-          stat[2 * q + 1] = l_run[qi];
+          stat[(warp * kDecMaxQ + q) * 2] = m_w[q];
+          stat[(warp * kDecMaxQ + q) * 2 + 1] = l_w[q];
+        }
+    }
+    const int first = dec_first_cta(h, p), last = dec_last_cta(h, p);
+    const bool whole = first == last;
+    const int slot = h + static_cast<int>(blockIdx.x);
+    const int64_t row0 = static_cast<int64_t>(h) * p.nq;
+    for (int q0 = 0; q0 < p.nq; q0 += L::kRedQ) {
+      dec_bar();  // earlier readers of the shared region are done
+#pragma unroll
+      for (int q = 0; q < QMAX; ++q)
+        if (q >= q0 && q < q0 + L::kRedQ && q < p.nq) {
+          float *dst = red + (warp * L::kRedQ + (q - q0)) * D + lane * E;
+          if constexpr (E == 4)
+            *reinterpret_cast<float4 *>(dst) = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+          else
+            *reinterpret_cast<float2 *>(dst) = make_float2(acc[q][0], acc[q][1]);
+        }
+      dec_bar();
+      const int nr = min(L::kRedQ, p.nq - q0);
+      for (int item = tid; item < nr * (D / 2); item += kDecComputeThreads) {
+        const int ql = item / (D / 2), pair = item - ql * (D / 2);
+        const int q = q0 + ql;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < kDecComputeWarps; ++w)
+          M = fmaxf(M, stat[(w * kDecMaxQ + q) * 2]);
+        float lsum = 0.f, o0 = 0.f, o1 = 0.f;
+        if (M != -CUDART_INF_F) {
+#pragma unroll
+          for (int w = 0; w < kDecComputeWarps; ++w) {
+            const float mw = stat[(w * kDecMaxQ + q) * 2];
+            if (mw == -CUDART_INF_F) continue;
+            const float f = ex2_approx(mw - M);
+            lsum = fmaf(f, stat[(w * kDecMaxQ + q) * 2 + 1], lsum);
+            const float2 r = *reinterpret_cast<const float2 *>(
+                red + (w * L::kRedQ + ql) * D + 2 * pair);
+            o0 = fmaf(f, r.x, o0);
+            o1 = fmaf(f, r.y, o1);
+          }
+        }
+        const bool any = lsum > 0.f;  // a part may see no key of a causal row
+        const float inv = any ? __frcp_rn(lsum) : 0.f;
+        const float lse2 = any ? M + lg2_approx(lsum) : -CUDART_INF_F;  // log2 units
+        if (whole) {
+          reinterpret_cast<uint32_t *>(p.o + (row0 + q) * D)[pair] =
+              pack_bf16x2(o0 * inv, o1 * inv);
+          if (pair == 0) p.lse[row0 + q] = lse2 * kLn2;
+        } else {
+          reinterpret_cast<float2 *>(p.part_o + (static_cast<int64_t>(slot) * p.nq + q) * D)[pair] =
+              make_float2(o0 * inv, o1 * inv);
+          if (pair == 0)
+            p.part_lse[static_cast<int64_t>(slot) * p.nq + q] = any ? lse2 * kLn2 : -CUDART_INF_F;
         }
       }
     }
-    dec_bar();
-    dec_finish_head<D>(smem, p, h, tid, acc);
+    if (!whole) {
+      __threadfence();  // the part is visible device-wide before it is counted
+      dec_bar();
+      if (tid == 0) *last_flag = (atomicAdd(p.counters + h, 1) == last - first);
+      dec_bar();
+      if (*last_flag) {
+        __threadfence();
+        const int nseg = last - first + 1;
+        for (int item = tid; item < p.nq * (D / 2); item += kDecComputeThreads) {
+          const int q = item / (D / 2), pair = item - q * (D / 2);
+          float M = -CUDART_INF_F;
+          for (int sgi = 0; sgi < nseg; ++sgi)
+            M = fmaxf(M, __ldcg(p.part_lse + static_cast<int64_t>(h + first + sgi) * p.nq + q));
+          float sum = 0.f, o0 = 0.f, o1 = 0.f;
+          for (int sgi = 0; sgi < nseg; ++sgi) {
+            const int64_t r = static_cast<int64_t>(h + first + sgi) * p.nq + q;
+            const float ls = __ldcg(p.part_lse + r);
+            if (ls == -CUDART_INF_F) continue;
+            const float wgt = ex2_approx((ls - M) * 1.4426950408889634f);
+            const float2 po = __ldcg(reinterpret_cast<const float2 *>(p.part_o + r * D) + pair);
+            sum += wgt;
+            o0 = fmaf(wgt, po.x, o0);
+            o1 = fmaf(wgt, po.y, o1);
+          }
+          const float inv = __frcp_rn(sum);
+          reinterpret_cast<uint32_t *>(p.o + (row0 + q) * D)[pair] = pack_bf16x2(o0 * inv, o1 * inv);
+          if (pair == 0) p.lse[row0 + q] = M + lg2_approx(sum) * kLn2;
+        }
+        if (tid == 0) p.counters[h] = 0;  // ready for the next launch
+      }
+    }
     g = gend;
   }
 }
 
 // ------------------------------------------------------------------ kernel
 
-template <int D>
-__global__ void __launch_bounds__(kDecThreads, 2)
+template <int D, int QMAX>
+__global__ void __launch_bounds__(kDecThreads, QMAX <= 4 ? 2 : 1)
     attn_decode_kernel(const DecodeParams p) {
   using L = DecSmem<D>;
   extern __shared__ __align__(128) uint8_t dsmem[];
@@ -418,7 +416,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (lane == 0) dec_producer<D>(base, p, wc, g0, g1);
     __syncwarp();
   } else {
-    dec_compute<D>(base, dsmem, p, wc, g0, g1, warp, lane);
+    dec_compute<D, QMAX>(base, dsmem, p, wc, g0, g1, warp, lane);
   }
   __syncthreads();
 }
