@@ -21,10 +21,12 @@
 //     between warps inside a tile:
 //       1. scores s[q][key] = (q . k) * scale * log2(e): four lanes per key,
 //          each a quarter of the dimensions, reduced by two shuffles;
-//       2. the slice's max per query (three shuffles), the warp's running
-//          max m, p = 2^(s - m), running sum l, rescale of the warp's O;
+//       2. p = 2^(s - m) against the warp's running reference m, which
+//          moves (with a rescale of l and O) only when a score exceeds it by
+//          more than 2^8 -- a warp vote per query, the maximum reduction
+//          only when the vote says so; each lane keeps its own part of l;
 //       3. O[q] += sum over the 8 keys of p v_key, each lane D/32 dimensions
-//          (p broadcast from the key's lanes by shuffle);
+//          (p passed through the warp's slice of shared memory);
 //     at the end of a head's share the eight warps' (m, l, O) are combined
 //     through shared memory (O in rounds of a few queries);
 //   * merge: a CTA that finished part of a head writes the part's (O_s,
@@ -51,6 +53,7 @@ constexpr int kDecComputeWarps = 8;
 constexpr int kDecComputeThreads = kDecComputeWarps * 32;
 constexpr int kDecThreads = kDecComputeThreads + 32;  // + producer warp
 constexpr int kDecMaxCtas = 1024;      // bound on the grid (workspace sizing)
+constexpr float kDecLazy = 8.f;        // log2 units: p <= 2^8
 
 template <int D>
 struct DecSmem {
@@ -60,11 +63,13 @@ struct DecSmem {
   static constexpr uint32_t kV = kK + kStages * kTileBytes;
   // the head's queries (fp32 [16][D], pre-scaled) while a share runs; at its
   // end the same bytes hold the warps' O for a round of kRedQ queries
-  static constexpr uint32_t kRedBytes = 12 * 1024;
-  static constexpr int kRedQ = kRedBytes / (kDecComputeWarps * D * 4);  // 3 or 6
+  static constexpr uint32_t kRedBytes = 8 * 1024;
+  static constexpr int kRedQ = kRedBytes / (kDecComputeWarps * D * 4);  // 2 or 4
   static_assert(kDecMaxQ * D * 4 <= kRedBytes, "queries fit the shared region");
   static constexpr uint32_t kQ = kV + kStages * kTileBytes;
-  static constexpr uint32_t kStat = kQ + kRedBytes;  // m, l per warp [8][16][2]
+  // each warp's probabilities of its current slice, [8 keys][16 queries]
+  static constexpr uint32_t kP = kQ + kRedBytes;
+  static constexpr uint32_t kStat = kP + kDecComputeWarps * 8 * kDecMaxQ * 4;  // m, l [8][16][2]
   static constexpr uint32_t kBars = kStat + kDecComputeWarps * kDecMaxQ * 8;
   static constexpr int FULL = 0, EMPTY = kStages, NUM_BARS = 2 * kStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;         // abort flag, last flag
@@ -185,6 +190,7 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
   float *qf = reinterpret_cast<float *>(smem + L::kQ);
   float *red = qf;  // the same bytes once the share's last tile is done
   float *stat = reinterpret_cast<float *>(smem + L::kStat);
+  float *pw = reinterpret_cast<float *>(smem + L::kP) + warp * 8 * kDecMaxQ;
   volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
   int cons = 0;
   for (int g = g0; g < g1;) {
@@ -245,26 +251,24 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
         s[q] += __shfl_xor_sync(0xffffffffu, s[q], 1);
         s[q] += __shfl_xor_sync(0xffffffffu, s[q], 2);
         if (!(kvalid && (!p.causal || kabs <= p.nk - p.nq + q))) s[q] = -CUDART_INF_F;
-        float tm = s[q];
-        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
-        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
-        tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
-        const float mn = fmaxf(m_w[q], tm);
-        float alpha = 1.f, pk = 0.f;
-        if (mn != -CUDART_INF_F) {  // a key of this slice visible so far
-          alpha = ex2_approx(m_w[q] - mn);  // 0 while none was
-          pk = ex2_approx(s[q] - mn);
-        }
-        float ts = pk;
-        ts += __shfl_xor_sync(0xffffffffu, ts, 4);
-        ts += __shfl_xor_sync(0xffffffffu, ts, 8);
-        ts += __shfl_xor_sync(0xffffffffu, ts, 16);
-        l_w[q] = fmaf(l_w[q], alpha, ts);
-        m_w[q] = mn;
+        if (__any_sync(0xffffffffu, s[q] > m_w[q] + kDecLazy)) {
+          float tm = s[q];
+          tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+          tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+          tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+          const float mn = fmaxf(m_w[q], tm);  // finite: some score beat m
+          const float alpha = ex2_approx(m_w[q] - mn);  // 0 while m was -inf
+          l_w[q] *= alpha;
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[q][e] *= alpha;
-        s[q] = pk;
+          for (int e = 0; e < E; ++e) acc[q][e] *= alpha;
+          m_w[q] = mn;
+        }
+        // p <= 2^8; no visible key yet (m = -inf) means p = 0
+        const float pk = (m_w[q] == -CUDART_INF_F) ? 0.f : ex2_approx(s[q] - m_w[q]);
+        l_w[q] += pk;  // each of the key's four lanes adds it: l = sum / 4
+        if ((q & 3) == q4) pw[kl * kDecMaxQ + q] = pk;
       }
+      __syncwarp();
       // 3. O += p v over the slice's keys, E dimensions per lane
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -279,17 +283,31 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
           vv[0] = bf16lo(w1); vv[1] = bf16hi(w1);
         }
 #pragma unroll
-        for (int q = 0; q < QMAX; ++q) {
-          if (q >= p.nq) break;
-          const float pq = __shfl_sync(0xffffffffu, s[q], 4 * k);
+        for (int q4b = 0; q4b < QMAX; q4b += 4) {
+          if (q4b >= p.nq) break;
+          const float4 pq = *reinterpret_cast<const float4 *>(pw + k * kDecMaxQ + q4b);
+          const float pv4[4] = {pq.x, pq.y, pq.z, pq.w};
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[q][e] = fmaf(pq, vv[e], acc[q][e]);
+          for (int qq = 0; qq < 4; ++qq) {
+            if (q4b + qq >= p.nq) break;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+              acc[q4b + qq][e] = fmaf(pv4[qq], vv[e], acc[q4b + qq][e]);
+          }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::EMPTY + st));  // K and V of this stage read
     }
     if (!dec_bar_and(ok)) return;  // a wait ran out: every compute thread leaves
+#pragma unroll
+    for (int q = 0; q < QMAX; ++q) {
+      if (q >= p.nq) break;
+      float t = l_w[q];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+      l_w[q] = 0.25f * t;  // every key's p was added by its four lanes
+    }
 
     // ---- the eight warps' (m, l, O) combined, then written (whole head) or
     // recorded as a part; O goes through the shared region kRedQ queries at
