@@ -47,13 +47,14 @@ CSRC = os.path.join(ROOT, "exact_io_aware_73_b200", "csrc")
 
 
 KERNEL_SOURCES = ("attn_fwd_kernel.cuh", "ptx_sm100.cuh")
+DECODE_SOURCES = ("attn_decode_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
     """Hash of the device-code sources; a committed traffic figure is only
     used while it matches (the counters describe that exact kernel)."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
@@ -69,7 +70,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def load_traffic(workload: str, prefix: str = "traffic_"):
+def load_traffic(workload: str, prefix: str = "traffic_", sources=KERNEL_SOURCES):
     """DRAM bytes per launch from a committed ncu capture of this workload,
     or None when there is none or the kernel changed since it was taken."""
     path = os.path.join(ROOT, "profiles", f"{prefix}{workload}.json")
@@ -78,7 +79,7 @@ def load_traffic(workload: str, prefix: str = "traffic_"):
             t = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("kernel_source_hash") != kernel_source_hash():
+    if t.get("kernel_source_hash") != kernel_source_hash(sources):
         return None
     return t.get("dram_bytes_per_launch")
 
@@ -663,7 +664,8 @@ def run_decode(args):
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} HBM copy bandwidth",
-                         "traffic": load_traffic(w.name, "traffic_decode_"),
+                         "traffic": load_traffic(w.name, "traffic_decode_",
+                                                 DECODE_SOURCES),
                          "algorithmic_bytes_per_launch": algo_bytes,
                          "kernel": f"attn_decode_kernel<{w.d}>"},
             "cpu_baseline": cb,
