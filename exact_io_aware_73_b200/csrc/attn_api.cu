@@ -216,6 +216,41 @@ int launch(DeviceState &st, int variant, const CUtensorMap *maps,
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// attn_fwd_host's copy / compute pipeline: three streams and their events,
+// created once per device on first use and kept until process exit.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+  bool ready = false;
+  std::mutex mu;  // one call enqueues at a time (events are reused)
+  cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t in_done[kHostChunks] = {}, k_done[kHostChunks] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+
+int host_pipe(int dev, HostPipe **out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  HostPipe &hp = g_pipe[dev];
+  if (!hp.ready) {
+    const unsigned fl = cudaStreamNonBlocking;
+    bool ok = cudaStreamCreateWithFlags(&hp.h2d, fl) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.comp, fl) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.d2h, fl) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.end, cudaEventDisableTiming) == cudaSuccess;
+    for (int c = 0; ok && c < kHostChunks; ++c)
+      ok = cudaEventCreateWithFlags(&hp.in_done[c], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.k_done[c], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    hp.ready = true;
+  }
+  *out = &hp;
+  return ATTN_OK;
+}
+
 // fp32 vectors [bh, npad] (npad a multiple of 128) as a 2-D tensor with
 // 128-entry boxes: row stride npad * 4 bytes and every box start (x = 128 i)
 // are 512-byte multiples.
@@ -401,29 +436,58 @@ int attn_fwd_host(const void *q, const void *k, const void *v, void *o,
   if (!workspace || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
     return ATTN_ERR_WORKSPACE;
-  const size_t rows = static_cast<size_t>(B) * H * N;
+  const int bh = B * H;
+  const size_t rows = static_cast<size_t>(bh) * N;
   const size_t tb = rows * d * 2, tbr = round256(tb);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  void *dq = ws, *dk = ws + tbr, *dv = ws + 2 * tbr, *dout = ws + 3 * tbr;
+  uint8_t *dq = ws, *dk = ws + tbr, *dv = ws + 2 * tbr, *dout = ws + 3 * tbr;
   float *dl = reinterpret_cast<float *>(ws + 4 * tbr);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int dev;
   DeviceState *st;
   if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
-  if (cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
+  HostPipe *hp = nullptr;
+  if ((rc = host_pipe(dev, &hp)) != ATTN_OK) return rc;
+  // Heads are split into chunks; chunk i's copies in, kernel and copies out
+  // run on three streams so that they overlap chunk i+1's copies in and
+  // chunk i-1's copies out.  `stream` orders the whole call: the streams
+  // start after its earlier work and it waits for the last copy out.
+  const int nchunks = (tb >= (32u << 20)) ? (bh < kHostChunks ? bh : kHostChunks) : 1;
+  const int per = (bh + nchunks - 1) / nchunks;
+  std::lock_guard<std::mutex> lk(hp->mu);
+  auto fail = [] { cudaGetLastError(); return ATTN_ERR_CUDA; };
+  if (cudaEventRecord(hp->start, s) != cudaSuccess) return fail();
+  for (cudaStream_t t : {hp->h2d, hp->comp, hp->d2h})
+    if (cudaStreamWaitEvent(t, hp->start, 0) != cudaSuccess) return fail();
+  for (int c = 0; c < nchunks; ++c) {
+    const int h0 = c * per;
+    const int nh = (bh - h0 < per) ? (bh - h0) : per;
+    if (nh <= 0) break;
+    const size_t off = static_cast<size_t>(h0) * N * d * 2;
+    const size_t len = static_cast<size_t>(nh) * N * d * 2;
+    const size_t loff = static_cast<size_t>(h0) * N, llen = static_cast<size_t>(nh) * N;
+    const uint8_t *hq = static_cast<const uint8_t *>(q), *hk = static_cast<const uint8_t *>(k),
+                  *hv = static_cast<const uint8_t *>(v);
+    if (cudaMemcpyAsync(dq + off, hq + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dk + off, hk + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dv + off, hv + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaEventRecord(hp->in_done[c], hp->h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->comp, hp->in_done[c], 0) != cudaSuccess)
+      return fail();
+    rc = attn_fwd(dq + off, dk + off, dv + off, dout + off, dl + loff, 1, nh, N, d, causal,
+                  scale, reinterpret_cast<attn_stream_t>(hp->comp));
+    if (rc != ATTN_OK) return rc;
+    if (cudaEventRecord(hp->k_done[c], hp->comp) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->d2h, hp->k_done[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t *>(o) + off, dout + off, len,
+                        cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess ||
+        cudaMemcpyAsync(lse + loff, dl + loff, llen * 4, cudaMemcpyDeviceToHost,
+                        hp->d2h) != cudaSuccess)
+      return fail();
   }
-  rc = attn_fwd(dq, dk, dv, dout, dl, B, H, N, d, causal, scale, stream);
-  if (rc != ATTN_OK) return rc;
-  if (cudaMemcpyAsync(o, dout, tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemcpyAsync(lse, dl, rows * 4, cudaMemcpyDeviceToHost, s) !=
-          cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
+  if (cudaEventRecord(hp->end, hp->d2h) != cudaSuccess ||
+      cudaStreamWaitEvent(s, hp->end, 0) != cudaSuccess)
+    return fail();
   return ATTN_OK;
 }
 

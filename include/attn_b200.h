@@ -107,12 +107,18 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
 /*
  * attn_fwd_host -- the same operation on HOST buffers, end to end.
  *
- * Queues on `stream`: copies of q, k, v from the host into `workspace`, the
- * attn_fwd kernel on the workspace copies, and copies of o and lse back into
- * the host buffers.  Returns once queued; the host outputs are valid after
- * the stream is synchronised.  For asynchronous copies the host buffers must
- * be page-locked (cudaHostAlloc / pinned); pageable buffers work but the
- * copies then block the calling thread.
+ * Copies q, k, v from the host into `workspace`, runs the attn_fwd kernel on
+ * the copies, and copies o and lse back into the host buffers.  Problems of
+ * 32 MiB or more per tensor are split by heads into up to 8 chunks whose
+ * copies in, kernels and copies out overlap on three library-owned streams
+ * (created on the device's first call, kept until process exit; make that
+ * first call outside any stream capture).  The whole call is ordered on
+ * `stream`: it starts after work already queued there, and work queued
+ * there afterwards starts after its last copy out.  Returns once queued; the
+ * host outputs are valid after `stream` is synchronised.  For asynchronous,
+ * overlapping copies the host buffers must be page-locked (cudaHostAlloc /
+ * pinned); pageable buffers work but the copies then block the calling
+ * thread.  Calls on one device enqueue one at a time (a library mutex).
  *
  *   workspace        device memory of at least attn_fwd_host_workspace_bytes
  *                    (B, H, N, d) bytes, 256-byte aligned, caller-owned.

@@ -227,6 +227,32 @@ def test_host_buffer_entry_matches_device_entry():
     assert torch.equal(o_h, o_dev.cpu()) and torch.equal(l_h, l_dev.cpu())
 
 
+def test_host_buffer_entry_chunked_pipeline_matches_device_entry():
+    """Large problems go through attn_fwd_host's copy / compute pipeline
+    (heads in chunks on three streams); 13 heads make a ragged last chunk.
+    Every head is computed by the same kernel either way, so the outputs
+    match the device entry bit for bit, and work queued on the caller's
+    stream afterwards sees them."""
+    w = W.shape_case(1, 13, 16384, 128, False, seed=11)
+    q, k, v = W.make_qkv(w)
+    assert q.numel() * 2 >= 32 << 20
+    o_dev, l_dev = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=False)
+    qp, kp, vp = (t.pin_memory() for t in (q, k, v))
+    o_h = torch.empty_like(q).pin_memory()
+    l_h = torch.empty(1, 13, 16384, dtype=torch.float32).pin_memory()
+    ws = torch.empty(attn.host_workspace_bytes(1, 13, 16384, 128),
+                     dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        attn.attn_fwd_host(qp, kp, vp, o_h, l_h, False, w.scale, ws,
+                           stream=stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+    done.synchronize()
+    assert attn.status() == 0
+    assert torch.equal(o_h, o_dev.cpu()) and torch.equal(l_h, l_dev.cpu())
+
+
 def test_device_errors_are_reported():
     q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16, device="cuda")
     buf = torch.zeros(2 * 64 * 64 + 8, dtype=torch.bfloat16, device="cuda")
