@@ -1,7 +1,7 @@
 """Benchmark of the B200 exact attention forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--pass fwd|bwd|fp8|decode]
+                    [--impl ours|reference] [--pass fwd|bwd|fp8|decode|seqpar]
                     [--no-cpu-baseline]
 
 A step is one attention forward pass over the whole workload (default: the
@@ -680,6 +680,88 @@ def run_decode(args):
     return 0
 
 
+METRIC_SEQPAR = ("attention fwd TFLOP/s, one sequence sharded over ranks "
+                 "(ring of K/V shards + exact lse merge)")
+
+
+def run_seqpar(args, w):
+    """Sequence-sharded forward: the workload's sequence split into P
+    contiguous shards.  Under torchrun each rank holds one shard and the K/V
+    shards go around the ring (NCCL point-to-point); with one process and
+    --shards P > 1 the P ranks run emulated on the one GPU, one after
+    another (the same blocks and merges, no exchange)."""
+    import torch
+    from exact_io_aware_73_b200 import attn, seqpar
+    world, rank, local = R.env_ranks()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    R.init("nccl", world, device=dev)
+    shards = world if world > 1 else max(1, args.shards)
+    if w.N % shards:
+        raise SystemExit(f"N = {w.N} is not a multiple of {shards} shards")
+    q, k, v = (t.to(dev) for t in W.make_qkv(w))
+    n = w.N // shards
+    if world > 1:
+        sl = slice(rank * n, (rank + 1) * n)
+        q, k, v = (t[:, :, sl].contiguous() for t in (q, k, v))
+
+        def step():
+            return seqpar.ring_attention(q, k, v, w.causal, w.scale)
+    else:
+        qs, ks, vs = (seqpar.shard(t, shards) for t in (q, k, v))
+        del q, k, v
+
+        def step():
+            return seqpar.ring_attention_emulated(qs, ks, vs, w.causal, w.scale)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step()
+    if attn.status() != 0:
+        raise RuntimeError("device status after warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if attn.status() != 0:
+        raise RuntimeError("device status after the timed region")
+    ms_per_step = R.max_over_ranks(a.elapsed_time(b), world, dev) / args.steps
+    flops = w.flops()
+    value = flops / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC_SEQPAR, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian bf16 inputs)",
+            "config": {"workload": w.name, "pass": "seqpar", "shards": shards,
+                       "emulated": world == 1 and shards > 1, "B": w.B, "H": w.H,
+                       "N": w.N, "d": w.d, "causal": w.causal,
+                       "l2": "inputs larger than L2" if 3 * w.B * w.H * w.N * w.d * 2 > L2_BYTES
+                             else "inputs may stay in L2",
+                       "parallelism": (f"sequence sharded over {world} ranks" if world > 1
+                                       else f"{shards} shards emulated on one GPU")},
+            "roofline": {"bound": "tensor", "achieved": value,
+                         "peak": peaks["bf16_tflops"] * world, "unit": "TFLOP/s",
+                         "frac": value / (peaks["bf16_tflops"] * world),
+                         "peak_source": f"{peak_src} bf16 burst (cuBLAS) x ranks",
+                         "traffic": None},
+            "cpu_baseline": None, "e2e": None,
+            "gpu_launches": None, "clocks": clk}), flush=True)
+    R.finish(world)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -689,10 +771,13 @@ def main():
                     choices=sorted(W.WORKLOADS) + sorted(W.DECODE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--pass", dest="pass_", default="fwd",
-                    choices=["fwd", "bwd", "fp8", "decode"],
+                    choices=["fwd", "bwd", "fp8", "decode", "seqpar"],
                     help="fwd (default): the forward hot path; bwd: attn_bwd; "
                          "fp8: the FP8 forward with incoherent processing; "
-                         "decode: split-KV decode (decode_* workloads)")
+                         "decode: split-KV decode (decode_* workloads); "
+                         "seqpar: one sequence sharded over ranks")
+    ap.add_argument("--shards", type=int, default=1,
+                    help="seqpar on one process: shards emulated on one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     args = ap.parse_args()
@@ -711,6 +796,8 @@ def main():
         return run_backward(args, w)
     if args.pass_ == "fp8":
         return run_fp8(args, w)
+    if args.pass_ == "seqpar":
+        return run_seqpar(args, w)
 
     import torch
     from exact_io_aware_73_b200 import attn

@@ -420,3 +420,42 @@ def attn_decode(q, k, v, causal: bool = True, scale: float | None = None,
                          _stream_handle(stream))
     _check(rc, "attn_decode")
     return out, lse
+
+
+# ------------------------------------------------------------------ merge
+
+def _merge_fns():
+    L = lib()
+    if L.attn_merge_fold.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        L.attn_merge_fold.argtypes = [vp, vp, vp, vp, ctypes.c_int64, i, i, vp]
+        L.attn_merge_fold.restype = i
+        L.attn_merge_finish.argtypes = [vp, vp, vp, vp, ctypes.c_int64, i, vp]
+        L.attn_merge_finish.restype = i
+    return L
+
+
+def merge_fold(acc_o, acc_lse, part_o, part_lse, first: bool, stream=None):
+    """Fold a partial result (part_o bf16 [..., d], part_lse fp32 [...]) into
+    the fp32 accumulator (acc_o [..., d], acc_lse [...]) by the exact
+    log-sum-exp merge; `first` initialises the accumulator."""
+    d = part_o.shape[-1]
+    rows = part_lse.numel()
+    rc = _merge_fns().attn_merge_fold(acc_o.data_ptr(), acc_lse.data_ptr(),
+                                      part_o.data_ptr(), part_lse.data_ptr(),
+                                      rows, d, int(bool(first)),
+                                      _stream_handle(stream))
+    _check(rc, "attn_merge_fold")
+
+
+def merge_finish(acc_o, acc_lse, stream=None):
+    """(O bf16, lse fp32) from a merge accumulator."""
+    import torch
+    o = torch.empty(acc_o.shape, dtype=torch.bfloat16, device=acc_o.device)
+    lse = torch.empty_like(acc_lse)
+    rc = _merge_fns().attn_merge_finish(acc_o.data_ptr(), acc_lse.data_ptr(),
+                                        o.data_ptr(), lse.data_ptr(),
+                                        acc_lse.numel(), acc_o.shape[-1],
+                                        _stream_handle(stream))
+    _check(rc, "attn_merge_finish")
+    return o, lse

@@ -17,6 +17,7 @@
 #include "attn_bwd_kernel.cuh"
 #include "fp8_quant_kernel.cuh"
 #include "attn_decode_kernel.cuh"
+#include "attn_merge_kernel.cuh"
 
 namespace {
 
@@ -801,6 +802,70 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
 }
 
 void attn_set_decode_max_ctas(int n) { g_decode_max_ctas.store(n > 0 ? n : 0); }
+
+int attn_merge_fold(float *acc_o, float *acc_lse, const void *part_o,
+                    const float *part_lse, int64_t rows, int d, int first,
+                    attn_stream_t stream) {
+  if (rows < 0) return ATTN_ERR_INVALID_SIZE;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  if (rows == 0) return ATTN_OK;
+  if (!acc_o || !acc_lse || !part_o || !part_lse) return ATTN_ERR_NULL_POINTER;
+  if (!aligned(acc_o, 16) || !aligned(part_o, 16) || !aligned(acc_lse, 4) ||
+      !aligned(part_lse, 4))
+    return ATTN_ERR_MISALIGNED;
+  const size_t ob = static_cast<size_t>(rows) * d * 4, lb = static_cast<size_t>(rows) * 4;
+  if (overlaps(acc_o, ob, part_o, ob / 2) || overlaps(acc_o, ob, part_lse, lb) ||
+      overlaps(acc_lse, lb, part_o, ob / 2) || overlaps(acc_lse, lb, part_lse, lb) ||
+      overlaps(acc_o, ob, acc_lse, lb))
+    return ATTN_ERR_ALIAS;
+  int rc, dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  const void *all[4] = {acc_o, acc_lse, part_o, part_lse};
+  for (const void *ptr : all)
+    if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
+  const int64_t want = (rows + 7) / 8;
+  const int blocks = static_cast<int>(want < st->sm_count * 16 ? want : st->sm_count * 16);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t *po = static_cast<const uint16_t *>(part_o);
+  if (d == 128)
+    attn_b200::attn_merge_fold_kernel<128><<<blocks, 256, 0, s>>>(acc_o, acc_lse, po, part_lse, rows, first);
+  else
+    attn_b200::attn_merge_fold_kernel<64><<<blocks, 256, 0, s>>>(acc_o, acc_lse, po, part_lse, rows, first);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+int attn_merge_finish(const float *acc_o, const float *acc_lse, void *o, float *lse,
+                      int64_t rows, int d, attn_stream_t stream) {
+  if (rows < 0) return ATTN_ERR_INVALID_SIZE;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  if (rows == 0) return ATTN_OK;
+  if (!acc_o || !acc_lse || !o || !lse) return ATTN_ERR_NULL_POINTER;
+  if (!aligned(acc_o, 16) || !aligned(o, 16) || !aligned(acc_lse, 4) || !aligned(lse, 4))
+    return ATTN_ERR_MISALIGNED;
+  const size_t ob = static_cast<size_t>(rows) * d * 4, lb = static_cast<size_t>(rows) * 4;
+  if (overlaps(o, ob / 2, acc_o, ob) || overlaps(o, ob / 2, acc_lse, lb) ||
+      overlaps(lse, lb, acc_o, ob) || overlaps(lse, lb, o, ob / 2) ||
+      (lse != acc_lse && overlaps(lse, lb, acc_lse, lb)))
+    return ATTN_ERR_ALIAS;
+  int rc, dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  const void *all[4] = {acc_o, acc_lse, o, lse};
+  for (const void *ptr : all)
+    if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
+  const int64_t want = (rows + 7) / 8;
+  const int blocks = static_cast<int>(want < st->sm_count * 16 ? want : st->sm_count * 16);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint16_t *oo = static_cast<uint16_t *>(o);
+  if (d == 128)
+    attn_b200::attn_merge_finish_kernel<128><<<blocks, 256, 0, s>>>(acc_o, acc_lse, oo, lse, rows);
+  else
+    attn_b200::attn_merge_finish_kernel<64><<<blocks, 256, 0, s>>>(acc_o, acc_lse, oo, lse, rows);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
 
 int attn_status(attn_stream_t stream) {
   int dev = -1;

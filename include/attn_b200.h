@@ -356,6 +356,31 @@ size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d);
  * so that small problems can be split over many CTAs.  Process-wide. */
 void attn_set_decode_max_ctas(int n);
 
+/*
+ * Merging partial attention results -- the softmax statistics kept per row
+ * (the marketmaker.cc post's section "Backward pass", folded into lse) make
+ * attention over disjoint key sets exactly combinable:
+ *     lse = log sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
+ * This is what sequence-sharded attention over several devices needs (the
+ * briefgpt.xyz summary page of FlashAttention-2, arXiv 2307.08691, entry
+ * "BurstAttention"): each device attends its queries to one shard of the
+ * keys at a time and folds the result in.
+ *
+ * attn_merge_fold: fold one part (part_o bf16 [rows, d], part_lse fp32
+ * [rows], as attn_fwd writes them) into the accumulator (acc_o fp32 [rows, d],
+ * acc_lse fp32 [rows]); first != 0 initialises the accumulator from the part.
+ * A row that sees no key in a part must have part_lse = -inf there.
+ * attn_merge_finish: o = bf16(acc_o), lse = acc_lse (lse may equal acc_lse).
+ * rows = B * H * N_queries; d in {64, 128}; acc_o, part_o, o 16-byte
+ * aligned, the lse arrays 4-byte aligned, device memory of the current
+ * device, outputs not overlapping inputs.  Queued on `stream`.
+ */
+int attn_merge_fold(float *acc_o, float *acc_lse, const void *part_o,
+                    const float *part_lse, int64_t rows, int d, int first,
+                    attn_stream_t stream);
+int attn_merge_finish(const float *acc_o, const float *acc_lse, void *o, float *lse,
+                      int64_t rows, int d, attn_stream_t stream);
+
 /* Human-readable text for an error code (static string, never NULL). */
 const char *attn_strerror(int code);
 

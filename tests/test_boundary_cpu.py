@@ -198,3 +198,16 @@ def test_decode_entry_refuses_bad_arguments_without_a_device(attn):
     slots = B * H + 1024
     assert attn.decode_workspace_bytes(B, H, Nq, 1000, d) == \
         r(slots * Nq * d * 4) + r(slots * Nq * 4) + r(B * H * 4)
+
+
+def test_merge_entries_refuse_bad_arguments_without_a_device(attn):
+    far = 1 << 40
+    L = attn._merge_fns()
+    assert L.attn_merge_fold(far, 2 * far, 3 * far, 4 * far, 10, 96, 1, None) == 3
+    assert L.attn_merge_fold(far, 2 * far, 3 * far, 4 * far, -1, 128, 1, None) == 2
+    assert L.attn_merge_fold(None, 2 * far, 3 * far, 4 * far, 10, 128, 1, None) == 1
+    assert L.attn_merge_fold(far + 4, 2 * far, 3 * far, 4 * far, 10, 128, 1, None) == 4
+    assert L.attn_merge_fold(far, 2 * far, far + 64, 4 * far, 10, 128, 1, None) == 6
+    assert L.attn_merge_fold(None, None, None, None, 0, 128, 1, None) == 0
+    assert L.attn_merge_finish(far, 2 * far, 3 * far, 4 * far, 10, 100, None) == 3
+    assert L.attn_merge_finish(far, 2 * far, far + 16, 4 * far, 10, 64, None) == 6
