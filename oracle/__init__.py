@@ -32,4 +32,5 @@ from .oracle import (  # noqa: F401
     quantize_qkv_fp8,
     attention_decode,
     attention_decode_rows_bf16,
+    attention_backward_rows_bf16,
 )

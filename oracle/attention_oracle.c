@@ -503,6 +503,109 @@ int oracle_attention_backward_f64(const double *Q, const double *K,
 }
 
 /* Threads OpenMP would use by default (for reporting). */
+/* Backward on sampled rows of ONE head of bf16 inputs (raw bit patterns,
+ * Q, K, V, dO each [N, d]): dQ for query rows qrows[0..nq) and dK, dV for
+ * key rows krows[0..nk), the same formulas as oracle_attention_backward_f64.
+ * Every row's lse and D_i = sum_t dO_it O_it come first (the whole forward of
+ * the head, O(N^2 d)); then each sampled query row needs its score row, and
+ * each sampled key row one column of P and dS over all queries.  For the
+ * full-size checks, where the full backward would take too long. */
+int oracle_attention_backward_rows_bf16(
+    const uint16_t *Qb, const uint16_t *Kb, const uint16_t *Vb,
+    const uint16_t *dOb, int64_t N, int64_t d, int causal, double scale,
+    const int64_t *qrows, int64_t nq, double *dQ, const int64_t *krows,
+    int64_t nk, double *dK, double *dV, int nthreads) {
+  if (!Qb || !Kb || !Vb || !dOb || N < 1 || d < 1 || (nq && (!qrows || !dQ)) ||
+      (nk && (!krows || !dK || !dV)))
+    return ORACLE_EBADARG;
+  for (int64_t a = 0; a < nq; ++a)
+    if (qrows[a] < 0 || qrows[a] >= N) return ORACLE_EBADARG;
+  for (int64_t a = 0; a < nk; ++a)
+    if (krows[a] < 0 || krows[a] >= N) return ORACLE_EBADARG;
+  double *Q = (double *)malloc(sizeof(double) * (size_t)(N * d));
+  double *K = (double *)malloc(sizeof(double) * (size_t)(N * d));
+  double *V = (double *)malloc(sizeof(double) * (size_t)(N * d));
+  double *dO = (double *)malloc(sizeof(double) * (size_t)(N * d));
+  double *lse = (double *)malloc(sizeof(double) * (size_t)N);
+  double *Dv = (double *)malloc(sizeof(double) * (size_t)N);
+  if (!Q || !K || !V || !dO || !lse || !Dv) {
+    free(Q); free(K); free(V); free(dO); free(lse); free(Dv);
+    return ORACLE_ENOMEM;
+  }
+  for (int64_t e = 0; e < N * d; ++e) {
+    Q[e] = bf16_bits_to_double(Qb[e]);
+    K[e] = bf16_bits_to_double(Kb[e]);
+    V[e] = bf16_bits_to_double(Vb[e]);
+    dO[e] = bf16_bits_to_double(dOb[e]);
+  }
+  int err = ORACLE_OK;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!s || !o) {
+#pragma omp atomic write
+      err = ORACLE_ENOMEM;
+    }
+    /* every row: lse_i and D_i (the forward of the head) */
+#pragma omp for schedule(dynamic, 8)
+    for (int64_t i = 0; i < N; ++i) {
+      if (!s || !o) continue;
+      const int64_t n = visible_keys(i, N, causal);
+      for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < d; ++t) acc += Q[i * d + t] * K[j * d + t];
+        s[j] = scale * acc;
+      }
+      attend_row(s, n, V, d, o, lse + i, NULL);
+      double Di = 0.0;
+      for (int64_t t = 0; t < d; ++t) Di += dO[i * d + t] * o[t];
+      Dv[i] = Di;
+    }
+    /* dQ for the sampled query rows */
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t a = 0; a < nq; ++a) {
+      if (!s || !o) continue;
+      const int64_t i = qrows[a];
+      const int64_t n = visible_keys(i, N, causal);
+      for (int64_t t = 0; t < d; ++t) dQ[a * d + t] = 0.0;
+      for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0, dp = 0.0;
+        for (int64_t t = 0; t < d; ++t) {
+          acc += Q[i * d + t] * K[j * d + t];
+          dp += dO[i * d + t] * V[j * d + t];
+        }
+        const double pij = exp(scale * acc - lse[i]);
+        const double dsij = pij * (dp - Dv[i]);
+        for (int64_t t = 0; t < d; ++t) dQ[a * d + t] += scale * dsij * K[j * d + t];
+      }
+    }
+    /* dK, dV for the sampled key rows: over every query that sees the key */
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t b = 0; b < nk; ++b) {
+      if (!s || !o) continue;
+      const int64_t j = krows[b];
+      for (int64_t t = 0; t < d; ++t) dK[b * d + t] = dV[b * d + t] = 0.0;
+      for (int64_t i = causal ? j : 0; i < N; ++i) {
+        double acc = 0.0, dp = 0.0;
+        for (int64_t t = 0; t < d; ++t) {
+          acc += Q[i * d + t] * K[j * d + t];
+          dp += dO[i * d + t] * V[j * d + t];
+        }
+        const double pij = exp(scale * acc - lse[i]);
+        const double dsij = pij * (dp - Dv[i]);
+        for (int64_t t = 0; t < d; ++t) {
+          dV[b * d + t] += pij * dO[i * d + t];
+          dK[b * d + t] += scale * dsij * Q[i * d + t];
+        }
+      }
+    }
+    free(s); free(o);
+  }
+  free(Q); free(K); free(V); free(dO); free(lse); free(Dv);
+  return err;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

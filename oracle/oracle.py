@@ -49,8 +49,12 @@ def _load():
         lib.oracle_attention_decode_rows_bf16.argtypes = [
             u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_int, ctypes.c_double,
             i64p, i64, dp, dp, ctypes.c_int]
+        lib.oracle_attention_backward_rows_bf16.argtypes = [
+            u16p, u16p, u16p, u16p, i64, i64, ctypes.c_int, ctypes.c_double,
+            i64p, i64, dp, i64p, i64, dp, dp, ctypes.c_int]
         for f in (lib.oracle_attention_decode_f64,
-                  lib.oracle_attention_decode_rows_bf16):
+                  lib.oracle_attention_decode_rows_bf16,
+                  lib.oracle_attention_backward_rows_bf16):
             f.restype = ctypes.c_int
         u8p = ctypes.POINTER(ctypes.c_uint8)
         i8p = ctypes.POINTER(ctypes.c_int8)
@@ -191,6 +195,31 @@ def attention_backward(q, k, v, do, causal: bool, scale: float, threads=None):
         _dptr(dv), B, H, N, d, int(bool(causal)), float(scale),
         _threads(threads)), "attention_backward")
     return dq, dk, dv
+
+
+def attention_backward_rows_bf16(qbits, kbits, vbits, dobits, causal: bool,
+                                 scale: float, qrows, krows, threads=None):
+    """Backward on sampled rows of one head of bf16 bit patterns [N, d]:
+    returns (dQ [len(qrows), d], dK [len(krows), d], dV [len(krows), d])."""
+    qbits, kbits, vbits, dobits = (np.ascontiguousarray(a, dtype=np.uint16)
+                                   for a in (qbits, kbits, vbits, dobits))
+    N, d = qbits.shape[-2], qbits.shape[-1]
+    if qbits.size != N * d:
+        raise ValueError("one head: arrays shaped [N, d]")
+    qrows = np.ascontiguousarray(qrows, dtype=np.int64)
+    krows = np.ascontiguousarray(krows, dtype=np.int64)
+    dQ = np.empty((qrows.size, d))
+    dK = np.empty((krows.size, d))
+    dV = np.empty((krows.size, d))
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    _check(_load().oracle_attention_backward_rows_bf16(
+        qbits.ctypes.data_as(u16p), kbits.ctypes.data_as(u16p),
+        vbits.ctypes.data_as(u16p), dobits.ctypes.data_as(u16p), N, d,
+        int(bool(causal)), float(scale), qrows.ctypes.data_as(i64p), qrows.size,
+        _dptr(dQ), krows.ctypes.data_as(i64p), krows.size, _dptr(dK), _dptr(dV),
+        _threads(threads)), "attention_backward_rows_bf16")
+    return dQ, dK, dV
 
 
 def attention_decode(q, k, v, causal: bool, scale: float, threads=None):

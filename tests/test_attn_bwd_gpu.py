@@ -124,3 +124,25 @@ def test_backward_argument_errors():
     assert attn.attn_bwd_raw(*args, ws.data_ptr(), ws.numel(), 1, 1, 64, 96, 0,
                              0.125, s) == 3
     assert attn.status() == 0
+
+
+@pytest.mark.parametrize("name", ["long_b1h32n16384d128", "b2h16n4096d128_causal"])
+def test_backward_full_size_sampled_rows(oracle_mod, name):
+    """The full-size configurations through the GPU forward and backward;
+    dQ of sampled query rows and dK, dV of sampled key rows of the first and
+    last head against the oracle (same tolerance as the shape sweep)."""
+    w = W.WORKLOADS[name]
+    q, k, v = W.make_qkv(w)
+    g = torch.Generator().manual_seed(w.seed + 99)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    dq, dk, dv = _run(w, q, k, v, do)
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, w.N - 1], rng.integers(0, w.N, 11)]))
+    BH = w.B * w.H
+    for bh in (0, BH - 1):
+        b, h = divmod(bh, w.H)
+        bits = [oracle_mod.bf16_bits(t[b, h].contiguous()) for t in (q, k, v, do)]
+        rq, rk, rv = oracle_mod.attention_backward_rows_bf16(*bits, w.causal, w.scale,
+                                                             rows, rows)
+        got = [dq[b, h][rows], dk[b, h][rows], dv[b, h][rows]]
+        _compare(got, [rq, rk, rv], f"{name} head {bh}")

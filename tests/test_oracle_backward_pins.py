@@ -111,3 +111,24 @@ def test_backward_rejects_bad_arguments(oracle_mod):
     with pytest.raises(RuntimeError):
         x = np.zeros((1, 1, 2, 0))
         oracle_mod.attention_backward(x, x, x, x, False, 1.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_rows_equal_the_full_backward(oracle_mod, causal):
+    """The sampled-row backward (for full-size checks) equals the full fp64
+    backward at those rows, on bf16 inputs of one head."""
+    import torch
+    g = torch.Generator().manual_seed(41)
+    N, d = 150, 16
+    q, k, v, do = (torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+                   for _ in range(4))
+    bits = [oracle_mod.bf16_bits(t) for t in (q, k, v, do)]
+    f = [oracle_mod.bf16_bits_to_f64(b) for b in bits]
+    dq, dk, dv = oracle_mod.attention_backward(*f, causal, 0.3)
+    qrows = np.array([0, 1, 77, 149])
+    krows = np.array([0, 5, 148, 149])
+    sq, sk, sv = oracle_mod.attention_backward_rows_bf16(
+        *(b.reshape(N, d) for b in bits), causal, 0.3, qrows, krows)
+    np.testing.assert_allclose(sq, dq[0, 0, qrows], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(sk, dk[0, 0, krows], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(sv, dv[0, 0, krows], rtol=1e-11, atol=1e-13)
