@@ -411,7 +411,7 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
   p.num_units = bh * ((N + 255) / 256);
   p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns.load();
-  p.debug_flags = g_inject.load();
+  p.debug_flags = g_inject.load() & 1u;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128)
@@ -795,6 +795,7 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
   p.causal = causal ? 1 : 0;
   p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns.load();
+  p.debug_flags = g_inject.load();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128)
     return Nq <= 4 ? launch_decode<128, 4>(*st, 0, p, s) : launch_decode<128, 16>(*st, 1, p, s);
@@ -939,7 +940,7 @@ void attn_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs);
 }
 
-void attn_set_fault_injection(uint32_t flags) { g_inject.store(flags & 1u); }
+void attn_set_fault_injection(uint32_t flags) { g_inject.store(flags & 3u); }
 
 }  // extern "C"
 
@@ -1053,7 +1054,7 @@ extern "C" int attn_fwd_host_noalloc(const void *q, const void *k,
   p.num_units = bh * ((N + 255) / 256);
   p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns.load();
-  p.debug_flags = g_inject.load();
+  p.debug_flags = g_inject.load() & 1u;
   if (d == 128)
     rc = causal ? launch<128, true>(*st, 0, maps, p, s)
                 : launch<128, false>(*st, 1, maps, p, s);

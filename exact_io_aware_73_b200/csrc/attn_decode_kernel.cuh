@@ -95,6 +95,7 @@ struct DecodeParams {
   int causal;
   float c_log2;        // scale * log2(e)
   unsigned long long timeout_ns;
+  uint32_t debug_flags;  // bit 1: CTA 0's producer skips its first tile
 };
 
 // All 256 compute threads meet at named barrier 1 (the producer warp never
@@ -145,6 +146,9 @@ __device__ __forceinline__ void dec_producer(uint32_t base, const DecodeParams &
   using L = DecSmem<D>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   int issued = 0;
+  // injected fault: the first tile's copies are never issued, so the compute
+  // warps' wait for it must run out (its stage is then not drained)
+  const int skipped = ((p.debug_flags & 2u) && blockIdx.x == 0) ? 0 : -1;
   for (int g = g0; g < g1; ++g) {
     const int h = g / p.ntiles;
     const int j = g - h * p.ntiles;
@@ -152,6 +156,10 @@ __device__ __forceinline__ void dec_producer(uint32_t base, const DecodeParams &
     if (!mbar_wait(bar(L::EMPTY + st), ((issued / L::kStages) & 1) ^ 1, wc,
                    kRoleProducer))
       break;
+    if (issued == skipped) {
+      ++issued;
+      continue;
+    }
     const int rows = min(kDecTileKeys, p.nk - j * kDecTileKeys);
     const uint32_t bytes = static_cast<uint32_t>(rows) * D * 2;
     mbar_arrive_expect_tx(bar(L::FULL + st), 2 * bytes);
@@ -165,6 +173,7 @@ __device__ __forceinline__ void dec_producer(uint32_t base, const DecodeParams &
     for (int st = 0; st < L::kStages; ++st)
       if (issued > st) {
         const int last = st + ((issued - 1 - st) / L::kStages) * L::kStages;
+        if (last == skipped) continue;  // nothing was copied for it
         mbar_wait_drain(bar(L::FULL + st), (last / L::kStages) & 1, wc);
       }
   }

@@ -394,11 +394,14 @@ const char *attn_strerror(int code);
 void attn_set_wait_timeout_ns(uint64_t ns);
 
 /*
- * attn_set_fault_injection -- test hook.  flags = 1: in later launches the
- * first CTA's loader never issues its first Q-tile copy, so the MMA warp's
- * wait on it runs out after the wait time limit and the launch ends with
- * ATTN_ERR_DEVICE_TIMEOUT in attn_status.  flags = 0 (the default) turns it
- * off.  No other value is defined.
+ * attn_set_fault_injection -- test hook.  Bit 0: in later attn_fwd launches
+ * the first CTA's loader never issues its first Q-tile copy, so the MMA
+ * warp's wait on it runs out after the wait time limit.  Bit 1: in later
+ * attn_decode launches the first CTA's producer never issues its first K/V
+ * tile, so the compute warps' wait runs out.  Either launch then ends with
+ * ATTN_ERR_DEVICE_TIMEOUT in attn_status (outputs invalid) and the CUDA
+ * context stays usable.  flags = 0 (the default) turns both off; other bits
+ * are ignored.
  */
 void attn_set_fault_injection(uint32_t flags);
 
