@@ -737,6 +737,11 @@ def run_seqpar(args, w):
     flops = w.flops()
     value = flops / (ms_per_step * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
+    cb = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_baseline(w, W.make_qkv(w), args.cpu_budget_s)
+        cb["sample"] = ("sharding does not change the result: the fp64 oracle "
+                        "on " + cb["sample"])
     if rank == 0:
         print(json.dumps({
             "metric": METRIC_SEQPAR, "value": value, "unit": "TFLOP/s",
@@ -756,7 +761,7 @@ def run_seqpar(args, w):
                          "frac": value / (peaks["bf16_tflops"] * world),
                          "peak_source": f"{peak_src} bf16 burst (cuBLAS) x ranks",
                          "traffic": None},
-            "cpu_baseline": None, "e2e": None,
+            "cpu_baseline": cb, "e2e": None,
             "gpu_launches": None, "clocks": clk}), flush=True)
     R.finish(world)
     return 0
