@@ -101,3 +101,29 @@ def test_merge_of_disjoint_key_sets(oracle_mod):
                                          f[2][:, :1, keep], False, 0.1)
     assert np.abs(o.float().cpu().numpy()[0, 0, 5] - O5[0, 0, 0]).max() <= O_TOL
     assert abs(float(lse[0, 0, 5]) - l5[0, 0, 0]) <= 1e-4
+
+
+@pytest.mark.parametrize("name,world", [("long_b1h32n16384d128", 4),
+                                        ("b2h16n4096d128_causal", 4)])
+def test_emulated_ring_full_size_sampled_rows(oracle_mod, name, world):
+    """Full-size configurations sharded over 4 emulated ranks; sampled rows
+    (both ends of every shard boundary included) against the oracle."""
+    w = W.WORKLOADS[name]
+    q, k, v = W.make_qkv(w)
+    outs, lses = seqpar.ring_attention_emulated(
+        *(seqpar.shard(t.cuda(), world) for t in (q, k, v)), w.causal, w.scale)
+    assert attn.status() == 0
+    o = torch.cat(outs, dim=2).float().cpu().numpy().reshape(-1, w.d)
+    lse = torch.cat(lses, dim=2).cpu().numpy().reshape(-1)
+    n = w.N // world
+    rows = set(W.sample_rows(w, 48))
+    for bh in (0, w.B * w.H - 1):
+        for r in range(world):
+            rows.update({bh * w.N + r * n, bh * w.N + r * n + n - 1})
+    rows = np.array(sorted(rows))
+    bits = [oracle_mod.bf16_bits(t) for t in (q, k, v)]
+    O_ref, l_ref = oracle_mod.attention_rows_bf16(*bits, w.causal, w.scale, rows)
+    eo = float(np.abs(o[rows] - O_ref).max())
+    el = float(np.abs(lse[rows] - l_ref).max())
+    assert eo <= O_TOL and el <= LSE_TOL, (eo, el)
+    print(name, "max|dO| %.2e max|dlse| %.2e" % (eo, el))
