@@ -459,3 +459,34 @@ def merge_finish(acc_o, acc_lse, stream=None):
                                         _stream_handle(stream))
     _check(rc, "attn_merge_finish")
     return o, lse
+
+
+# modes of attn_fwd_merge
+MERGE_FIRST, MERGE_INTO, MERGE_LAST = 1, 2, 3
+
+
+def attn_fwd_merge(q, k, v, acc_o, acc_lse, mode: int, causal: bool = False,
+                   scale: float | None = None, stream=None):
+    """attn_fwd folded into the fp32 accumulator (acc_o [B, H, N, d],
+    acc_lse [B, H, N]) in the kernel's epilogue.  mode MERGE_FIRST writes it,
+    MERGE_INTO merges into it, MERGE_LAST returns the merged (O bf16, lse)."""
+    import torch
+    L = lib()
+    f = L.attn_fwd_merge
+    if f.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        f.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, ctypes.c_float, i, vp]
+        f.restype = i
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    o = lse = None
+    if mode == MERGE_LAST:
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = f(q.data_ptr(), k.data_ptr(), v.data_ptr(), acc_o.data_ptr(),
+           acc_lse.data_ptr(), o.data_ptr() if o is not None else None,
+           lse.data_ptr() if lse is not None else None, B, H, N, d,
+           int(bool(causal)), float(scale), int(mode), _stream_handle(stream))
+    _check(rc, "attn_fwd_merge")
+    return (o, lse) if mode == MERGE_LAST else None

@@ -421,6 +421,65 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                 : launch<64, false>(*st, 3, maps, p, s);
 }
 
+int attn_fwd_merge(const void *q, const void *k, const void *v, float *acc_o,
+                   float *acc_lse, void *o, float *lse, int B, int H, int N, int d,
+                   int causal, float scale, int mode, attn_stream_t stream) {
+  if (mode != attn_b200::kMergeFirst && mode != attn_b200::kMergeInto &&
+      mode != attn_b200::kMergeLast)
+    return ATTN_ERR_INVALID_SIZE;
+  const bool last = mode == attn_b200::kMergeLast;
+  // the bf16 outputs are checked as attn_fwd's when they are written; the
+  // accumulator takes their place otherwise (same alignment rules)
+  int rc = check_args(q, k, v, last ? o : static_cast<void *>(acc_o),
+                      last ? lse : acc_lse, B, H, N, d, scale, true);
+  if (rc != ATTN_OK || B == 0 || H == 0 || N == 0) return rc;
+  if (!acc_o || !acc_lse) return ATTN_ERR_NULL_POINTER;
+  if (!aligned(acc_o, 16) || !aligned(acc_lse, 4)) return ATTN_ERR_MISALIGNED;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  const size_t tb = rows * d * 2, ab = rows * d * 4, lb = rows * 4;
+  const void *ins[3] = {q, k, v};
+  for (const void *in : ins)
+    if (overlaps(acc_o, ab, in, tb) || overlaps(acc_lse, lb, in, tb)) return ATTN_ERR_ALIAS;
+  if (overlaps(acc_o, ab, acc_lse, lb)) return ATTN_ERR_ALIAS;
+  if (last && (overlaps(o, tb, acc_o, ab) || overlaps(o, tb, acc_lse, lb) ||
+               overlaps(lse, lb, acc_o, ab) || overlaps(lse, lb, acc_lse, lb)))
+    return ATTN_ERR_ALIAS;
+  int dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  const void *all[5] = {q, k, v, acc_o, acc_lse};
+  for (const void *ptr : all)
+    if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
+  if (last && (!is_device_memory_of(o, dev) || !is_device_memory_of(lse, dev)))
+    return ATTN_ERR_NOT_DEVICE_MEMORY;
+  EncodeTiledFn enc;
+  if ((rc = get_encode_fn(&enc)) != ATTN_OK) return rc;
+  const int bh = B * H;
+  CUtensorMap maps[3];
+  if ((rc = encode_map(enc, &maps[0], q, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[1], k, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[2], v, bh, N, d)) != ATTN_OK) return rc;
+  FwdParams p;
+  p.o = last ? static_cast<uint16_t *>(o) : nullptr;
+  p.lse = last ? lse : nullptr;
+  p.acc_o = acc_o;
+  p.acc_lse = acc_lse;
+  p.merge_mode = mode;
+  p.status = st->status;
+  p.bh = bh;
+  p.n = N;
+  p.num_units = bh * ((N + 255) / 256);
+  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.timeout_ns = g_timeout_ns.load();
+  p.debug_flags = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch<128, true>(*st, 0, maps, p, s)
+                  : launch<128, false>(*st, 1, maps, p, s);
+  return causal ? launch<64, true>(*st, 2, maps, p, s)
+                : launch<64, false>(*st, 3, maps, p, s);
+}
+
 size_t attn_fwd_host_workspace_bytes(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128)) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;

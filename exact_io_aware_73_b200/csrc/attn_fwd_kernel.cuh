@@ -153,7 +153,16 @@ struct FwdParams {
   const float *k_scale;  // [BH, tiles] one per 128-row K tile
   const float *v_scale;  // [BH] one per head
   int tiles;             // ceil(n / 128)
+  // Merge into an accumulator of partial results (attention over disjoint
+  // key sets, combined exactly through the log-sum-exp).  kMergeNone: write
+  // O (bf16) and lse.  First: write this result to acc_o (fp32 [BH, N, D])
+  // and acc_lse.  Into: acc <- merge(acc, this).  Last: O, lse <-
+  // merge(acc, this), in bf16 / fp32.
+  float *acc_o = nullptr;
+  float *acc_lse = nullptr;
+  int merge_mode = 0;
 };
+constexpr int kMergeNone = 0, kMergeFirst = 1, kMergeInto = 2, kMergeLast = 3;
 
 // Pairs of FP8 exponentials (out of 8) evaluated on the FMA pipe.
 #ifndef ATTN_EXP2_EMU_PER8_FP8
@@ -738,31 +747,87 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     tc_fence_after_sync();
     const float inv_l = __frcp_rn(l_run) * v_mul;
     const bool row_ok = qs + r < p.n;
-    uint4 *orow = reinterpret_cast<uint4 *>(
-        p.o + (static_cast<int64_t>(w.bh) * p.n + qs + r) * D);
+    const int64_t grow = static_cast<int64_t>(w.bh) * p.n + qs + r;
+    // this block's log-sum-exp (natural log)
+    const float lse_this = (m_run - (FP8 ? 8.f : 0.f) + lg2_approx(l_run)) * kLn2;
+    float lse_out = lse_this;
+    if (p.merge_mode == kMergeNone) {
+      uint4 *orow = reinterpret_cast<uint4 *>(p.o + grow * D);
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      tmem_ld_32x32b_x32(tO + c * 32, o);
-      tmem_wait_ld(o);
-      uint32_t h[16];
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + c * 32, o);
+        tmem_wait_ld(o);
+        uint32_t h[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
-                           __uint_as_float(o[2 * i + 1]) * inv_l);
-      if (row_ok) {
+        for (int i = 0; i < 16; ++i)
+          h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                             __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (row_ok) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          orow[c * 4 + i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2],
-                                       h[4 * i + 3]);
+          for (int i = 0; i < 4; ++i)
+            orow[c * 4 + i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2],
+                                         h[4 * i + 3]);
+        }
+      }
+    } else {
+      // weights of the accumulator and of this block: exp(lse_x - lse_new)
+      float wa = 0.f, wp = 1.f;
+      if (p.merge_mode != kMergeFirst && row_ok) {
+        const float la = p.acc_lse[grow];
+        const float mx = fmaxf(la, lse_this);
+        wa = (la == -CUDART_INF_F) ? 0.f : ex2_approx((la - mx) * 1.4426950408889634f);
+        wp = ex2_approx((lse_this - mx) * 1.4426950408889634f);
+        const float tot = wa + wp;
+        lse_out = mx + lg2_approx(tot) * kLn2;
+        const float it = __frcp_rn(tot);
+        wa *= it;
+        wp *= it;
+      }
+      float4 *arow = reinterpret_cast<float4 *>(p.acc_o + grow * D);
+      uint4 *orow = reinterpret_cast<uint4 *>(p.o + grow * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + c * 32, o);
+        tmem_wait_ld(o);
+        if (!row_ok) continue;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o[i]) * inv_l * wp;
+        if (p.merge_mode != kMergeFirst) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 a4 = arow[c * 8 + i];
+            v[4 * i] = fmaf(wa, a4.x, v[4 * i]);
+            v[4 * i + 1] = fmaf(wa, a4.y, v[4 * i + 1]);
+            v[4 * i + 2] = fmaf(wa, a4.z, v[4 * i + 2]);
+            v[4 * i + 3] = fmaf(wa, a4.w, v[4 * i + 3]);
+          }
+        }
+        if (p.merge_mode == kMergeLast) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            orow[c * 4 + i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]),
+                                         pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                         pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
+                                         pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            arow[c * 8 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
       }
     }
     tc_fence_before_sync();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar(L::O_EMPTY + t));  // O columns reusable
-    if (row_ok)
-      p.lse[static_cast<int64_t>(w.bh) * p.n + qs + r] =
-          (m_run - (FP8 ? 8.f : 0.f) + lg2_approx(l_run)) * kLn2;
+    if (row_ok) {
+      if (p.merge_mode == kMergeFirst || p.merge_mode == kMergeInto)
+        p.acc_lse[grow] = lse_out;
+      else
+        p.lse[grow] = lse_out;
+    }
   }
 }
 

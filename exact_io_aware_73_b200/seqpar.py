@@ -11,14 +11,16 @@ around the ring (rank r sends to r + 1 and receives from r - 1) while each
 rank attends its queries to the shard it holds with the single-GPU kernel
 (non-causal for an earlier shard, causal for its own, skipped for a later
 one under the causal mask) and folds the partial (O, lse) into an fp32
-accumulator:  lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s.
+accumulator:  lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s --
+inside the kernel's epilogue (attn_fwd_merge: the first block writes the
+accumulator, later ones merge into it, the last writes the bf16 result).
 The result is exact attention for the rank's queries.  The exchange of the
 next shard is started before the current step's compute, so the transfer
 overlaps it.
 
 Everything here is orchestration: every arithmetic step runs in the CUDA
-library (attn_fwd for a block, attn_merge_fold / attn_merge_finish for the
-merge) through ``GpuOps``; tests may pass other ops with the same methods.
+library (attn_fwd_merge, or attn_fwd for a rank with one block) through
+``GpuOps``; tests may pass other ops with the same method.
 """
 from __future__ import annotations
 
@@ -43,26 +45,28 @@ def shard_plan(rank: int, world: int, causal: bool):
 
 
 class GpuOps:
-    """The CUDA library's block attention and merge (no fallback)."""
+    """The CUDA library's block attention with the fold in its epilogue (no
+    fallback)."""
 
     def __init__(self):
         from . import attn
         self.attn = attn
 
-    def attend(self, q, k, v, causal: bool, scale: float):
-        return self.attn.attn_fwd(q, k, v, causal=causal, scale=scale)
-
-    def new_acc(self, q):
+    def block(self, q, k, v, causal: bool, scale: float, state: dict, i: int,
+              n: int):
+        """Block i of the n blocks this rank attends; returns (O, lse) after
+        the last (i = n - 1), None before."""
         import torch
-        B, H, n, d = q.shape
-        return (torch.empty((B, H, n, d), dtype=torch.float32, device=q.device),
-                torch.empty((B, H, n), dtype=torch.float32, device=q.device))
-
-    def fold(self, acc, part, first: bool):
-        self.attn.merge_fold(acc[0], acc[1], part[0], part[1], first)
-
-    def finish(self, acc):
-        return self.attn.merge_finish(acc[0], acc[1])
+        if n == 1:
+            return self.attn.attn_fwd(q, k, v, causal=causal, scale=scale)
+        if i == 0:
+            B, H, m, d = q.shape
+            state["o"] = torch.empty((B, H, m, d), dtype=torch.float32, device=q.device)
+            state["lse"] = torch.empty((B, H, m), dtype=torch.float32, device=q.device)
+        mode = (self.attn.MERGE_FIRST if i == 0 else
+                self.attn.MERGE_LAST if i == n - 1 else self.attn.MERGE_INTO)
+        return self.attn.attn_fwd_merge(q, k, v, state["o"], state["lse"], mode,
+                                        causal=causal, scale=scale)
 
 
 @dataclass
@@ -86,11 +90,10 @@ def ring_attention(q, k, v, causal: bool, scale: float, group=None, ops=None,
     world = dist.get_world_size(group) if (group is not None or dist.is_initialized()) else 1
     rank = dist.get_rank(group) if world > 1 else 0
     plan = shard_plan(rank, world, causal)
-    single = sum(how is not None for _, how in plan) == 1
+    nblocks = sum(how is not None for _, how in plan)
     kv = torch.stack([k, v]).contiguous()
     nxt = torch.empty_like(kv) if world > 1 else None
-    acc = None if single else ops.new_acc(q)
-    first = True
+    state, done = {}, 0
     for t, (s, how) in enumerate(plan):
         reqs = []
         if world > 1 and t + 1 < world:
@@ -103,12 +106,11 @@ def ring_attention(q, k, v, causal: bool, scale: float, group=None, ops=None,
             if stats is not None:
                 stats.bytes_sent += kv.numel() * kv.element_size()
         if how is not None:
-            part = ops.attend(q, kv[0], kv[1], how == "causal", scale)
-            if single:
-                result = part  # one block: folding it would reproduce its bits
-            else:
-                ops.fold(acc, part, first)
-            first = False
+            out = ops.block(q, kv[0], kv[1], how == "causal", scale, state, done,
+                            nblocks)
+            done += 1
+            if done == nblocks:
+                result = out
             if stats is not None:
                 stats.blocks += 1
         elif stats is not None:
@@ -119,7 +121,7 @@ def ring_attention(q, k, v, causal: bool, scale: float, group=None, ops=None,
             kv, nxt = nxt, kv
         if stats is not None:
             stats.steps += 1
-    return result if single else ops.finish(acc)
+    return result
 
 
 def shard(x, world: int):
@@ -143,9 +145,8 @@ def ring_attention_emulated(qs, ks, vs, causal: bool, scale: float, ops=None,
     outs, lses = [], []
     for r in range(world):
         plan = shard_plan(r, world, causal)
-        single = sum(how is not None for _, how in plan) == 1
-        acc = None if single else ops.new_acc(qs[r])
-        first, result = True, None
+        nblocks = sum(how is not None for _, how in plan)
+        state, done, result = {}, 0, None
         for s, how in plan:
             if stats is not None:
                 stats.steps += 1
@@ -153,15 +154,13 @@ def ring_attention_emulated(qs, ks, vs, causal: bool, scale: float, ops=None,
                 if stats is not None:
                     stats.skipped += 1
                 continue
-            part = ops.attend(qs[r], ks[s], vs[s], how == "causal", scale)
-            if single:
-                result = part
-            else:
-                ops.fold(acc, part, first)
-            first = False
+            out = ops.block(qs[r], ks[s], vs[s], how == "causal", scale, state,
+                            done, nblocks)
+            done += 1
+            if done == nblocks:
+                result = out
             if stats is not None:
                 stats.blocks += 1
-        o, lse = result if single else ops.finish(acc)
-        outs.append(o)
-        lses.append(lse)
+        outs.append(result[0])
+        lses.append(result[1])
     return outs, lses

@@ -375,6 +375,22 @@ void attn_set_decode_max_ctas(int n);
  * aligned, the lse arrays 4-byte aligned, device memory of the current
  * device, outputs not overlapping inputs.  Queued on `stream`.
  */
+/*
+ * attn_fwd_merge -- attn_fwd with its result folded into an accumulator in
+ * the kernel's epilogue (no separate merge pass, no bf16 rounding of parts):
+ *   mode 1 (first): acc_o = O of this call (fp32), acc_lse = its lse;
+ *   mode 2 (into):  (acc_o, acc_lse) = merge(accumulator, this call);
+ *   mode 3 (last):  o (bf16), lse = merge(accumulator, this call); the
+ *                   accumulator is only read.
+ * acc_o fp32 [B, H, N, d] (16-byte aligned), acc_lse fp32 [B, H, N]; o and
+ * lse as attn_fwd's, used by mode 3 only (may be NULL otherwise).  Every
+ * call of a sequence of folds must cover the same queries (q is the same
+ * shape; k, v are another disjoint part of the keys, same length N).
+ */
+int attn_fwd_merge(const void *q, const void *k, const void *v, float *acc_o,
+                   float *acc_lse, void *o, float *lse, int B, int H, int N, int d,
+                   int causal, float scale, int mode, attn_stream_t stream);
+
 int attn_merge_fold(float *acc_o, float *acc_lse, const void *part_o,
                     const float *part_lse, int64_t rows, int d, int first,
                     attn_stream_t stream);

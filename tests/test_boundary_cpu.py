@@ -211,3 +211,18 @@ def test_merge_entries_refuse_bad_arguments_without_a_device(attn):
     assert L.attn_merge_fold(None, None, None, None, 0, 128, 1, None) == 0
     assert L.attn_merge_finish(far, 2 * far, 3 * far, 4 * far, 10, 100, None) == 3
     assert L.attn_merge_finish(far, 2 * far, far + 16, 4 * far, 10, 64, None) == 6
+
+
+def test_fwd_merge_refuses_bad_modes_without_a_device(attn):
+    far = 1 << 40
+    f = attn.lib().attn_fwd_merge
+    import ctypes
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, ctypes.c_float, i, vp]
+    f.restype = i
+    args = [far, 2 * far, 3 * far, 4 * far, 5 * far, 6 * far, 7 * far, 1, 1, 64, 64, 0, 0.1]
+    assert f(*args, 0, None) == 2              # no such mode
+    assert f(*args, 4, None) == 2
+    assert f(*(args[:3] + [None] + args[4:]), 2, None) == 1   # accumulator missing
+    assert f(*(args[:3] + [4 * far + 8] + args[4:]), 2, None) == 4
+    assert f(*(args[:3] + [far + 64] + args[4:]), 2, None) == 6  # acc over q

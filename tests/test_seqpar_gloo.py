@@ -29,35 +29,26 @@ def _free_port():
 
 
 class _CpuOps:
+    """fp64 stand-ins: the oracle for a block, the log-sum-exp merge in
+    torch (the same fold the kernel's epilogue performs)."""
+
     def __init__(self, oracle):
         self.oracle = oracle
 
-    def attend(self, q, k, v, causal, scale):
+    def block(self, q, k, v, causal, scale, state, i, n):
         import torch
         O, lse = self.oracle.attention(q.double().numpy(), k.double().numpy(),
                                        v.double().numpy(), causal, scale, threads=1)
-        return torch.from_numpy(O), torch.from_numpy(lse)
-
-    def new_acc(self, q):
-        import torch
-        B, H, n, d = q.shape
-        return [torch.zeros(B, H, n, d, dtype=torch.float64),
-                torch.full((B, H, n), float("-inf"), dtype=torch.float64)]
-
-    def fold(self, acc, part, first):
-        import torch
-        o, lse = part
-        if first:
-            acc[0], acc[1] = o.clone(), lse.clone()
-            return
-        m = torch.maximum(acc[1], lse)
-        wa, wp = torch.exp(acc[1] - m), torch.exp(lse - m)
-        t = wa + wp
-        acc[0] = (wa / t)[..., None] * acc[0] + (wp / t)[..., None] * o
-        acc[1] = m + torch.log(t)
-
-    def finish(self, acc):
-        return acc[0], acc[1]
+        O, lse = torch.from_numpy(O), torch.from_numpy(lse)
+        if i == 0:
+            state["o"], state["lse"] = O, lse
+        else:
+            m = torch.maximum(state["lse"], lse)
+            wa, wp = torch.exp(state["lse"] - m), torch.exp(lse - m)
+            t = wa + wp
+            state["o"] = (wa / t)[..., None] * state["o"] + (wp / t)[..., None] * O
+            state["lse"] = m + torch.log(t)
+        return (state["o"], state["lse"]) if i == n - 1 else None
 
 
 def _worker(rank, world, port, causal, out_dir):

@@ -127,3 +127,29 @@ def test_emulated_ring_full_size_sampled_rows(oracle_mod, name, world):
     el = float(np.abs(lse[rows] - l_ref).max())
     assert eo <= O_TOL and el <= LSE_TOL, (eo, el)
     print(name, "max|dO| %.2e max|dlse| %.2e" % (eo, el))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fwd_merge_modes_fold_in_the_epilogue(oracle_mod, d):
+    """attn_fwd_merge over three key blocks (first, into, last) equals
+    attention over all their keys; only the final output is rounded to bf16,
+    so the bound is that of a plain forward."""
+    g = torch.Generator().manual_seed(8 + d)
+    B, H, n = 2, 2, 700
+    q = torch.randn(B, H, n, d, generator=g).to(torch.bfloat16)
+    ks = [torch.randn(B, H, n, d, generator=g).to(torch.bfloat16) for _ in range(3)]
+    vs = [torch.randn(B, H, n, d, generator=g).to(torch.bfloat16) for _ in range(3)]
+    acc_o = torch.empty(B, H, n, d, dtype=torch.float32, device="cuda")
+    acc_l = torch.empty(B, H, n, dtype=torch.float32, device="cuda")
+    modes = [attn.MERGE_FIRST, attn.MERGE_INTO, attn.MERGE_LAST]
+    for kb, vb, mode in zip(ks, vs, modes):
+        out = attn.attn_fwd_merge(q.cuda(), kb.cuda(), vb.cuda(), acc_o, acc_l, mode,
+                                  causal=False, scale=0.09)
+    o, lse = out
+    assert attn.status() == 0
+    f = [oracle_mod.bf16_bits_to_f64(oracle_mod.bf16_bits(t))
+         for t in (q, torch.cat(ks, dim=2), torch.cat(vs, dim=2))]
+    O_ref, l_ref = oracle_mod.attention_decode(*f, False, 0.09)
+    err = np.abs(o.float().cpu().numpy() - O_ref)
+    assert np.all(err <= 2.0 ** -8 * np.abs(O_ref) + 2e-3), err.max()
+    assert np.abs(lse.cpu().numpy() - l_ref).max() <= 1e-4
