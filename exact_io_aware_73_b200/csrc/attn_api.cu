@@ -328,10 +328,9 @@ int launch_decode(DeviceState &st, int variant, attn_b200::DecodeParams &p,
       st.dec_attr_set[variant] = true;
     }
   }
-  // stream-K: an equal share of the key tiles per CTA, two CTAs per SM (one
-  // for the 16-query variant, whose registers allow one)
+  // stream-K: an equal share of the key tiles per CTA, two CTAs per SM
   int ctas = g_decode_max_ctas.load();
-  if (ctas <= 0) ctas = (QMAX <= 4 ? 2 : 1) * st.sm_count;
+  if (ctas <= 0) ctas = 2 * st.sm_count;
   if (ctas > attn_b200::kDecMaxCtas) ctas = attn_b200::kDecMaxCtas;
   const int grid0 = p.total < ctas ? p.total : ctas;
   p.per_cta = (p.total + grid0 - 1) / grid0;
@@ -788,9 +787,12 @@ size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
   if (B < 0 || H < 0 || Nq < 0 || Nq > ATTN_DECODE_MAX_Q || Nk < 0 ||
       (d != 64 && d != 128))
     return 0;
+  // launches serve at most 4 queries per head each and run one after another
+  // on the stream, so they share the partial slots
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t slots = bh + attn_b200::kDecMaxCtas;
-  return round256(slots * Nq * d * 4) + round256(slots * Nq * 4) + round256(bh * 4);
+  const size_t g = Nq < 4 ? static_cast<size_t>(Nq) : 4;
+  return round256(slots * g * d * 4) + round256(slots * g * 4) + round256(bh * 4);
 }
 
 int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -833,32 +835,43 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
   for (const void *ptr : all)
     if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
   const size_t slots = static_cast<size_t>(bh64) + attn_b200::kDecMaxCtas;
+  const size_t g = Nq < 4 ? static_cast<size_t>(Nq) : 4;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  attn_b200::DecodeParams p;
-  p.q = static_cast<const uint16_t *>(q);
-  p.k = static_cast<const uint16_t *>(k);
-  p.v = static_cast<const uint16_t *>(v);
-  p.o = static_cast<uint16_t *>(o);
-  p.lse = lse;
-  p.part_o = reinterpret_cast<float *>(ws);
-  p.part_lse = reinterpret_cast<float *>(ws + round256(slots * Nq * d * 4));
-  p.counters = reinterpret_cast<int *>(ws + round256(slots * Nq * d * 4) +
-                                       round256(slots * Nq * 4));
-  p.status = st->status;
-  p.bh = static_cast<int>(bh64);
-  p.nq = Nq;
-  p.nk = Nk;
-  p.ntiles = static_cast<int>(ntiles);
-  p.total = static_cast<int>(bh64 * ntiles);
-  p.per_cta = 1;
-  p.causal = causal ? 1 : 0;
-  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  p.timeout_ns = g_timeout_ns.load();
-  p.debug_flags = g_inject.load();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return Nq <= 4 ? launch_decode<128, 4>(*st, 0, p, s) : launch_decode<128, 16>(*st, 1, p, s);
-  return Nq <= 4 ? launch_decode<64, 4>(*st, 2, p, s) : launch_decode<64, 16>(*st, 3, p, s);
+  // groups of up to 4 queries, one launch each; under the causal mask a
+  // group's last query sees keys 0 .. Nk - Nq + q0 + m - 1, so its launch
+  // stops there (same visibility rule with Nk' = that count, Nq' = m)
+  for (int q0 = 0; q0 < Nq; q0 += 4) {
+    const int m = (Nq - q0 < 4) ? (Nq - q0) : 4;
+    const int nk = causal ? Nk - Nq + q0 + m : Nk;
+    const int64_t ntiles = (nk + attn_b200::kDecTileKeys - 1) / attn_b200::kDecTileKeys;
+    attn_b200::DecodeParams p;
+    p.q = static_cast<const uint16_t *>(q) + static_cast<int64_t>(q0) * d;
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.o = static_cast<uint16_t *>(o) + static_cast<int64_t>(q0) * d;
+    p.lse = lse + q0;
+    p.part_o = reinterpret_cast<float *>(ws);
+    p.part_lse = reinterpret_cast<float *>(ws + round256(slots * g * d * 4));
+    p.counters = reinterpret_cast<int *>(ws + round256(slots * g * d * 4) +
+                                         round256(slots * g * 4));
+    p.status = st->status;
+    p.bh = static_cast<int>(bh64);
+    p.nq = m;
+    p.nk = nk;
+    p.qstride = Nq;
+    p.kstride = Nk;
+    p.ntiles = static_cast<int>(ntiles);
+    p.total = static_cast<int>(bh64 * ntiles);
+    p.per_cta = 1;
+    p.causal = causal ? 1 : 0;
+    p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.timeout_ns = g_timeout_ns.load();
+    p.debug_flags = q0 == 0 ? g_inject.load() : 0u;
+    rc = d == 128 ? launch_decode<128, 4>(*st, 0, p, s) : launch_decode<64, 4>(*st, 2, p, s);
+    if (rc != ATTN_OK) return rc;
+  }
+  return ATTN_OK;
 }
 
 void attn_set_decode_max_ctas(int n) { g_decode_max_ctas.store(n > 0 ? n : 0); }

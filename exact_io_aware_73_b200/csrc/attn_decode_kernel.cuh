@@ -8,7 +8,10 @@
 //
 // Decode is a matrix-vector product per (batch, head): every key and value
 // byte is used for a handful of queries, so the bound is HBM bandwidth, not
-// the tensor cores.  The kernel therefore streams K/V through shared memory
+// the tensor cores.  One launch serves up to 4 queries per head (their
+// state stays in registers with two CTAs per SM); more queries are served in
+// groups of 4 by successive launches, each stopping at the last key its
+// queries can see.  The kernel therefore streams K/V through shared memory
 // with bulk asynchronous copies and does the arithmetic on the CUDA cores:
 //   * stream-K split: the B*H*ceil(Nk/64) key tiles of all heads are one
 //     sequence; CTA c takes tiles [c T, (c+1) T) -- an equal share, which may
@@ -89,6 +92,8 @@ struct DecodeParams {
   int *counters;       // [BH] parts finished per head (zero at launch)
   uint32_t *status;
   int bh, nq, nk;
+  int qstride;         // rows per head of q, o, lse (nq unless a group of them)
+  int kstride;         // rows per head of k, v (nk unless the keys are cut short)
   int ntiles;          // key tiles per head
   int total;           // bh * ntiles
   int per_cta;         // T: tiles per CTA
@@ -163,7 +168,7 @@ __device__ __forceinline__ void dec_producer(uint32_t base, const DecodeParams &
     const int rows = min(kDecTileKeys, p.nk - j * kDecTileKeys);
     const uint32_t bytes = static_cast<uint32_t>(rows) * D * 2;
     mbar_arrive_expect_tx(bar(L::FULL + st), 2 * bytes);
-    const int64_t off = (static_cast<int64_t>(h) * p.nk + j * kDecTileKeys) * D;
+    const int64_t off = (static_cast<int64_t>(h) * p.kstride + j * kDecTileKeys) * D;
     bulk_g2s(base + L::kK + st * L::kTileBytes, p.k + off, bytes, bar(L::FULL + st));
     bulk_g2s(base + L::kV + st * L::kTileBytes, p.v + off, bytes, bar(L::FULL + st));
     ++issued;
@@ -206,7 +211,7 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
     const int h = g / p.ntiles;
     const int gend = min(g1, (h + 1) * p.ntiles);
     dec_bar();  // the previous part's readers of the shared region are done
-    const uint16_t *qsrc = p.q + static_cast<int64_t>(h) * p.nq * D;
+    const uint16_t *qsrc = p.q + static_cast<int64_t>(h) * p.qstride * D;
     for (int i = tid; i < p.nq * D; i += kDecComputeThreads)
       qf[i] = __uint_as_float(static_cast<uint32_t>(qsrc[i]) << 16) * p.c_log2;
     dec_bar();
@@ -332,7 +337,7 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
     const int first = dec_first_cta(h, p), last = dec_last_cta(h, p);
     const bool whole = first == last;
     const int slot = h + static_cast<int>(blockIdx.x);
-    const int64_t row0 = static_cast<int64_t>(h) * p.nq;
+    const int64_t row0 = static_cast<int64_t>(h) * p.qstride;
     for (int q0 = 0; q0 < p.nq; q0 += L::kRedQ) {
       dec_bar();  // earlier readers of the shared region are done
 #pragma unroll

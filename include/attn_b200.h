@@ -338,8 +338,11 @@ size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
  *
  * The key tiles of all heads are split into equal contiguous shares, one per
  * CTA (two CTAs per SM); a head split over several CTAs is combined exactly
- * by the CTA that finishes its last share.  Queued on `stream`; a wait that
- * runs out of time shows in attn_status (outputs are then invalid).
+ * by the CTA that finishes its last share.  One launch serves up to 4
+ * queries per head; more are served in groups of 4 by successive launches
+ * (each reads K/V again, up to the last key its group sees).  Queued on
+ * `stream`; a wait that runs out of time shows in attn_status (outputs are
+ * then invalid).
  */
 #define ATTN_DECODE_MAX_Q 16
 #define ATTN_MAX_DECODE_KEYS (1 << 26)
@@ -348,8 +351,8 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
                 void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /* Workspace bytes attn_decode needs (0 on bad sizes): partial outputs and
- * log-sum-exps for B*H + 1024 parts, and B*H counters, each rounded up to
- * 256 bytes. */
+ * log-sum-exps of min(Nq, 4) queries for B*H + 1024 parts, and B*H
+ * counters, each rounded up to 256 bytes. */
 size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d);
 
 /* Test hook: cap the number of CTAs attn_decode launches (0 = two per SM),

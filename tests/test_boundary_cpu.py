@@ -198,6 +198,11 @@ def test_decode_entry_refuses_bad_arguments_without_a_device(attn):
     slots = B * H + 1024
     assert attn.decode_workspace_bytes(B, H, Nq, 1000, d) == \
         r(slots * Nq * d * 4) + r(slots * Nq * 4) + r(B * H * 4)
+    # queries beyond 4 run as further groups of 4 that reuse the same slots
+    assert attn.decode_workspace_bytes(B, H, 16, 1000, d) == \
+        attn.decode_workspace_bytes(B, H, 4, 1000, d)
+    assert attn.decode_workspace_bytes(B, H, 3, 1000, d) == \
+        r(slots * 3 * d * 4) + r(slots * 3 * 4) + r(B * H * 4)
 
 
 def test_merge_entries_refuse_bad_arguments_without_a_device(attn):
