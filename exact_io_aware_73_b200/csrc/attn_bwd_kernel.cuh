@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       int uocc = 0, kv_issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
         int bh, qt, nkv;
         dq_unit<CAUSAL>(u, p.bh, p.tiles, bh, qt, nkv);
         if (uocc > 0) {
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // and dP_{j+1} run during the next P phase.
       int uocc = 0, kv_cons = 0, jcnt = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
         int bh, qt, nkv;
         dq_unit<CAUSAL>(u, p.bh, p.tiles, bh, qt, nkv);
         ok = mbar_wait_spin(bar(L::Q_FULL), uocc & 1, wc, kRoleMma);
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lb = static_cast<uint32_t>(wq * 32) << 16;
     int s_cnt = 0, uocc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+    for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
       int bh, qt, nkv;
       dq_unit<CAUSAL>(u, p.bh, p.tiles, bh, qt, nkv);
       const int row = qt * kBlockM + r;  // < npad: padded vectors in range
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       int uocc = 0, q_issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
         int bh, kt, q0;
         dkv_unit<CAUSAL>(u, p.bh, p.tiles, bh, kt, q0);
         if (uocc > 0) {
@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // dP^T is issued after the one reading P^T or dS^T from those columns.
       int uocc = 0, q_cons = 0, tcnt = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
         int bh, kt, q0;
         dkv_unit<CAUSAL>(u, p.bh, p.tiles, bh, kt, q0);
         ok = mbar_wait_spin(bar(L::KV_FULL), uocc & 1, wc, kRoleMma);
@@ -585,7 +585,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lb = static_cast<uint32_t>(wq * 32) << 16;
     int s_cnt = 0, uocc = 0, q_cons = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+    for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
       int bh, kt, q0;
       dkv_unit<CAUSAL>(u, p.bh, p.tiles, bh, kt, q0);
       for (int i = q0; i < p.tiles; ++i) {

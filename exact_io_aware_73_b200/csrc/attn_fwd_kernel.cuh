@@ -231,6 +231,18 @@ __device__ __forceinline__ Unit decode_unit(int u, int bh_count, int n) {
   return w;
 }
 
+// The k-th unit a persistent CTA takes: round-robin over the CTAs, reversed
+// in every other round under the causal mask.  Causal units are numbered
+// heaviest first, so the reversal (a snake order) gives the CTA that took
+// one of the heaviest units of a round one of the lightest of the next; the
+// work per CTA then stays within about one unit of the mean, where plain
+// round-robin leaves the first CTAs up to a third above it.
+template <bool CAUSAL>
+__device__ __forceinline__ int unit_at(int k) {
+  const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return k * g + ((CAUSAL && (k & 1)) ? g - 1 - c : c);
+}
+
 struct WaitCtx {
   volatile int *abort;
   uint32_t *status;
@@ -326,7 +338,7 @@ __device__ __forceinline__ void producer_role(uint32_t base,
   const uint64_t pol_kv = policy_evict_last();
   const uint64_t pol_q = policy_evict_first();
 
-  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+  for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
     const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
     const int nt[2] = {w.n0, w.n1};
     for (int t = 0; MODE != kLoadV && t < 2; ++t) {
@@ -459,7 +471,7 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
   int kcons = 0, vcons = 0;
   bool ok = true;
 
-  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+  for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
     const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
     const int nt[2] = {w.n0, w.n1};
     const int nmax = max(nt[0], nt[1]);
@@ -666,7 +678,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
   int scnt = 0, ocnt = 0;
   bool ok = true;
 
-  for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+  for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
     const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
     const int n = t ? w.n1 : w.n0;
     if (n == 0) continue;
