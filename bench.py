@@ -48,6 +48,7 @@ CSRC = os.path.join(ROOT, "exact_io_aware_73_b200", "csrc")
 
 KERNEL_SOURCES = ("attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 DECODE_SOURCES = ("attn_decode_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
+BWD_SOURCES = ("attn_bwd_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 
 
 def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
@@ -323,10 +324,11 @@ def run_backward(args, w):
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
-                         "traffic": None,
+                         "traffic": load_traffic(w.name, "traffic_bwd_", BWD_SOURCES),
                          "note": "FLOPs = 2.5 x forward (5 GEMMs); the kernels "
                                  "run 7 (S and dP are recomputed in both the "
-                                 "dQ and the dK/dV kernel)"},
+                                 "dQ and the dK/dV kernel); traffic is the "
+                                 "dK/dV kernel's (the larger share), per launch"},
             "cpu_baseline": cb, "e2e": None,
             "gpu_launches": 3 * args.steps, "clocks": clk}), flush=True)
     R.finish(world)
