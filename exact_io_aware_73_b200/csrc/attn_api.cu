@@ -791,7 +791,8 @@ size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
   // on the stream, so they share the partial slots
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t slots = bh + attn_b200::kDecMaxCtas;
-  const size_t g = Nq < 4 ? static_cast<size_t>(Nq) : 4;
+  constexpr int kGroup = attn_b200::kDecMaxQ;  // queries per launch
+  const size_t g = Nq < kGroup ? static_cast<size_t>(Nq) : kGroup;
   return round256(slots * g * d * 4) + round256(slots * g * 4) + round256(bh * 4);
 }
 
@@ -807,7 +808,9 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL_POINTER;
   const int64_t bh64 = static_cast<int64_t>(B) * H;
   if (Nk > ATTN_MAX_DECODE_KEYS || bh64 > ATTN_MAX_HEADS) return ATTN_ERR_INVALID_SIZE;
-  const int64_t ntiles = (Nk + attn_b200::kDecTileKeys - 1) / attn_b200::kDecTileKeys;
+  const int tile_keys = d == 128 ? attn_b200::DecSmem<128>::kTileKeys
+                                  : attn_b200::DecSmem<64>::kTileKeys;
+  const int64_t ntiles = (Nk + tile_keys - 1) / tile_keys;
   if (bh64 * ntiles > 0x7fffffffLL) return ATTN_ERR_INVALID_SIZE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4))
@@ -835,16 +838,17 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
   for (const void *ptr : all)
     if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
   const size_t slots = static_cast<size_t>(bh64) + attn_b200::kDecMaxCtas;
-  const size_t g = Nq < 4 ? static_cast<size_t>(Nq) : 4;
+  constexpr int kGroup = attn_b200::kDecMaxQ;  // queries per launch
+  const size_t g = Nq < kGroup ? static_cast<size_t>(Nq) : kGroup;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // groups of up to 4 queries, one launch each; under the causal mask a
   // group's last query sees keys 0 .. Nk - Nq + q0 + m - 1, so its launch
   // stops there (same visibility rule with Nk' = that count, Nq' = m)
-  for (int q0 = 0; q0 < Nq; q0 += 4) {
-    const int m = (Nq - q0 < 4) ? (Nq - q0) : 4;
+  for (int q0 = 0; q0 < Nq; q0 += kGroup) {
+    const int m = (Nq - q0 < kGroup) ? (Nq - q0) : kGroup;
     const int nk = causal ? Nk - Nq + q0 + m : Nk;
-    const int64_t ntiles = (nk + attn_b200::kDecTileKeys - 1) / attn_b200::kDecTileKeys;
+    const int64_t ntiles = (nk + tile_keys - 1) / tile_keys;
     attn_b200::DecodeParams p;
     p.q = static_cast<const uint16_t *>(q) + static_cast<int64_t>(q0) * d;
     p.k = static_cast<const uint16_t *>(k);

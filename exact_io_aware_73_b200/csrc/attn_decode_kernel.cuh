@@ -50,8 +50,7 @@
 
 namespace attn_b200 {
 
-constexpr int kDecTileKeys = 64;
-constexpr int kDecMaxQ = 16;           // queries per (batch, head)
+constexpr int kDecMaxQ = 4;            // queries per (batch, head) and launch
 constexpr int kDecComputeWarps = 8;
 constexpr int kDecComputeThreads = kDecComputeWarps * 32;
 constexpr int kDecThreads = kDecComputeThreads + 32;  // + producer warp
@@ -60,19 +59,27 @@ constexpr float kDecLazy = 8.f;        // log2 units: p <= 2^8
 
 template <int D>
 struct DecSmem {
-  static constexpr uint32_t kTileBytes = kDecTileKeys * D * 2;  // K or V tile
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  // keys per tile: 16 KB of K (and of V) either way; at d = 64 each lane
+  // group takes two keys of its warp's slice, so that every query value it
+  // reads from shared memory serves two keys
+  static constexpr int kTileKeys = (D == 64) ? 128 : 64;
+  static constexpr int kKeysPerLane = kTileKeys / (8 * kDecComputeWarps);  // R
+  static constexpr int kSlice = 8 * kKeysPerLane;  // keys of a warp per tile
+  static constexpr uint32_t kTileBytes = kTileKeys * D * 2;  // K or V tile
+  static constexpr int kStages = 3;
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kStages * kTileBytes;
-  // the head's queries (fp32 [16][D], pre-scaled) while a share runs; at its
-  // end the same bytes hold the warps' O for a round of kRedQ queries
+  // the head's queries (fp32 [4][D], pre-scaled; within a query the first
+  // halves of all 8-dimension chunks, then the second halves) while a share
+  // runs; at its end the same bytes hold the warps' O for a round of kRedQ
+  // queries
   static constexpr uint32_t kRedBytes = 8 * 1024;
   static constexpr int kRedQ = kRedBytes / (kDecComputeWarps * D * 4);  // 2 or 4
   static_assert(kDecMaxQ * D * 4 <= kRedBytes, "queries fit the shared region");
   static constexpr uint32_t kQ = kV + kStages * kTileBytes;
-  // each warp's probabilities of its current slice, [8 keys][16 queries]
+  // each warp's probabilities of its current slice, [kSlice keys][4 queries]
   static constexpr uint32_t kP = kQ + kRedBytes;
-  static constexpr uint32_t kStat = kP + kDecComputeWarps * 8 * kDecMaxQ * 4;  // m, l [8][16][2]
+  static constexpr uint32_t kStat = kP + kDecComputeWarps * kSlice * kDecMaxQ * 4;  // m, l [8][4][2]
   static constexpr uint32_t kBars = kStat + kDecComputeWarps * kDecMaxQ * 8;
   static constexpr int FULL = 0, EMPTY = kStages, NUM_BARS = 2 * kStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;         // abort flag, last flag
@@ -165,10 +172,10 @@ __device__ __forceinline__ void dec_producer(uint32_t base, const DecodeParams &
       ++issued;
       continue;
     }
-    const int rows = min(kDecTileKeys, p.nk - j * kDecTileKeys);
+    const int rows = min(L::kTileKeys, p.nk - j * L::kTileKeys);
     const uint32_t bytes = static_cast<uint32_t>(rows) * D * 2;
     mbar_arrive_expect_tx(bar(L::FULL + st), 2 * bytes);
-    const int64_t off = (static_cast<int64_t>(h) * p.kstride + j * kDecTileKeys) * D;
+    const int64_t off = (static_cast<int64_t>(h) * p.kstride + j * L::kTileKeys) * D;
     bulk_g2s(base + L::kK + st * L::kTileBytes, p.k + off, bytes, bar(L::FULL + st));
     bulk_g2s(base + L::kV + st * L::kTileBytes, p.v + off, bytes, bar(L::FULL + st));
     ++issued;
@@ -189,22 +196,33 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 
 // ------------------------------------------------------------------ compute
 
-// One CTA's share of key tiles, head part by head part.  QMAX (4 or 16)
-// bounds the queries so that a lane's per-query state stays in registers.
+// One CTA's share of key tiles, head part by head part.  QMAX (the 4
+// queries of a launch) bounds the queries so that a lane's per-query state
+// stays in registers.
+//
+// Lane (kl, q4) = (lane / 4, lane % 4) of warp w scores keys
+// w * kSlice + kl + 8 r (r < R), a quarter of the dimensions each: the
+// 16-byte chunks q4, q4 + 4, ... of the row, visited in the order
+// c ^ (kl & 1) so that the two keys read by one quarter-warp fall in
+// different banks (rows are 128 or 256 bytes, so the same chunk of two rows
+// shares banks).  The queries' matching halves of those chunks lie 16 bytes
+// apart in the query layout, so their reads are conflict-free too.
 template <int D, int QMAX>
 __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
                                             const DecodeParams &p, const WaitCtx &wc,
                                             int g0, int g1, int warp, int lane) {
   using L = DecSmem<D>;
+  static_assert(QMAX == kDecMaxQ, "one query group per launch");
   constexpr int E = D / 32;        // output dimensions per lane
   constexpr int kChunks = D / 8;   // 16-byte chunks per row
+  constexpr int R = L::kKeysPerLane;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   const int tid = warp * 32 + lane;
   const int kl = lane >> 2, q4 = lane & 3;  // key of the warp's slice, quarter
   float *qf = reinterpret_cast<float *>(smem + L::kQ);
   float *red = qf;  // the same bytes once the share's last tile is done
   float *stat = reinterpret_cast<float *>(smem + L::kStat);
-  float *pw = reinterpret_cast<float *>(smem + L::kP) + warp * 8 * kDecMaxQ;
+  float *pw = reinterpret_cast<float *>(smem + L::kP) + warp * L::kSlice * kDecMaxQ;
   volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
   int cons = 0;
   for (int g = g0; g < g1;) {
@@ -212,8 +230,12 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
     const int gend = min(g1, (h + 1) * p.ntiles);
     dec_bar();  // the previous part's readers of the shared region are done
     const uint16_t *qsrc = p.q + static_cast<int64_t>(h) * p.qstride * D;
-    for (int i = tid; i < p.nq * D; i += kDecComputeThreads)
-      qf[i] = __uint_as_float(static_cast<uint32_t>(qsrc[i]) << 16) * p.c_log2;
+    for (int i = tid; i < p.nq * D; i += kDecComputeThreads) {
+      // dimension x of query q: chunk x / 8, half (x / 4) & 1, element x & 3
+      const int q = i / D, x = i - q * D;
+      const int at = q * D + ((x >> 2) & 1) * (D / 2) + (x >> 3) * 4 + (x & 3);
+      qf[at] = __uint_as_float(static_cast<uint32_t>(qsrc[i]) << 16) * p.c_log2;
+    }
     dec_bar();
     float m_w[QMAX], l_w[QMAX], acc[QMAX][E];
 #pragma unroll
@@ -230,31 +252,46 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::FULL + st), (cons / L::kStages) & 1,
                                              wc, kRoleSoftmax));
       if (!ok) break;
-      const int rows = min(kDecTileKeys, p.nk - j * kDecTileKeys);
-      const int key = warp * 8 + kl;  // this lane's key within the tile
-      const bool kvalid = key < rows;
-      const int kabs = j * kDecTileKeys + key;
+      const int rows = min(L::kTileKeys, p.nk - j * L::kTileKeys);
       const uint8_t *kt = smem + L::kK + st * L::kTileBytes;
       const uint8_t *vt = smem + L::kV + st * L::kTileBytes;
-      // 1. scores of the slice's 8 keys
-      float s[QMAX];
+      int key[R];
+      bool kvalid[R];
 #pragma unroll
-      for (int q = 0; q < QMAX; ++q) s[q] = 0.f;
-      if (kvalid) {
+      for (int r = 0; r < R; ++r) {
+        key[r] = warp * L::kSlice + kl + 8 * r;  // this lane's keys within the tile
+        kvalid[r] = key[r] < rows;
+      }
+      // 1. scores of the slice's keys
+      float s[R][QMAX];
 #pragma unroll
-        for (int c = 0; c < kChunks / 4; ++c) {
-          const int ch = q4 + 4 * c;
-          const uint4 raw = *reinterpret_cast<const uint4 *>(kt + key * D * 2 + ch * 16);
-          const float kf[8] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y),
-                               bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w)};
+      for (int r = 0; r < R; ++r)
 #pragma unroll
-          for (int q = 0; q < QMAX; ++q) {
-            if (q >= p.nq) break;
-            const float4 a = *reinterpret_cast<const float4 *>(qf + q * D + ch * 8);
-            const float4 b = *reinterpret_cast<const float4 *>(qf + q * D + ch * 8 + 4);
-            s[q] = fmaf(a.x, kf[0], fmaf(a.y, kf[1], fmaf(a.z, kf[2], fmaf(a.w, kf[3],
-                   fmaf(b.x, kf[4], fmaf(b.y, kf[5], fmaf(b.z, kf[6], fmaf(b.w, kf[7], s[q]))))))));
-          }
+        for (int q = 0; q < QMAX; ++q) s[r][q] = 0.f;
+#pragma unroll
+      for (int c = 0; c < kChunks / 4; ++c) {
+        const int ch = q4 + 4 * (c ^ (kl & 1));
+        float kf[R][8];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint4 raw = kvalid[r]
+              ? *reinterpret_cast<const uint4 *>(kt + key[r] * D * 2 + ch * 16)
+              : make_uint4(0u, 0u, 0u, 0u);
+          kf[r][0] = bf16lo(raw.x); kf[r][1] = bf16hi(raw.x);
+          kf[r][2] = bf16lo(raw.y); kf[r][3] = bf16hi(raw.y);
+          kf[r][4] = bf16lo(raw.z); kf[r][5] = bf16hi(raw.z);
+          kf[r][6] = bf16lo(raw.w); kf[r][7] = bf16hi(raw.w);
+        }
+#pragma unroll
+        for (int q = 0; q < QMAX; ++q) {
+          if (q >= p.nq) break;
+          const float4 a = *reinterpret_cast<const float4 *>(qf + q * D + ch * 4);
+          const float4 b = *reinterpret_cast<const float4 *>(qf + q * D + D / 2 + ch * 4);
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+            s[r][q] = fmaf(a.x, kf[r][0], fmaf(a.y, kf[r][1], fmaf(a.z, kf[r][2],
+                      fmaf(a.w, kf[r][3], fmaf(b.x, kf[r][4], fmaf(b.y, kf[r][5],
+                      fmaf(b.z, kf[r][6], fmaf(b.w, kf[r][7], s[r][q]))))))));
         }
       }
       // 2. the warp's online softmax over its slice (all lanes of a key
@@ -262,11 +299,17 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
 #pragma unroll
       for (int q = 0; q < QMAX; ++q) {
         if (q >= p.nq) break;  // uniform across the warp
-        s[q] += __shfl_xor_sync(0xffffffffu, s[q], 1);
-        s[q] += __shfl_xor_sync(0xffffffffu, s[q], 2);
-        if (!(kvalid && (!p.causal || kabs <= p.nk - p.nq + q))) s[q] = -CUDART_INF_F;
-        if (__any_sync(0xffffffffu, s[q] > m_w[q] + kDecLazy)) {
-          float tm = s[q];
+        float smax = -CUDART_INF_F;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          s[r][q] += __shfl_xor_sync(0xffffffffu, s[r][q], 1);
+          s[r][q] += __shfl_xor_sync(0xffffffffu, s[r][q], 2);
+          const int kabs = j * L::kTileKeys + key[r];
+          if (!(kvalid[r] && (!p.causal || kabs <= p.nk - p.nq + q))) s[r][q] = -CUDART_INF_F;
+          smax = fmaxf(smax, s[r][q]);
+        }
+        if (__any_sync(0xffffffffu, smax > m_w[q] + kDecLazy)) {
+          float tm = smax;
           tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
           tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
           tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
@@ -277,16 +320,19 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
           for (int e = 0; e < E; ++e) acc[q][e] *= alpha;
           m_w[q] = mn;
         }
-        // p <= 2^8; no visible key yet (m = -inf) means p = 0
-        const float pk = (m_w[q] == -CUDART_INF_F) ? 0.f : ex2_approx(s[q] - m_w[q]);
-        l_w[q] += pk;  // each of the key's four lanes adds it: l = sum / 4
-        if ((q & 3) == q4) pw[kl * kDecMaxQ + q] = pk;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          // p <= 2^8; no visible key yet (m = -inf) means p = 0
+          const float pk = (m_w[q] == -CUDART_INF_F) ? 0.f : ex2_approx(s[r][q] - m_w[q]);
+          l_w[q] += pk;  // each of the key's four lanes adds it: l = sum / 4
+          if (q == q4) pw[(kl + 8 * r) * kDecMaxQ + q] = pk;
+        }
       }
       __syncwarp();
       // 3. O += p v over the slice's keys, E dimensions per lane
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int krow = warp * 8 + k;
+      for (int k = 0; k < L::kSlice; ++k) {
+        const int krow = warp * L::kSlice + k;
         if (krow >= rows) break;  // uniform across the warp
         float vv[E];
         if constexpr (E == 4) {
@@ -296,18 +342,13 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
           const uint32_t w1 = *reinterpret_cast<const uint32_t *>(vt + krow * D * 2 + lane * 4);
           vv[0] = bf16lo(w1); vv[1] = bf16hi(w1);
         }
+        const float4 pq = *reinterpret_cast<const float4 *>(pw + k * kDecMaxQ);
+        const float pv4[4] = {pq.x, pq.y, pq.z, pq.w};
 #pragma unroll
-        for (int q4b = 0; q4b < QMAX; q4b += 4) {
-          if (q4b >= p.nq) break;
-          const float4 pq = *reinterpret_cast<const float4 *>(pw + k * kDecMaxQ + q4b);
-          const float pv4[4] = {pq.x, pq.y, pq.z, pq.w};
+        for (int q = 0; q < QMAX; ++q) {
+          if (q >= p.nq) break;
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            if (q4b + qq >= p.nq) break;
-#pragma unroll
-            for (int e = 0; e < E; ++e)
-              acc[q4b + qq][e] = fmaf(pv4[qq], vv[e], acc[q4b + qq][e]);
-          }
+          for (int e = 0; e < E; ++e) acc[q][e] = fmaf(pv4[q], vv[e], acc[q][e]);
         }
       }
       __syncwarp();
@@ -425,7 +466,7 @@ __device__ __forceinline__ void dec_compute(uint32_t base, uint8_t *smem,
 // ------------------------------------------------------------------ kernel
 
 template <int D, int QMAX>
-__global__ void __launch_bounds__(kDecThreads, QMAX <= 4 ? 2 : 1)
+__global__ void __launch_bounds__(kDecThreads, 2)
     attn_decode_kernel(const DecodeParams p) {
   using L = DecSmem<D>;
   extern __shared__ __align__(128) uint8_t dsmem[];
