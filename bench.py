@@ -86,8 +86,11 @@ def load_traffic(workload: str, prefix: str = "traffic_", sources=KERNEL_SOURCES
 
 
 class ClockSampler:
-    """SM clock and throttle reasons sampled every 10 ms through NVML while
-    the timed region runs (read-only queries); nvidia-smi is the fallback."""
+    """SM clock and throttle reasons sampled every 10 ms through NVML
+    (read-only queries; nvidia-smi is the fallback), each sample with its
+    host time.  begin() / end() mark the timed region; the record keeps the
+    samples inside it, or, when the region is shorter than the sampling
+    needs, the last sample before it and the first after it."""
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
                "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
@@ -98,6 +101,8 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = None
         self._nvml = None
+        self.t_begin = None
+        self.t_end = None
 
     def start(self):
         try:
@@ -132,22 +137,46 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(self._query())
+                mhz, mask = self._query()
+                self.samples.append((time.monotonic(), mhz, mask))
             except Exception:
                 return
             self._stop.wait(0.01 if self._nvml is not None else 0.2)
 
+    def begin(self):
+        self.t_begin = time.monotonic()
+
+    def end(self):
+        self.t_end = time.monotonic()
+
     def stop(self):
+        if self.t_end is None:
+            self.end()
+        if self.t_begin is None:  # started right before the region
+            self.t_begin = self.samples[0][0] if self.samples else self.t_end
+        # keep sampling until one sample lies after the region
+        for _ in range(50):
+            if self.samples and self.samples[-1][0] >= self.t_end:
+                break
+            time.sleep(0.01)
         self._stop.set()
         if self._t:
             self._t.join(timeout=5)
         if not self.samples:
             return None
+        inside = [x for x in self.samples if self.t_begin <= x[0] <= self.t_end]
+        where = "inside the timed region"
+        if len(inside) < 2:
+            before = [x for x in self.samples if x[0] < self.t_begin][-1:]
+            after = [x for x in self.samples if x[0] > self.t_end][:1]
+            inside = inside + before + after
+            where = "the region's own samples plus the nearest one on each side"
         reasons = sorted(n for n, bit in self.REASONS.items()
-                         if any(m & bit for _, m in self.samples))
-        return {"sm_mhz": statistics.median(c for c, _ in self.samples),
+                         if any(m & bit for _, _, m in inside))
+        return {"sm_mhz": statistics.median(c for _, c, _ in inside),
                 "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(self.samples),
+                "samples": len(inside), "window": where,
+                "region_ms": round((self.t_end - self.t_begin) * 1e3, 1),
                 "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
@@ -276,14 +305,15 @@ def run_backward(args, w):
         if rc != 0:
             raise attn.AttnError(rc, "attn_bwd")
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     if attn.status() != 0:
         raise RuntimeError("device status after warm-up")
-    clocks = ClockSampler(local)
-    clocks.start()
     R.barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.begin()
     evs = []
     for _ in range(args.steps):
         if flush is not None:
@@ -296,6 +326,7 @@ def run_backward(args, w):
         evs.append((a, b))
     R.barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.end()
     clk = clocks.stop()
     if attn.status() != 0:
         raise RuntimeError("device status after the timed region")
@@ -440,17 +471,19 @@ def run_fp8(args, w):
         torch.cuda.synchronize(dev)
         return sum(a.elapsed_time(b) for a, b in evs)
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
         kernel_only()
     if attn.status() != 0:
         raise RuntimeError("device status after warm-up")
-    clocks = ClockSampler(local)
-    clocks.start()
     R.barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.begin()
     step_ms = timed(step, args.steps)
     kern_ms = timed(kernel_only, args.steps)
+    clocks.end()
     clk = clocks.stop()
     if attn.status() != 0:
         raise RuntimeError("device status after the timed region")
@@ -588,14 +621,15 @@ def run_decode(args):
         if rc != 0:
             raise attn.AttnError(rc, "attn_decode")
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     if attn.status() != 0:
         raise RuntimeError("device status after warm-up")
-    clocks = ClockSampler(local)
-    clocks.start()
     R.barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.begin()
     evs = []
     for _ in range(args.steps):
         if flush is not None:
@@ -608,6 +642,7 @@ def run_decode(args):
         evs.append((a, b))
     R.barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.end()
     clk = clocks.stop()
     if attn.status() != 0:
         raise RuntimeError("device status after the timed region")
@@ -716,14 +751,15 @@ def run_seqpar(args, w):
         def step():
             return seqpar.ring_attention_emulated(qs, ks, vs, w.causal, w.scale)
     stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     if attn.status() != 0:
         raise RuntimeError("device status after warm-up")
-    clocks = ClockSampler(local)
-    clocks.start()
     R.barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.begin()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
@@ -732,6 +768,7 @@ def run_seqpar(args, w):
     b.record(stream)
     R.barrier(world)
     torch.cuda.synchronize(dev)
+    clocks.end()
     clk = clocks.stop()
     if attn.status() != 0:
         raise RuntimeError("device status after the timed region")
@@ -838,6 +875,8 @@ def main():
         if rc != 0:
             raise attn.AttnError(rc, "attn_fwd")
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     rc = attn.status()
@@ -845,10 +884,9 @@ def main():
         raise attn.AttnError(rc, "warm-up")
 
     # ---- device-timed region
-    clocks = ClockSampler(local)
-    clocks.start()
     barrier()
     torch.cuda.synchronize(dev)
+    clocks.begin()
     if flush is None:
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
@@ -873,6 +911,7 @@ def main():
         torch.cuda.synchronize(dev)
         kernel_ms = sum(a.elapsed_time(b) for a, b in evs)
         l2_note = "L2 flushed between steps (252 MiB write outside the events)"
+    clocks.end()
     clk = clocks.stop()
     rc = attn.status()
     if rc != 0:
