@@ -511,17 +511,34 @@ int attn_fwd_host(const void *q, const void *k, const void *v, void *o,
   // run on three streams so that they overlap chunk i+1's copies in and
   // chunk i-1's copies out.  `stream` orders the whole call: the streams
   // start after its earlier work and it waits for the last copy out.
-  const int nchunks = (tb >= (32u << 20)) ? (bh < kHostChunks ? bh : kHostChunks) : 1;
-  const int per = (bh + nchunks - 1) / nchunks;
+  // The step ends with the last chunk's kernel and copies out, after all
+  // copies in; the chunks therefore shrink towards the end (for 32 heads:
+  // 6, 6, 6, 6, 4, 2, 1, 1), so that little work is left once the last
+  // copy in lands.  Compute (a few ms) stays well behind the copies in.
+  int sizes[kHostChunks];
+  int nchunks = 1;
+  sizes[0] = bh;
+  if (tb >= (32u << 20) && bh > 1) {
+    if (bh <= kHostChunks) {
+      nchunks = bh;
+      for (int c = 0; c < nchunks; ++c) sizes[c] = 1;
+    } else {
+      const int tail[4] = {bh / 8 > 0 ? bh / 8 : 1, bh / 16 > 0 ? bh / 16 : 1,
+                           bh / 32 > 0 ? bh / 32 : 1, bh / 32 > 0 ? bh / 32 : 1};
+      const int head = bh - (tail[0] + tail[1] + tail[2] + tail[3]);
+      nchunks = kHostChunks;
+      for (int c = 0; c < 4; ++c) sizes[c] = head / 4 + (c < head % 4 ? 1 : 0);
+      for (int c = 0; c < 4; ++c) sizes[4 + c] = tail[c];
+    }
+  }
   std::lock_guard<std::mutex> lk(hp->mu);
   auto fail = [] { cudaGetLastError(); return ATTN_ERR_CUDA; };
   if (cudaEventRecord(hp->start, s) != cudaSuccess) return fail();
   for (cudaStream_t t : {hp->h2d, hp->comp, hp->d2h})
     if (cudaStreamWaitEvent(t, hp->start, 0) != cudaSuccess) return fail();
-  for (int c = 0; c < nchunks; ++c) {
-    const int h0 = c * per;
-    const int nh = (bh - h0 < per) ? (bh - h0) : per;
-    if (nh <= 0) break;
+  for (int c = 0, h0 = 0; c < nchunks; h0 += sizes[c], ++c) {
+    const int nh = sizes[c];
+    if (nh <= 0) continue;
     const size_t off = static_cast<size_t>(h0) * N * d * 2;
     const size_t len = static_cast<size_t>(nh) * N * d * 2;
     const size_t loff = static_cast<size_t>(h0) * N, llen = static_cast<size_t>(nh) * N;
