@@ -51,13 +51,38 @@ DECODE_SOURCES = ("attn_decode_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cu
 BWD_SOURCES = ("attn_bwd_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and with whitespace runs collapsed, so
+    that editing a comment does not change the hash of the code."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":  # string or character literal: copied as is
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
-    """Hash of the device-code sources; a committed traffic figure is only
-    used while it matches (the counters describe that exact kernel)."""
+    """Hash of the device code (comments and whitespace ignored); a committed
+    traffic figure is only used while it matches (the counters describe that
+    exact kernel)."""
     h = hashlib.sha256()
     for f in sources:
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

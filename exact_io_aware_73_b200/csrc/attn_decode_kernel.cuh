@@ -13,14 +13,15 @@
 // groups of 4 by successive launches, each stopping at the last key its
 // queries can see.  The kernel therefore streams K/V through shared memory
 // with bulk asynchronous copies and does the arithmetic on the CUDA cores:
-//   * stream-K split: the B*H*ceil(Nk/64) key tiles of all heads are one
-//     sequence; CTA c takes tiles [c T, (c+1) T) -- an equal share, which may
+//   * stream-K split: the B*H*ceil(Nk/K) key tiles of all heads are one
+//     sequence (K = 64 keys at d = 128, 128 at d = 64: 16 KB of K either
+//     way); CTA c takes tiles [c T, (c+1) T) -- an equal share, which may
 //     cross heads -- so every SM streams the same number of bytes whatever
 //     B*H is;
-//   * per CTA: one producer warp (one elected lane) fills a ring of K/V
-//     stages (cp.async.bulk, one copy per 64-key K or V tile, completion on
-//     an mbarrier); eight compute warps each own an 8-key slice of every
-//     tile and run their own online softmax over it -- no communication
+//   * per CTA: one producer warp (one elected lane) fills a 3-stage ring of
+//     K/V tiles (cp.async.bulk, one copy per K or V tile, completion on an
+//     mbarrier); eight compute warps each own a slice of every tile (8 or 16
+//     keys) and run their own online softmax over it -- no communication
 //     between warps inside a tile:
 //       1. scores s[q][key] = (q . k) * scale * log2(e): four lanes per key,
 //          each a quarter of the dimensions, reduced by two shuffles;
@@ -28,8 +29,8 @@
 //          moves (with a rescale of l and O) only when a score exceeds it by
 //          more than 2^8 -- a warp vote per query, the maximum reduction
 //          only when the vote says so; each lane keeps its own part of l;
-//       3. O[q] += sum over the 8 keys of p v_key, each lane D/32 dimensions
-//          (p passed through the warp's slice of shared memory);
+//       3. O[q] += sum over the slice's keys of p v_key, each lane D/32
+//          dimensions (p passed through the warp's slice of shared memory);
 //     at the end of a head's share the eight warps' (m, l, O) are combined
 //     through shared memory (O in rounds of a few queries);
 //   * merge: a CTA that finished part of a head writes the part's (O_s,
