@@ -77,6 +77,35 @@ def _check(rc: int, what: str):
         raise AttnError(rc, what)
 
 
+def _expect(name, t, dtype, shape=None, cuda=True, device=None, numel=None):
+    """Refuse a tensor the C ABI would misread: it sees only a pointer, so
+    dtype, layout (contiguous) and shape are checked here (or only the
+    element count, for arrays whose leading dimensions may be merged)."""
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.is_cuda != cuda:
+        where = "CUDA" if cuda else "host"
+        raise TypeError(f"{name} must be a {dtype} {where} tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} must have {numel} elements, got {t.numel()}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, like the queries")
+
+
+def _expect_qkv(q, k, v, cuda=True):
+    """q, k, v: 4-D bf16 tensors of one shape [B, H, N, d] (on one device)."""
+    import torch
+    _expect("q", q, torch.bfloat16, cuda=cuda)
+    if q.dim() != 4:
+        raise ValueError("q must be 4-D [B, H, N, d]")
+    dev = q.device if cuda else None
+    _expect("k", k, torch.bfloat16, q.shape, cuda, dev)
+    _expect("v", v, torch.bfloat16, q.shape, cuda, dev)
+
+
 def attn_fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, causal,
                  scale, stream_handle) -> int:
     """Direct call with integer pointers; returns the library's code."""
@@ -92,13 +121,7 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None,
     Allocates O (bf16) and lse (fp32 [B, H, N]) with torch unless given.
     """
     import torch
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 4:
-            raise TypeError(f"{name} must be a 4-D bf16 CUDA tensor")
-        if not t.is_contiguous():
-            raise ValueError(f"{name} must be contiguous [B, H, N, d]")
-    if k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    _expect_qkv(q, k, v)
     B, H, N, d = q.shape
     if scale is None:
         scale = d ** -0.5
@@ -106,6 +129,8 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _expect("out", out, torch.bfloat16, q.shape, device=q.device)
+    _expect("lse", lse, torch.float32, (B, H, N), device=q.device)
     rc = attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                       lse.data_ptr(), B, H, N, d, causal, scale,
                       _stream_handle(stream))
@@ -118,7 +143,12 @@ def attn_fwd_host(q, k, v, out, lse, causal: bool, scale: float, workspace,
     """End-to-end call on host (ideally pinned) bf16 tensors; `workspace` is a
     CUDA uint8 tensor of at least ``host_workspace_bytes`` bytes.  Queued on
     `stream`; synchronise before reading `out` / `lse`."""
+    import torch
+    _expect_qkv(q, k, v, cuda=False)
     B, H, N, d = q.shape
+    _expect("out", out, torch.bfloat16, q.shape, cuda=False)
+    _expect("lse", lse, torch.float32, (B, H, N), cuda=False)
+    _expect("workspace", workspace, torch.uint8)
     rc = lib().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                              out.data_ptr(), lse.data_ptr(), B, H, N, d,
                              int(bool(causal)), float(scale),
@@ -171,7 +201,11 @@ def attn_fwd_host_noalloc(q, k, v, out, lse, causal: bool, scale: float,
     a static 32 MiB device array inside the library, shared by every call on
     the device (so overlapping calls race).  Synchronous: `out` and `lse` are
     filled on return.  For callers without a device allocator of their own."""
+    import torch
+    _expect_qkv(q, k, v, cuda=False)
     B, H, N, d = q.shape
+    _expect("out", out, torch.bfloat16, q.shape, cuda=False)
+    _expect("lse", lse, torch.float32, (B, H, N), cuda=False)
     rc = _noalloc_fn()(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                        out.data_ptr(), lse.data_ptr(), B, H, N, d,
                        int(bool(causal)), float(scale), _stream_handle(stream))
@@ -224,13 +258,18 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False,
     """dQ, dK, dV of attn_fwd for upstream gradient dout (bf16 CUDA tensors
     [B, H, N, d]; o and lse are attn_fwd's outputs)."""
     import torch
+    _expect_qkv(q, k, v)
     B, H, N, d = q.shape
+    _expect("o", o, torch.bfloat16, q.shape, device=q.device)
+    _expect("dout", dout, torch.bfloat16, q.shape, device=q.device)
+    _expect("lse", lse, torch.float32, (B, H, N), device=q.device)
     if scale is None:
         scale = d ** -0.5
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     need = bwd_workspace_bytes(B, H, N)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _expect("workspace", workspace, torch.uint8, device=q.device)
     rc = attn_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                       dout.data_ptr(), lse.data_ptr(), dq.data_ptr(),
                       dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
@@ -294,6 +333,9 @@ def fp8_quantize(x, rotate: bool, signs=None, per_head: bool = False,
     [B, H, N, 128]: per 128-row tile ([B, H, ceil(N/128)]) or per head
     ([B, H]); Q and K rotated with the signs when `rotate`."""
     import torch
+    _expect("x", x, torch.bfloat16)
+    if x.dim() != 4:
+        raise ValueError("x must be 4-D [B, H, N, d]")
     B, H, N, d = x.shape
     lo, hi = sign_mask(signs) if rotate else (0, 0)
     tiles = -(-N // 128)
@@ -315,7 +357,18 @@ def attn_fwd_fp8_quantized(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
     """O (bf16), lse of the FP8 attention on quantized operands; `scale` is
     the softmax scale of the problem the codes encode."""
     import torch
+    _expect("q8", q8, torch.uint8)
+    if q8.dim() != 4:
+        raise ValueError("q8 must be 4-D [B, H, N, d]")
     B, H, N, d = q8.shape
+    tiles = -(-N // 128)
+    dev = q8.device
+    _expect("k8", k8, torch.uint8, q8.shape, device=dev)
+    _expect("v8", v8, torch.uint8, q8.shape, device=dev)
+    # scales: [B, H, tiles] and [B, H] in memory (any merging of B and H)
+    _expect("q_scale", q_scale, torch.float32, device=dev, numel=B * H * tiles)
+    _expect("k_scale", k_scale, torch.float32, device=dev, numel=B * H * tiles)
+    _expect("v_scale", v_scale, torch.float32, device=dev, numel=B * H)
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
     rc = _fp8_fns().attn_fwd_fp8_quantized(
@@ -341,6 +394,7 @@ def attn_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None,
     and block-quantized to E4M3 with V, then the FP8 kernel.  Returns
     (O bf16, lse fp32)."""
     import torch
+    _expect_qkv(q, k, v)
     B, H, N, d = q.shape
     if scale is None:
         scale = d ** -0.5
@@ -349,9 +403,12 @@ def attn_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _expect("out", out, torch.bfloat16, q.shape, device=q.device)
+    _expect("lse", lse, torch.float32, (B, H, N), device=q.device)
     need = fp8_workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _expect("workspace", workspace, torch.uint8, device=q.device)
     rc = attn_fwd_fp8_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                           out.data_ptr(), lse.data_ptr(), B, H, N, d, causal,
                           scale, signs is not None, lo, hi,
@@ -377,7 +434,7 @@ def _decode_fns():
     return L
 
 
-DECODE_MAX_Q = 16
+DECODE_MAX_Q = 16  # served in groups of 4 queries, one launch each
 
 
 def decode_workspace_bytes(B, H, Nq, Nk, d) -> int:
@@ -398,22 +455,29 @@ def attn_decode_raw(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, ws,
 
 def attn_decode(q, k, v, causal: bool = True, scale: float | None = None,
                 workspace=None, out=None, lse=None, stream=None):
-    """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16)
-    against k, v bf16 [B, H, Nk, d]; returns (O bf16, lse fp32 [B, H, Nq])."""
+    """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16,
+    served 4 per launch) against k, v bf16 [B, H, Nk, d]; returns (O bf16,
+    lse fp32 [B, H, Nq])."""
     import torch
+    _expect("q", q, torch.bfloat16)
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be 4-D [B, H, Nq, d] and [B, H, Nk, d]")
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
-    if k.shape != (B, H, Nk, d) or v.shape != k.shape:
-        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H, d")
+    _expect("k", k, torch.bfloat16, (B, H, Nk, d), device=q.device)
+    _expect("v", v, torch.bfloat16, (B, H, Nk, d), device=q.device)
     if scale is None:
         scale = d ** -0.5
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _expect("out", out, torch.bfloat16, q.shape, device=q.device)
+    _expect("lse", lse, torch.float32, (B, H, Nq), device=q.device)
     need = decode_workspace_bytes(B, H, Nq, Nk, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _expect("workspace", workspace, torch.uint8, device=q.device)
     rc = attn_decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                          out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
                          causal, scale, workspace.data_ptr(), workspace.numel(),
@@ -439,8 +503,14 @@ def merge_fold(acc_o, acc_lse, part_o, part_lse, first: bool, stream=None):
     """Fold a partial result (part_o bf16 [..., d], part_lse fp32 [...]) into
     the fp32 accumulator (acc_o [..., d], acc_lse [...]) by the exact
     log-sum-exp merge; `first` initialises the accumulator."""
-    d = part_o.shape[-1]
+    import torch
+    _expect("part_lse", part_lse, torch.float32)
+    dev = part_lse.device
+    d = part_o.shape[-1] if part_o.dim() else 0
     rows = part_lse.numel()
+    _expect("part_o", part_o, torch.bfloat16, (*part_lse.shape, d), device=dev)
+    _expect("acc_o", acc_o, torch.float32, (*part_lse.shape, d), device=dev)
+    _expect("acc_lse", acc_lse, torch.float32, part_lse.shape, device=dev)
     rc = _merge_fns().attn_merge_fold(acc_o.data_ptr(), acc_lse.data_ptr(),
                                       part_o.data_ptr(), part_lse.data_ptr(),
                                       rows, d, int(bool(first)),
@@ -451,6 +521,9 @@ def merge_fold(acc_o, acc_lse, part_o, part_lse, first: bool, stream=None):
 def merge_finish(acc_o, acc_lse, stream=None):
     """(O bf16, lse fp32) from a merge accumulator."""
     import torch
+    _expect("acc_lse", acc_lse, torch.float32)
+    d = acc_o.shape[-1] if acc_o.dim() else 0
+    _expect("acc_o", acc_o, torch.float32, (*acc_lse.shape, d), device=acc_lse.device)
     o = torch.empty(acc_o.shape, dtype=torch.bfloat16, device=acc_o.device)
     lse = torch.empty_like(acc_lse)
     rc = _merge_fns().attn_merge_finish(acc_o.data_ptr(), acc_lse.data_ptr(),
@@ -477,7 +550,10 @@ def attn_fwd_merge(q, k, v, acc_o, acc_lse, mode: int, causal: bool = False,
         vp, i = ctypes.c_void_p, ctypes.c_int
         f.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, ctypes.c_float, i, vp]
         f.restype = i
+    _expect_qkv(q, k, v)
     B, H, N, d = q.shape
+    _expect("acc_o", acc_o, torch.float32, q.shape, device=q.device)
+    _expect("acc_lse", acc_lse, torch.float32, (B, H, N), device=q.device)
     if scale is None:
         scale = d ** -0.5
     o = lse = None
