@@ -31,9 +31,25 @@
 
 namespace attn_b200 {
 
-constexpr int kBwdThreads = 192;   // warps 0-3 compute, 4 loader, 5 MMA
-constexpr int kBwdLoaderWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+// Warps 0-7 compute, 8 loader, 9 MMA.  The compute work on a tile is
+// elementwise (P from the saved lse, dS from P, dP and D), so the two
+// compute warpgroups split its columns: warp w takes TMEM lane quarter w % 4
+// (rows 32 (w % 4) ..) and the 64 columns of half w / 4.  Two warps per SM
+// sub-partition hide each other's TMEM and MUFU latencies.
+constexpr int kBwdComputeWarps = 8;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdLoaderWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+
+// The two compute warps of TMEM lane quarter wq (warps wq and wq + 4) meet
+// here between loading their fp32 columns and storing bf16 results: chunk c's
+// bf16 values go to columns 16c .. 16c + 15, so the upper half's results
+// (c = 2, 3) land on fp32 columns 32 .. 63, which the lower half reads.
+__device__ __forceinline__ void bwd_pair_sync(int wq) {
+  tc_fence_before_sync();
+  asm volatile("barrier.cta.sync %0, 64;" ::"r"(1 + wq) : "memory");
+  tc_fence_after_sync();
+}
 
 struct BwdParams {
   const uint16_t *o;     // [BH, N, D] forward output (prep only)
@@ -143,10 +159,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(L::Q_EMPTY), 1);
     mbar_init(bar(L::S_FULL), 1);
     mbar_init(bar(L::DP_FULL), 1);
-    mbar_init(bar(L::S_FREE), 4);
-    mbar_init(bar(L::DS_FULL), 4);
+    mbar_init(bar(L::S_FREE), kBwdComputeWarps);
+    mbar_init(bar(L::DS_FULL), kBwdComputeWarps);
     mbar_init(bar(L::ACC_FULL), 1);
-    mbar_init(bar(L::ACC_EMPTY), 4);
+    mbar_init(bar(L::ACC_EMPTY), kBwdComputeWarps);
     mbar_init(bar(L::DRAIN), 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(bar(L::KV_FULL + s), 1);
@@ -277,8 +293,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else {
-    // compute warpgroup: thread = query row r of the tile
-    const int wq = warp;  // warps 0-3 = TMEM lane quarters 0-3
+    // compute warpgroups: thread = query row r of the tile, columns of half hc
+    const int wq = warp & 3;  // TMEM lane quarter
+    const int hc = warp >> 2;  // 64-column half of the tile
     const int r = wq * 32 + lane;
     const uint32_t lb = static_cast<uint32_t>(wq * 32) << 16;
     int s_cnt = 0, uocc = 0;
@@ -300,16 +317,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after_sync();
         const bool mask = (j == nkv - 1) && (CAUSAL || (p.n & (kBlockN - 1)));
         const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
-        float pr[128];
+        float pr[64];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * hc + cc;  // 32-column chunk of the tile
           uint32_t sv[32];
           tmem_ld_32x32b_x32(tS + lb + c * 32, sv);
           tmem_wait_ld(sv);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float e = ex2_approx(fmaf(__uint_as_float(sv[i]), p.c_log2, nlse));
-            pr[c * 32 + i] = (mask && c * 32 + i > limit) ? 0.f : e;
+            pr[cc * 32 + i] = (mask && c * 32 + i > limit) ? 0.f : e;
           }
         }
         tc_fence_before_sync();
@@ -321,18 +339,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after_sync();
+        uint32_t dv[2][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t dv[32];
-          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
-          tmem_wait_ld(dv);
+        for (int cc = 0; cc < 2; ++cc) tmem_ld_32x32b_x32(tdP + lb + (2 * hc + cc) * 32, dv[cc]);
+        tmem_wait_ld(dv[0]);
+        reg_fence(dv[1]);
+        bwd_pair_sync(wq);  // both halves hold their dP before dS overwrites it
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * hc + cc;
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(pr[c * 32 + 2 * i] * (__uint_as_float(dv[2 * i]) - drow),
-                                pr[c * 32 + 2 * i + 1] *
-                                    (__uint_as_float(dv[2 * i + 1]) - drow));
-          tmem_st_32x32b_x16(tdP + lb + c * 16, pk);  // over loaded dP columns
+            pk[i] = pack_bf16x2(pr[cc * 32 + 2 * i] * (__uint_as_float(dv[cc][2 * i]) - drow),
+                                pr[cc * 32 + 2 * i + 1] *
+                                    (__uint_as_float(dv[cc][2 * i + 1]) - drow));
+          tmem_st_32x32b_x16(tdP + lb + c * 16, pk);  // bf16 dS over dP columns
         }
         tmem_wait_st();
         tc_fence_before_sync();
@@ -347,7 +369,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after_sync();
       uint4 *out = reinterpret_cast<uint4 *>(p.dq + grow * D);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int c = hc * (D / 64) + cc;  // this half's 32-column chunks of dQ
         uint32_t o[32];
         tmem_ld_32x32b_x32(tdQ + lb + c * 32, o);
         tmem_wait_ld(o);
@@ -437,10 +460,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(L::KV_EMPTY), 1);
     mbar_init(bar(L::S_FULL), 1);
     mbar_init(bar(L::DP_FULL), 1);
-    mbar_init(bar(L::P_READY), 4);
-    mbar_init(bar(L::DS_READY), 4);
+    mbar_init(bar(L::P_READY), kBwdComputeWarps);
+    mbar_init(bar(L::DS_READY), kBwdComputeWarps);
     mbar_init(bar(L::ACC_FULL), 1);
-    mbar_init(bar(L::ACC_EMPTY), 4);
+    mbar_init(bar(L::ACC_EMPTY), kBwdComputeWarps);
     mbar_init(bar(L::DRAIN), 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(bar(L::Q_FULL + s), 1);
@@ -579,8 +602,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     __syncwarp();
   } else {
-    // compute warpgroup: thread = key row r of the tile
-    const int wq = warp;
+    // compute warpgroups: thread = key row r of the tile, query columns of
+    // half hc
+    const int wq = warp & 3;   // TMEM lane quarter
+    const int hc = warp >> 2;  // 64-column half of the tile
     const int r = wq * 32 + lane;
     const uint32_t lb = static_cast<uint32_t>(wq * 32) << 16;
     int s_cnt = 0, uocc = 0, q_cons = 0;
@@ -609,12 +634,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool diag = CAUSAL && (i == kt);
         const bool tail = (i == p.tiles - 1) && (p.n & (kBlockM - 1));
         const int qlimit = p.n - 1 - i * kBlockM;
-        float pr[128];
+        float pr[64];
+        uint32_t sv[2][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32];
-          tmem_ld_32x32b_x32(tS + lb + c * 32, sv);
-          tmem_wait_ld(sv);
+        for (int cc = 0; cc < 2; ++cc) tmem_ld_32x32b_x32(tS + lb + (2 * hc + cc) * 32, sv[cc]);
+        tmem_wait_ld(sv[0]);
+        reg_fence(sv[1]);
+        bwd_pair_sync(wq);  // both halves hold their S^T before P^T overwrites it
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * hc + cc;  // 32-column chunk of the tile
           uint32_t ppk[16];
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
@@ -623,13 +652,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int qc = c * 32 + 4 * g + e;  // query column in the tile
-              float pe = ex2_approx(fmaf(__uint_as_float(sv[4 * g + e]), p.c_log2,
+              float pe = ex2_approx(fmaf(__uint_as_float(sv[cc][4 * g + e]), p.c_log2,
                                          -lse4[e]));
               if ((diag && qc < r) || (tail && qc > qlimit)) pe = 0.f;
-              pr[qc] = pe;
+              pr[cc * 32 + 4 * g + e] = pe;
             }
-            ppk[2 * g] = pack_bf16x2(pr[c * 32 + 4 * g], pr[c * 32 + 4 * g + 1]);
-            ppk[2 * g + 1] = pack_bf16x2(pr[c * 32 + 4 * g + 2], pr[c * 32 + 4 * g + 3]);
+            ppk[2 * g] = pack_bf16x2(pr[cc * 32 + 4 * g], pr[cc * 32 + 4 * g + 1]);
+            ppk[2 * g + 1] = pack_bf16x2(pr[cc * 32 + 4 * g + 2], pr[cc * 32 + 4 * g + 3]);
           }
           tmem_st_32x32b_x16(tS + lb + c * 16, ppk);   // P^T over S^T
         }
@@ -643,21 +672,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after_sync();
+        uint32_t dv[2][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t dv[32];
-          tmem_ld_32x32b_x32(tdP + lb + c * 32, dv);
-          tmem_wait_ld(dv);
+        for (int cc = 0; cc < 2; ++cc) tmem_ld_32x32b_x32(tdP + lb + (2 * hc + cc) * 32, dv[cc]);
+        tmem_wait_ld(dv[0]);
+        reg_fence(dv[1]);
+        bwd_pair_sync(wq);  // both halves hold their dP^T before dS^T overwrites it
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * hc + cc;
           uint32_t dpk[16];
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
             const float4 dd = ld_shared_f4(vec + 512 + (c * 32 + 4 * g) * 4);
-            const int q4 = c * 32 + 4 * g;
-            dpk[2 * g] = pack_bf16x2(pr[q4] * (__uint_as_float(dv[4 * g]) - dd.x),
-                                     pr[q4 + 1] * (__uint_as_float(dv[4 * g + 1]) - dd.y));
+            const int q4 = cc * 32 + 4 * g;  // index into pr
+            dpk[2 * g] = pack_bf16x2(pr[q4] * (__uint_as_float(dv[cc][4 * g]) - dd.x),
+                                     pr[q4 + 1] * (__uint_as_float(dv[cc][4 * g + 1]) - dd.y));
             dpk[2 * g + 1] =
-                pack_bf16x2(pr[q4 + 2] * (__uint_as_float(dv[4 * g + 2]) - dd.z),
-                            pr[q4 + 3] * (__uint_as_float(dv[4 * g + 3]) - dd.w));
+                pack_bf16x2(pr[q4 + 2] * (__uint_as_float(dv[cc][4 * g + 2]) - dd.z),
+                            pr[q4 + 3] * (__uint_as_float(dv[cc][4 * g + 3]) - dd.w));
           }
           tmem_st_32x32b_x16(tdP + lb + c * 16, dpk);  // dS^T over dP^T
         }
@@ -681,7 +714,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float mul = which ? p.scale : 1.f;
         uint4 *out = reinterpret_cast<uint4 *>((which ? p.dk : p.dv) + grow * D);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int cc = 0; cc < D / 64; ++cc) {
+          const int c = hc * (D / 64) + cc;  // this half's 32-column chunks
           uint32_t o[32];
           tmem_ld_32x32b_x32(src + lb + c * 32, o);
           tmem_wait_ld(o);
