@@ -422,15 +422,20 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem,
                              | ((FP8 ? 0u : 1u) << 10)           // B: bf16 | e4m3
                              | ((uint32_t)(kBlockN >> 3) << 17)  // N
                              | ((uint32_t)(kBlockM >> 4) << 24); // M
+  // The descriptors are built once; a step adds its byte offset / 16 to the
+  // 14-bit address field (shared addresses are below 2^18 and 16-byte
+  // aligned, so the field cannot carry), which keeps the issuing thread's
+  // instructions between MMAs few.
+  const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024);
+  const uint64_t kd = smem_desc_sw128(k_smem, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < Smem<D, FP8>::kRowBytes / 32; ++kk) {
-    const uint32_t off = (kk >> 2) * Smem<D, FP8>::kPanelBytes + (kk & 3) * 32;
+    constexpr uint32_t kPanel = Smem<D, FP8>::kPanelBytes;
+    const uint64_t off = ((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
     if constexpr (FP8)
-      mma_f8_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024),
-                smem_desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
+      mma_f8_ss(d_tmem, qd + off, kd + off, idesc, kk > 0);
     else
-      mma_bf16_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024),
-                  smem_desc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
+      mma_bf16_ss(d_tmem, qd + off, kd + off, idesc, kk > 0);
   }
 }
 
@@ -448,10 +453,10 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
                              | ((uint32_t)(D >> 3) << 17)
                              | ((uint32_t)(kBlockM >> 4) << 24);
   constexpr int kKeys = FP8 ? 32 : 16;
+  const uint64_t vd = smem_desc_sw128(v_smem, Smem<D, FP8>::kPanelBytes, 1024);
 #pragma unroll
   for (int kk = 0; kk < kBlockN / kKeys; ++kk) {
-    const uint64_t bdesc =
-        smem_desc_sw128(v_smem + kk * kKeys * 128, Smem<D, FP8>::kPanelBytes, 1024);
+    const uint64_t bdesc = vd + static_cast<uint64_t>((kk * kKeys * 128) >> 4);
     if constexpr (FP8)
       mma_f8_ts(d_tmem, p_tmem + kk * 8, bdesc, idesc, (accumulate || kk > 0) ? 1u : 0u);
     else
