@@ -601,14 +601,16 @@ __device__ __forceinline__ float row_max_raw(const uint32_t (&s)[4][32]) {
 // p = 2^(s * scale * log2 e - m) for the whole row: one packed FMA per pair,
 // the exponential on the MUFU unit or (kEmuPer8 pairs in 8) the FMA pipe,
 // packed row sums, bf16x2 packing for the P.V MMA.  Returns the row sum.
-template <int D>
+template <int D, int HALF>
 __device__ __forceinline__ float exp_row(const uint32_t (&s)[4][32], float cl2,
-                                         float m, uint32_t (&pk)[2][32]) {
+                                         float m, uint32_t (&pk)[32]) {
+  // columns 64 HALF .. 64 HALF + 63: pairs c = 32 HALF .. 32 HALF + 31
   const uint64_t c2 = f32x2(cl2, cl2);
   const uint64_t nm2 = f32x2(-m, -m);
   uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
 #pragma unroll
-  for (int c = 0; c < 64; ++c) {
+  for (int cc = 0; cc < 32; ++cc) {
+    const int c = 32 * HALF + cc;
     const float s0 = __uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]);
     const float s1 = __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
     const uint64_t x2 = fma_f32x2(f32x2(s0, s1), c2, nm2);
@@ -623,7 +625,7 @@ __device__ __forceinline__ float exp_row(const uint32_t (&s)[4][32], float cl2,
     acc[c & 1] = add_f32x2(acc[c & 1], p2);
     float p0, p1;
     f32x2_split(p2, p0, p1);
-    pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+    pk[cc] = pack_bf16x2(p0, p1);
   }
   float a0, a1, b0, b1;
   f32x2_split(acc[0], a0, a1);
@@ -740,9 +742,11 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
         row_sum = exp_row_fp8(s, c, m_run - 8.f, pk);
         tmem_st_32x32b_x32(tS + 0, pk);
       } else {
+        // the first half's P is stored while the second half is computed
         uint32_t pk[2][32];
-        row_sum = exp_row<D>(s, c, m_run, pk);
+        row_sum = exp_row<D, 0>(s, c, m_run, pk[0]);
         tmem_st_32x32b_x32(tS + 0, pk[0]);
+        row_sum += exp_row<D, 1>(s, c, m_run, pk[1]);
         tmem_st_32x32b_x32(tS + 32, pk[1]);
       }
       l_run += row_sum;
