@@ -34,7 +34,7 @@ struct DeviceState {
   uint32_t *status = nullptr;  // 4-byte device status word, lazily allocated
   bool smem_attr_set[6] = {false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
-  bool dec_attr_set[4] = {false, false, false, false};
+  bool dec_attr_set[2] = {false, false};  // decode kernel, d = 128 / 64
 };
 
 std::mutex g_mu;
@@ -889,7 +889,7 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
     p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.timeout_ns = g_timeout_ns.load();
     p.debug_flags = q0 == 0 ? g_inject.load() : 0u;
-    rc = d == 128 ? launch_decode<128, 4>(*st, 0, p, s) : launch_decode<64, 4>(*st, 2, p, s);
+    rc = d == 128 ? launch_decode<128, 4>(*st, 0, p, s) : launch_decode<64, 4>(*st, 1, p, s);
     if (rc != ATTN_OK) return rc;
   }
   return ATTN_OK;
