@@ -297,6 +297,12 @@ def _fp8_fns():
         L.attn_fwd_fp8.restype = i
         L.attn_fwd_fp8_workspace_bytes.argtypes = [i, i, i, i]
         L.attn_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
+        L.attn_fwd_fp8_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i,
+                                        ctypes.c_float, i, u64, u64, vp,
+                                        ctypes.c_size_t, vp]
+        L.attn_fwd_fp8_host.restype = i
+        L.attn_fwd_fp8_host_workspace_bytes.argtypes = [i, i, i, i]
+        L.attn_fwd_fp8_host_workspace_bytes.restype = ctypes.c_size_t
     return L
 
 
@@ -416,6 +422,31 @@ def attn_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None,
                           _stream_handle(stream))
     _check(rc, "attn_fwd_fp8")
     return out, lse
+
+
+def fp8_host_workspace_bytes(B, H, N, d) -> int:
+    return int(_fp8_fns().attn_fwd_fp8_host_workspace_bytes(B, H, N, d))
+
+
+def attn_fwd_fp8_host(q, k, v, out, lse, causal: bool, scale: float, workspace,
+                      signs=None, stream=None):
+    """attn_fwd_fp8 end to end on host (ideally pinned) bf16 tensors
+    [B, H, N, 128]: copies in, rotation and quantization, the FP8 kernel and
+    copies out, overlapped by head chunks; `workspace` is a CUDA uint8
+    tensor of at least ``fp8_host_workspace_bytes`` bytes.  Queued on
+    `stream`; synchronise before reading `out` / `lse`."""
+    import torch
+    _expect_qkv(q, k, v, cuda=False)
+    B, H, N, d = q.shape
+    _expect("out", out, torch.bfloat16, q.shape, cuda=False)
+    _expect("lse", lse, torch.float32, (B, H, N), cuda=False)
+    _expect("workspace", workspace, torch.uint8)
+    lo, hi = sign_mask(signs) if signs is not None else (0, 0)
+    rc = _fp8_fns().attn_fwd_fp8_host(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+        B, H, N, d, int(bool(causal)), float(scale), int(signs is not None), lo, hi,
+        workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    _check(rc, "attn_fwd_fp8_host")
 
 
 # ------------------------------------------------------------------ decode

@@ -375,6 +375,88 @@ __global__ void exp2_selftest_kernel(const float *x, float *y, int n, int mode) 
   if (i + 1 < n) y[i + 1] = y1;
 }
 
+// Head chunks of the host-buffer entries.  The step ends with the last
+// chunk's kernel and copies out, after all copies in, so the chunks shrink
+// towards the end (for 32 heads: 6, 6, 6, 6, 4, 2, 1, 1) and little work is
+// left once the last copy in lands; compute (a few ms) stays well behind the
+// copies in.  Problems below 32 MiB per tensor run as one chunk.
+int host_chunks(int bh, size_t tensor_bytes, int (&sizes)[kHostChunks]) {
+  sizes[0] = bh;
+  if (tensor_bytes < (32u << 20) || bh <= 1) return 1;
+  if (bh <= kHostChunks) {
+    for (int c = 0; c < bh; ++c) sizes[c] = 1;
+    return bh;
+  }
+  const int tail[4] = {bh / 8 > 0 ? bh / 8 : 1, bh / 16 > 0 ? bh / 16 : 1,
+                       bh / 32 > 0 ? bh / 32 : 1, bh / 32 > 0 ? bh / 32 : 1};
+  const int head = bh - (tail[0] + tail[1] + tail[2] + tail[3]);
+  for (int c = 0; c < 4; ++c) sizes[c] = head / 4 + (c < head % 4 ? 1 : 0);
+  for (int c = 0; c < 4; ++c) sizes[4 + c] = tail[c];
+  return kHostChunks;
+}
+
+// The largest head chunk host_chunks gives for B*H heads of N x d.
+int host_max_chunk(int bh, int N, int d) {
+  int sizes[kHostChunks];
+  const int nc = host_chunks(bh, static_cast<size_t>(bh) * N * d * 2, sizes);
+  int m = 0;
+  for (int c = 0; c < nc; ++c) m = sizes[c] > m ? sizes[c] : m;
+  return m;
+}
+
+// The copy / compute pipeline shared by the host-buffer entries: chunk i's
+// copies in (host -> staging), its computation `chunk(h0, nh, comp stream)`
+// and its copies out run on three library-owned streams, so that they
+// overlap chunk i+1's copies in and chunk i-1's copies out.  `stream`
+// orders the whole call: the streams start after its earlier work and it
+// waits for the last copy out.  Staging: dq, dk, dv, dout [bh, N, d] bf16
+// and dl [bh, N] fp32 in device memory.
+template <typename ChunkFn>
+int run_host_pipeline(const void *q, const void *k, const void *v, void *o, float *lse,
+                      int bh, int N, int d, uint8_t *dq, uint8_t *dk, uint8_t *dv,
+                      uint8_t *dout, float *dl, cudaStream_t s, ChunkFn chunk) {
+  int rc, dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  HostPipe *hp = nullptr;
+  if ((rc = host_pipe(dev, &hp)) != ATTN_OK) return rc;
+  int sizes[kHostChunks];
+  const int nchunks = host_chunks(bh, static_cast<size_t>(bh) * N * d * 2, sizes);
+  std::lock_guard<std::mutex> lk(hp->mu);
+  auto fail = [] { cudaGetLastError(); return ATTN_ERR_CUDA; };
+  if (cudaEventRecord(hp->start, s) != cudaSuccess) return fail();
+  for (cudaStream_t t : {hp->h2d, hp->comp, hp->d2h})
+    if (cudaStreamWaitEvent(t, hp->start, 0) != cudaSuccess) return fail();
+  for (int c = 0, h0 = 0; c < nchunks; h0 += sizes[c], ++c) {
+    const int nh = sizes[c];
+    if (nh <= 0) continue;
+    const size_t off = static_cast<size_t>(h0) * N * d * 2;
+    const size_t len = static_cast<size_t>(nh) * N * d * 2;
+    const size_t loff = static_cast<size_t>(h0) * N, llen = static_cast<size_t>(nh) * N;
+    const uint8_t *hq = static_cast<const uint8_t *>(q), *hk = static_cast<const uint8_t *>(k),
+                  *hv = static_cast<const uint8_t *>(v);
+    if (cudaMemcpyAsync(dq + off, hq + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dk + off, hk + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaMemcpyAsync(dv + off, hv + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+        cudaEventRecord(hp->in_done[c], hp->h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->comp, hp->in_done[c], 0) != cudaSuccess)
+      return fail();
+    rc = chunk(h0, nh, reinterpret_cast<attn_stream_t>(hp->comp));
+    if (rc != ATTN_OK) return rc;
+    if (cudaEventRecord(hp->k_done[c], hp->comp) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->d2h, hp->k_done[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t *>(o) + off, dout + off, len,
+                        cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess ||
+        cudaMemcpyAsync(lse + loff, dl + loff, llen * 4, cudaMemcpyDeviceToHost,
+                        hp->d2h) != cudaSuccess)
+      return fail();
+  }
+  if (cudaEventRecord(hp->end, hp->d2h) != cudaSuccess ||
+      cudaStreamWaitEvent(s, hp->end, 0) != cudaSuccess)
+    return fail();
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -497,74 +579,17 @@ int attn_fwd_host(const void *q, const void *k, const void *v, void *o,
     return ATTN_ERR_WORKSPACE;
   const int bh = B * H;
   const size_t rows = static_cast<size_t>(bh) * N;
-  const size_t tb = rows * d * 2, tbr = round256(tb);
+  const size_t tbr = round256(rows * d * 2);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   uint8_t *dq = ws, *dk = ws + tbr, *dv = ws + 2 * tbr, *dout = ws + 3 * tbr;
   float *dl = reinterpret_cast<float *>(ws + 4 * tbr);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int dev;
-  DeviceState *st;
-  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
-  HostPipe *hp = nullptr;
-  if ((rc = host_pipe(dev, &hp)) != ATTN_OK) return rc;
-  // Heads are split into chunks; chunk i's copies in, kernel and copies out
-  // run on three streams so that they overlap chunk i+1's copies in and
-  // chunk i-1's copies out.  `stream` orders the whole call: the streams
-  // start after its earlier work and it waits for the last copy out.
-  // The step ends with the last chunk's kernel and copies out, after all
-  // copies in; the chunks therefore shrink towards the end (for 32 heads:
-  // 6, 6, 6, 6, 4, 2, 1, 1), so that little work is left once the last
-  // copy in lands.  Compute (a few ms) stays well behind the copies in.
-  int sizes[kHostChunks];
-  int nchunks = 1;
-  sizes[0] = bh;
-  if (tb >= (32u << 20) && bh > 1) {
-    if (bh <= kHostChunks) {
-      nchunks = bh;
-      for (int c = 0; c < nchunks; ++c) sizes[c] = 1;
-    } else {
-      const int tail[4] = {bh / 8 > 0 ? bh / 8 : 1, bh / 16 > 0 ? bh / 16 : 1,
-                           bh / 32 > 0 ? bh / 32 : 1, bh / 32 > 0 ? bh / 32 : 1};
-      const int head = bh - (tail[0] + tail[1] + tail[2] + tail[3]);
-      nchunks = kHostChunks;
-      for (int c = 0; c < 4; ++c) sizes[c] = head / 4 + (c < head % 4 ? 1 : 0);
-      for (int c = 0; c < 4; ++c) sizes[4 + c] = tail[c];
-    }
-  }
-  std::lock_guard<std::mutex> lk(hp->mu);
-  auto fail = [] { cudaGetLastError(); return ATTN_ERR_CUDA; };
-  if (cudaEventRecord(hp->start, s) != cudaSuccess) return fail();
-  for (cudaStream_t t : {hp->h2d, hp->comp, hp->d2h})
-    if (cudaStreamWaitEvent(t, hp->start, 0) != cudaSuccess) return fail();
-  for (int c = 0, h0 = 0; c < nchunks; h0 += sizes[c], ++c) {
-    const int nh = sizes[c];
-    if (nh <= 0) continue;
-    const size_t off = static_cast<size_t>(h0) * N * d * 2;
-    const size_t len = static_cast<size_t>(nh) * N * d * 2;
-    const size_t loff = static_cast<size_t>(h0) * N, llen = static_cast<size_t>(nh) * N;
-    const uint8_t *hq = static_cast<const uint8_t *>(q), *hk = static_cast<const uint8_t *>(k),
-                  *hv = static_cast<const uint8_t *>(v);
-    if (cudaMemcpyAsync(dq + off, hq + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
-        cudaMemcpyAsync(dk + off, hk + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
-        cudaMemcpyAsync(dv + off, hv + off, len, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
-        cudaEventRecord(hp->in_done[c], hp->h2d) != cudaSuccess ||
-        cudaStreamWaitEvent(hp->comp, hp->in_done[c], 0) != cudaSuccess)
-      return fail();
-    rc = attn_fwd(dq + off, dk + off, dv + off, dout + off, dl + loff, 1, nh, N, d, causal,
-                  scale, reinterpret_cast<attn_stream_t>(hp->comp));
-    if (rc != ATTN_OK) return rc;
-    if (cudaEventRecord(hp->k_done[c], hp->comp) != cudaSuccess ||
-        cudaStreamWaitEvent(hp->d2h, hp->k_done[c], 0) != cudaSuccess ||
-        cudaMemcpyAsync(static_cast<uint8_t *>(o) + off, dout + off, len,
-                        cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess ||
-        cudaMemcpyAsync(lse + loff, dl + loff, llen * 4, cudaMemcpyDeviceToHost,
-                        hp->d2h) != cudaSuccess)
-      return fail();
-  }
-  if (cudaEventRecord(hp->end, hp->d2h) != cudaSuccess ||
-      cudaStreamWaitEvent(s, hp->end, 0) != cudaSuccess)
-    return fail();
-  return ATTN_OK;
+  return run_host_pipeline(
+      q, k, v, o, lse, bh, N, d, dq, dk, dv, dout, dl,
+      reinterpret_cast<cudaStream_t>(stream), [&](int h0, int nh, attn_stream_t cs) {
+        const size_t off = static_cast<size_t>(h0) * N * d * 2;
+        return attn_fwd(dq + off, dk + off, dv + off, dout + off,
+                        dl + static_cast<size_t>(h0) * N, 1, nh, N, d, causal, scale, cs);
+      });
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int N) {
@@ -798,6 +823,45 @@ int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
   const float scale_qk = rotate ? scale / static_cast<float>(d) : scale;
   return attn_fwd_fp8_quantized(q8, qs, k8, ks, v8, vs, o, lse, B, H, N, d, causal,
                                 scale_qk, stream);
+}
+
+size_t attn_fwd_fp8_host_workspace_bytes(int B, int H, int N, int d) {
+  if (check_fp8_sizes(B, H, N, d) != ATTN_OK) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  const int maxc = host_max_chunk(B * H, N, d);
+  return 4 * round256(rows * d * 2) + round256(rows * 4) +
+         attn_fwd_fp8_workspace_bytes(1, maxc > 0 ? maxc : 1, N, d);
+}
+
+int attn_fwd_fp8_host(const void *q, const void *k, const void *v, void *o, float *lse,
+                      int B, int H, int N, int d, int causal, float scale, int rotate,
+                      uint64_t sign_lo, uint64_t sign_hi, void *workspace,
+                      size_t workspace_bytes, attn_stream_t stream) {
+  int rc = check_fp8_sizes(B, H, N, d);
+  if (rc != ATTN_OK) return rc;
+  if ((rc = check_args(q, k, v, o, lse, B, H, N, d, scale, false)) != ATTN_OK) return rc;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  const size_t need = attn_fwd_fp8_host_workspace_bytes(B, H, N, d);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+    return ATTN_ERR_WORKSPACE;
+  const int bh = B * H;
+  const size_t rows = static_cast<size_t>(bh) * N;
+  const size_t tbr = round256(rows * d * 2);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint8_t *dq = ws, *dk = ws + tbr, *dv = ws + 2 * tbr, *dout = ws + 3 * tbr;
+  float *dl = reinterpret_cast<float *>(ws + 4 * tbr);
+  // the FP8 codes and scales of one chunk at a time: chunks run one after
+  // another on the compute stream, so they share this area
+  uint8_t *fws = ws + 4 * tbr + round256(rows * 4);
+  const size_t fneed = need - (4 * tbr + round256(rows * 4));
+  return run_host_pipeline(
+      q, k, v, o, lse, bh, N, d, dq, dk, dv, dout, dl,
+      reinterpret_cast<cudaStream_t>(stream), [&](int h0, int nh, attn_stream_t cs) {
+        const size_t off = static_cast<size_t>(h0) * N * d * 2;
+        return attn_fwd_fp8(dq + off, dk + off, dv + off, dout + off,
+                            dl + static_cast<size_t>(h0) * N, 1, nh, N, d, causal, scale,
+                            rotate, sign_lo, sign_hi, fws, fneed, cs);
+      });
 }
 
 size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d) {

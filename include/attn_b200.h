@@ -319,6 +319,30 @@ int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o,
 size_t attn_fwd_fp8_workspace_bytes(int B, int H, int N, int d);
 
 /*
+ * attn_fwd_fp8_host -- attn_fwd_fp8 on HOST buffers, end to end: the FP8
+ * counterpart of attn_fwd_host.  q, k, v, o (bf16 [B, H, N, 128]) and lse
+ * (fp32 [B, H, N]) are host memory, ideally page-locked; the bf16 inputs are
+ * copied to the device, rotated and quantized there, attended with the FP8
+ * kernel, and O and lse copied back.  Problems of 32 MiB or more per tensor
+ * are split by heads into the same shrinking chunks as attn_fwd_host, whose
+ * copies in, FP8 computation and copies out overlap on the library's three
+ * streams; the result equals attn_fwd_fp8's bit for bit (the block scales
+ * are per head and tile, so splitting by heads changes none of them).
+ * workspace: device memory of at least attn_fwd_fp8_host_workspace_bytes
+ * bytes, 256-byte aligned (bf16 staging of q, k, v, o, lse and the codes and
+ * scales of one chunk).  Queued on `stream` like attn_fwd_host; the host
+ * outputs are valid after `stream` is synchronised.  Errors as
+ * attn_fwd_fp8, plus ATTN_ERR_WORKSPACE.
+ */
+int attn_fwd_fp8_host(const void *q, const void *k, const void *v, void *o, float *lse,
+                      int B, int H, int N, int d, int causal, float scale, int rotate,
+                      uint64_t sign_lo, uint64_t sign_hi, void *workspace,
+                      size_t workspace_bytes, attn_stream_t stream);
+
+/* Workspace bytes attn_fwd_fp8_host needs (0 on bad sizes). */
+size_t attn_fwd_fp8_host_workspace_bytes(int B, int H, int N, int d);
+
+/*
  * attn_decode -- split-KV decode attention: Nq new queries against Nk keys
  * per (batch, head), after the briefgpt.xyz summary page of FlashAttention-2
  * (arXiv 2307.08691), entry "LeanAttention" (the decode phase of long

@@ -161,6 +161,32 @@ def test_fp8_entries_refuse_bad_arguments_without_a_device(attn):
                                  0.125, 1, 0, 0, None, 0, None) == 0
 
 
+def test_fp8_host_entry_refuses_bad_arguments_without_a_device(attn):
+    far = 1 << 40
+    L = attn._fp8_fns()
+    args = [far, 2 * far, 3 * far, 4 * far, 5 * far, 1, 2, 1024, 128, 0, 0.125, 1,
+            0, 0]
+    assert L.attn_fwd_fp8_host(*args, None, 0, None) == 11          # no workspace
+    assert L.attn_fwd_fp8_host(*args, 6 * far, 16, None) == 11      # too small
+    assert L.attn_fwd_fp8_host(*args, 6 * far + 8, 1 << 40, None) == 11  # misaligned
+    assert L.attn_fwd_fp8_host(*(args[:8] + [64] + args[9:]), 6 * far,
+                               1 << 40, None) == 3                  # d != 128
+    assert L.attn_fwd_fp8_host(None, *args[1:], 6 * far, 1 << 40, None) == 1
+    assert L.attn_fwd_fp8_host(None, None, None, None, None, 0, 2, 1024, 128, 0,
+                               0.125, 1, 0, 0, None, 0, None) == 0  # empty
+    # staging for q, k, v, o, lse plus the FP8 scratch of the largest chunk
+    r = lambda x: (x + 255) // 256 * 256
+    B, H, N = 1, 32, 16384          # 32 heads of 4 MiB: chunks 6,6,6,6,4,2,1,1
+    rows = B * H * N
+    assert attn.fp8_host_workspace_bytes(B, H, N, 128) == \
+        4 * r(rows * 128 * 2) + r(rows * 4) + attn.fp8_workspace_bytes(1, 6, N, 128)
+    B, H, N = 1, 2, 64              # small: one chunk of both heads
+    rows = B * H * N
+    assert attn.fp8_host_workspace_bytes(B, H, N, 128) == \
+        4 * r(rows * 128 * 2) + r(rows * 4) + attn.fp8_workspace_bytes(1, 2, N, 128)
+    assert attn.fp8_host_workspace_bytes(1, 1, 16, 64) == 0
+
+
 def test_fp8_workspace_and_sign_mask(attn):
     B, H, N = 2, 3, 300
     r = lambda x: (x + 255) // 256 * 256

@@ -270,3 +270,30 @@ def test_fp8_full_size_sampled_rows(oracle_mod, causal):
         vmax = float(np.abs(oracle_mod.e4m3_decode(z["v8"])).max() * z["vs"].max())
         _compare(o[0, h, rows], lse[0, h, rows], O_ref, l_ref, flip, vmax, w.N,
                  f"{w.name} causal={causal} head {h}")
+
+
+@pytest.mark.parametrize("B,H,N,causal", [(1, 13, 16384, False), (1, 2, 300, True)])
+def test_fp8_host_entry_matches_device_entry(B, H, N, causal):
+    """attn_fwd_fp8_host: copies in, rotation, quantization, the FP8 kernel
+    and copies out.  13 heads of 4 MiB go through the chunked pipeline (a
+    ragged set of head chunks), 2 heads of 300 rows through one chunk.  The
+    block scales are per head and tile, so splitting by heads changes no
+    code: the outputs equal attn_fwd_fp8's bit for bit."""
+    w, q, k, v, signs = _case(B, H, N, causal, seed=70 + H)
+    sl = signs.tolist()
+    o_dev, l_dev = attn.attn_fwd_fp8(q.cuda(), k.cuda(), v.cuda(), causal=causal,
+                                     scale=w.scale, signs=sl)
+    qp, kp, vp = (t.pin_memory() for t in (q, k, v))
+    o_h = torch.empty_like(q).pin_memory()
+    l_h = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
+    ws = torch.empty(attn.fp8_host_workspace_bytes(B, H, N, 128), dtype=torch.uint8,
+                     device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        attn.attn_fwd_fp8_host(qp, kp, vp, o_h, l_h, causal, w.scale, ws, signs=sl,
+                               stream=stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+    done.synchronize()
+    assert attn.status() == 0
+    assert torch.equal(o_h, o_dev.cpu()) and torch.equal(l_h, l_dev.cpu())
