@@ -11,6 +11,8 @@ import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libattn_b200.so")
+# the same library built with the kernels' index checks (ATTN_DEBUG_BOUNDS)
+DEBUG_LIB_PATH = os.path.join(PKG, "libattn_b200_debug.so")
 
 ATTN_OK = 0
 ERROR_NAMES = {
@@ -21,6 +23,7 @@ ERROR_NAMES = {
     9: "ATTN_ERR_TENSOR_MAP", 10: "ATTN_ERR_NOT_DEVICE_MEMORY",
     11: "ATTN_ERR_WORKSPACE", 12: "ATTN_ERR_NOALLOC_TOO_LARGE",
     16: "ATTN_ERR_DEVICE_TIMEOUT",
+    17: "ATTN_ERR_DEVICE_BOUNDS",
 }
 
 _lib = None

@@ -492,7 +492,7 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
   p.num_units = bh * ((N + 255) / 256);
   p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns.load();
-  p.debug_flags = g_inject.load() & 1u;
+  p.debug_flags = g_inject.load() & 5u;  // bits 0 and 2 concern this kernel
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128)
@@ -1054,8 +1054,9 @@ int attn_status(attn_stream_t stream) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
-  return (bits & attn_b200::kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT
-                                            : ATTN_ERR_CUDA;
+  if (bits & attn_b200::kStatusTimeout) return ATTN_ERR_DEVICE_TIMEOUT;
+  if (bits & attn_b200::kStatusBounds) return ATTN_ERR_DEVICE_BOUNDS;
+  return ATTN_ERR_CUDA;
 }
 
 uint32_t attn_last_status_bits(void) { return g_last_bits.load(); }
@@ -1089,6 +1090,7 @@ const char *attn_strerror(int code) {
     case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case ATTN_ERR_NOALLOC_TOO_LARGE: return "problem needs more device scratch than the static ATTN_NOALLOC_SCRATCH_BYTES array of attn_fwd_host_noalloc";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a pipeline wait in the kernel ran out of time; outputs are invalid";
+    case ATTN_ERR_DEVICE_BOUNDS: return "an index check of the debug build failed; the access was skipped and outputs are invalid";
     default: return "unknown error code";
   }
 }
@@ -1097,7 +1099,7 @@ void attn_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs);
 }
 
-void attn_set_fault_injection(uint32_t flags) { g_inject.store(flags & 3u); }
+void attn_set_fault_injection(uint32_t flags) { g_inject.store(flags & 7u); }
 
 }  // extern "C"
 
@@ -1211,7 +1213,7 @@ extern "C" int attn_fwd_host_noalloc(const void *q, const void *k,
   p.num_units = bh * ((N + 255) / 256);
   p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns.load();
-  p.debug_flags = g_inject.load() & 1u;
+  p.debug_flags = g_inject.load() & 5u;  // bits 0 and 2 concern this kernel
   if (d == 128)
     rc = causal ? launch<128, true>(*st, 0, maps, p, s)
                 : launch<128, false>(*st, 1, maps, p, s);

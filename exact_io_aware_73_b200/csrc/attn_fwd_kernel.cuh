@@ -89,6 +89,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 // Device status word bits.
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBounds = 2u;  // debug build: an index check failed
 constexpr uint32_t kRoleProducer = 1u << 8;
 constexpr uint32_t kRoleMma = 1u << 9;
 constexpr uint32_t kRoleSoftmax = 1u << 10;
@@ -241,6 +242,25 @@ template <bool CAUSAL>
 __device__ __forceinline__ int unit_at(int k) {
   const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   return k * g + ((CAUSAL && (k & 1)) ? g - 1 - c : c);
+}
+
+// Index checks of the debug build (compiled with ATTN_DEBUG_BOUNDS): an index
+// the kernel is about to use for a global access must lie in [0, limit);
+// when it does not, the status word is flagged and the caller skips the
+// access.  In release builds the check is absent and always passes.
+#ifdef ATTN_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t limit, uint32_t *status) {
+  if constexpr (kDebugBounds) {
+    if (i < 0 || i >= limit) {
+      atomicOr(status, kStatusBounds);
+      return false;
+    }
+  }
+  return true;
 }
 
 struct WaitCtx {
@@ -767,8 +787,18 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     if (!ok) break;
     tc_fence_after_sync();
     const float inv_l = __frcp_rn(l_run) * v_mul;
-    const bool row_ok = qs + r < p.n;
-    const int64_t grow = static_cast<int64_t>(w.bh) * p.n + qs + r;
+    int64_t grow = static_cast<int64_t>(w.bh) * p.n + qs + r;
+    if constexpr (kDebugBounds) {
+      // injected index error (debug builds only): the first row stored by
+      // CTA 0 points past the output, which the check below must catch
+      if ((p.debug_flags & 4u) && blockIdx.x == 0 && k == 0 && t == 0 && r == 0)
+        grow += static_cast<int64_t>(p.bh) * p.n;
+    }
+    // a row past N is never stored; in the debug build neither is a row
+    // whose unit or global index is out of range
+    const bool row_ok = qs + r < p.n && in_bounds(w.bh, p.bh, p.status) &&
+                        in_bounds(qs, p.n, p.status) &&
+                        in_bounds(grow, static_cast<int64_t>(p.bh) * p.n, p.status);
     // this block's log-sum-exp (natural log)
     const float lse_this = (m_run - (FP8 ? 8.f : 0.f) + lg2_approx(l_run)) * kLn2;
     float lse_out = lse_this;

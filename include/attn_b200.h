@@ -70,9 +70,12 @@ enum {
   ATTN_ERR_WORKSPACE = 11,       /* attn_fwd_host workspace NULL or too small */
   ATTN_ERR_NOALLOC_TOO_LARGE = 12, /* attn_fwd_host_noalloc: problem needs more
                                       than ATTN_NOALLOC_SCRATCH_BYTES */
-  ATTN_ERR_DEVICE_TIMEOUT = 16   /* (attn_status) a pipeline wait in the
+  ATTN_ERR_DEVICE_TIMEOUT = 16,  /* (attn_status) a pipeline wait in the
                                     kernel ran past its time limit; the kernel
                                     stopped early and its outputs are invalid */
+  ATTN_ERR_DEVICE_BOUNDS = 17    /* (attn_status, debug build only) an index
+                                    check in the kernel failed; the access was
+                                    skipped and the outputs are invalid */
 };
 
 /* Size limits (inclusive).  N <= ATTN_MAX_SEQ; B * H <= ATTN_MAX_HEADS. */
@@ -444,7 +447,12 @@ void attn_set_wait_timeout_ns(uint64_t ns);
  * attn_decode launches the first CTA's producer never issues its first K/V
  * tile, so the compute warps' wait runs out.  Either launch then ends with
  * ATTN_ERR_DEVICE_TIMEOUT in attn_status (outputs invalid) and the CUDA
- * context stays usable.  flags = 0 (the default) turns both off; other bits
+ * context stays usable.  Bit 2, honoured only by the debug build
+ * (libattn_b200_debug.so, compiled with ATTN_DEBUG_BOUNDS, whose kernels check
+ * every global row index before they use it): in later attn_fwd launches the
+ * first row that CTA 0 stores gets an index past the output; the check
+ * catches it, the store is skipped and attn_status returns
+ * ATTN_ERR_DEVICE_BOUNDS.  flags = 0 (the default) turns all off; other bits
  * are ignored.
  */
 void attn_set_fault_injection(uint32_t flags);

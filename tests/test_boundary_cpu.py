@@ -49,6 +49,24 @@ def test_library_exports_every_declared_symbol(attn):
         assert hasattr(lib, name), name
 
 
+def test_debug_library_exports_the_same_entry_points(attn):
+    """The debug build (kernels' index checks compiled in) is the same ABI;
+    built here if missing, as the build step does."""
+    from exact_io_aware_73_b200 import build
+    path = build.build(debug=True)
+    assert path == attn.DEBUG_LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", path],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in _declared_functions():
+        assert name in exported, name
+    dbg = ctypes.CDLL(path)
+    dbg.attn_strerror.restype = ctypes.c_char_p
+    dbg.attn_strerror.argtypes = [ctypes.c_int]
+    assert b"index check" in dbg.attn_strerror(17)
+    assert attn.ERROR_NAMES[17] == "ATTN_ERR_DEVICE_BOUNDS"
+
+
 def test_build_targets_sm100a_only():
     from exact_io_aware_73_b200 import build
     f = build.flags()

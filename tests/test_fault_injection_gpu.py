@@ -86,3 +86,71 @@ def test_decode_wait_timeout_is_reported_and_the_context_survives():
     o, lse = attn.attn_decode(q, k, v, causal=True)
     assert attn.status() == 0
     assert torch.equal(o, good) and torch.equal(lse, good_lse)
+
+
+def _debug_lib():
+    """The debug build of the library (kernels' index checks compiled in),
+    loaded beside the release one; each keeps its own device state."""
+    import ctypes
+    import os
+    if not os.path.exists(attn.DEBUG_LIB_PATH):
+        pytest.fail(f"{attn.DEBUG_LIB_PATH} is missing: build it with "
+                    "`python -m exact_io_aware_73_b200.build --debug`")
+    L = ctypes.CDLL(attn.DEBUG_LIB_PATH)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, ctypes.c_float, vp]
+    L.attn_fwd.restype = i
+    L.attn_status.argtypes = [vp]
+    L.attn_status.restype = i
+    L.attn_last_status_bits.restype = ctypes.c_uint32
+    L.attn_set_fault_injection.argtypes = [ctypes.c_uint32]
+    L.attn_set_fault_injection.restype = None
+    return L
+
+
+@pytest.mark.parametrize("d,causal,N", [(128, False, 1000), (64, True, 777)])
+def test_debug_build_checks_indices_without_faulting(d, causal, N):
+    """The debug build computes exactly what the release build does (its
+    checks only read indices), and an index error injected into it (the first
+    row CTA 0 stores points past the output) is caught before the store:
+    attn_status reports ATTN_ERR_DEVICE_BOUNDS, nothing faults, the wrong
+    address is never written, and the next launch is correct."""
+    L = _debug_lib()
+    w = W.shape_case(2, 3, N, d, causal, seed=57)
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    o_rel, l_rel = attn.attn_fwd(q, k, v, causal=causal, scale=w.scale)
+    assert attn.status() == 0
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+
+    def run():
+        return L.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                          lse.data_ptr(), w.B, w.H, w.N, w.d, int(causal), w.scale, s)
+
+    assert run() == 0 and L.attn_status(s) == 0
+    assert torch.equal(o, o_rel) and torch.equal(lse, l_rel)
+    # a guard region after the output: the skipped store must not land there
+    big = torch.zeros(2 * q.numel(), dtype=torch.bfloat16, device="cuda")
+    o = big[: q.numel()].view_as(q)
+    L.attn_set_fault_injection(4)
+    try:
+        assert run() == 0
+        rc = L.attn_status(s)
+    finally:
+        L.attn_set_fault_injection(0)
+    assert rc == 17, attn.strerror(rc)
+    assert L.attn_last_status_bits() & 2
+    assert torch.count_nonzero(big[q.numel():]) == 0
+    # the context is intact and the debug build is exact again
+    o = torch.empty_like(q)
+    assert run() == 0 and L.attn_status(s) == 0
+    assert torch.equal(o, o_rel) and torch.equal(lse, l_rel)
+    # the release build ignores the injection bit
+    attn.set_fault_injection(4)
+    try:
+        o2, l2 = attn.attn_fwd(q, k, v, causal=causal, scale=w.scale)
+        rc = attn.status()
+    finally:
+        attn.set_fault_injection(0)
+    assert rc == 0 and torch.equal(o2, o_rel) and torch.equal(l2, l_rel)
