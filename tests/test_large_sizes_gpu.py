@@ -215,3 +215,30 @@ def test_backward_needles_long(causal):
     assert np.all(dvh[others] == 0.0)
     assert np.all(np.isfinite(dq.float().cpu().numpy()))
     assert np.all(np.isfinite(dk.float().cpu().numpy()))
+
+
+def test_decode_query_groups_at_maximum_key_count():
+    """13 queries (four launches of up to 4, the last ragged) against 2^26
+    keys under the causal mask: query i sees keys up to Nk - 13 + i.  Planted
+    scores 256 (key 0), 384 (key 2^25) and 512 (key Nk - 8, seen by queries
+    5 and later only), so a group's key limit or its query offset being wrong
+    shows in whole rows."""
+    B, H, Nq, Nk, d = 1, 1, 13, 1 << 26, 64
+    q = torch.zeros((B, H, Nq, d), dtype=torch.bfloat16, device="cuda")
+    q[..., 0] = QV
+    k = torch.zeros((B, H, Nk, d), dtype=torch.bfloat16, device="cuda")
+    marks = {0: 32.0, 1 << 25: 48.0, Nk - 8: 64.0}
+    for t, a in marks.items():
+        k[0, 0, t, 0] = a
+    v = _randn_bf16((B, H, Nk, d), 22)
+    o, lse = attn.attn_decode(q, k, v, causal=True, scale=SCALE)
+    assert attn.status() == 0
+    o, lse = o.float().cpu().numpy()[0, 0], lse.cpu().numpy()[0, 0]
+    for i in range(Nq):
+        t = max(tt for tt in marks if tt <= Nk - Nq + i)
+        assert (t == Nk - 8) == (i >= 5)
+        vt = v[0, 0, t].float().cpu().numpy()
+        assert np.all(np.abs(o[i] - vt) <= 2.0 ** -8 * np.abs(vt) + 1e-6), (i, t)
+        assert abs(lse[i] - 8.0 * marks[t]) <= 5e-3, (i, t, lse[i])
+    del k, v
+    torch.cuda.empty_cache()
