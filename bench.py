@@ -48,6 +48,7 @@ CSRC = os.path.join(ROOT, "exact_io_aware_73_b200", "csrc")
 
 KERNEL_SOURCES = ("attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 DECODE_SOURCES = ("attn_decode_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
+DECODE_MMA_SOURCES = ("attn_decode_mma_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 BWD_SOURCES = ("attn_bwd_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 
 
@@ -706,6 +707,11 @@ def run_decode(args):
     peaks, peak_src = load_peaks()
     achieved = kv / (ms_per_step * 1e-3) / 1e9
     algo_bytes = kv + 2 * q.numel() * 2 + lse.numel() * 4
+    # 5..16 queries at d = 128: one tensor-core launch; otherwise one CUDA-core
+    # launch per group of 4 queries
+    mma = w.d == 128 and w.Nq > attn.DECODE_GROUP_Q
+    launches = 1 if mma else -(-w.Nq // attn.DECODE_GROUP_Q)
+    kernel = "attn_decode_mma_kernel" if mma else f"attn_decode_kernel<{w.d}>"
     cb = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         cb = cpu_baseline_decode(w, qkv_host, args.cpu_budget_s)
@@ -727,9 +733,10 @@ def run_decode(args):
                          "frac": achieved / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} HBM copy bandwidth",
                          "traffic": load_traffic(w.name, "traffic_decode_",
-                                                 DECODE_SOURCES),
+                                                 DECODE_MMA_SOURCES if mma
+                                                 else DECODE_SOURCES),
                          "algorithmic_bytes_per_launch": algo_bytes,
-                         "kernel": f"attn_decode_kernel<{w.d}>"},
+                         "kernel": kernel},
             "cpu_baseline": cb,
             "e2e": {"value": kv / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
                     "h2d_bytes_per_step": qh.numel() * 2,
@@ -737,7 +744,7 @@ def run_decode(args):
                     "ms_per_step": e2e_ms, "steps": e2e_steps,
                     "api": "attn.attn_decode with the new queries copied in and "
                            "O / lse copied out; the K/V cache stays on the device"},
-            "gpu_launches": args.steps, "clocks": clk}), flush=True)
+            "gpu_launches": launches * args.steps, "clocks": clk}), flush=True)
     R.finish(world)
     return 0
 

@@ -468,7 +468,9 @@ def _decode_fns():
     return L
 
 
-DECODE_MAX_Q = 16  # served in groups of 4 queries, one launch each
+DECODE_MAX_Q = 16   # queries per (batch, head) and call
+DECODE_GROUP_Q = 4  # the CUDA-core kernel's queries per launch; 5..16 queries
+                    # at d = 128 take one tensor-core launch instead
 
 
 def decode_workspace_bytes(B, H, Nq, Nk, d) -> int:
@@ -489,8 +491,9 @@ def attn_decode_raw(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, ws,
 
 def attn_decode(q, k, v, causal: bool = True, scale: float | None = None,
                 workspace=None, out=None, lse=None, stream=None):
-    """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16,
-    served 4 per launch) against k, v bf16 [B, H, Nk, d]; returns (O bf16,
+    """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16;
+    on the CUDA cores 4 per launch, or all in one tensor-core launch when
+    d = 128 and Nq > 4) against k, v bf16 [B, H, Nk, d]; returns (O bf16,
     lse fp32 [B, H, Nq])."""
     import torch
     _expect("q", q, torch.bfloat16)

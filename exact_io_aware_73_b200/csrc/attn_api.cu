@@ -17,6 +17,7 @@
 #include "attn_bwd_kernel.cuh"
 #include "fp8_quant_kernel.cuh"
 #include "attn_decode_kernel.cuh"
+#include "attn_decode_mma_kernel.cuh"
 #include "attn_merge_kernel.cuh"
 
 namespace {
@@ -35,6 +36,7 @@ struct DeviceState {
   bool smem_attr_set[6] = {false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
   bool dec_attr_set[2] = {false, false};  // decode kernel, d = 128 / 64
+  bool dm_attr_set = false;               // tensor-core decode kernel
 };
 
 std::mutex g_mu;
@@ -158,15 +160,15 @@ int check_args(const void *q, const void *k, const void *v, const void *o,
 }
 
 // [B*H, N, d] bf16 viewed as a 3-D tensor (d innermost); boxes of 64 x 128
-// rows, 128-byte swizzle -- the shared-memory layout the UMMA descriptors in
-// the kernel expect.  Rows beyond N read as zero.
+// rows (or box_rows), 128-byte swizzle -- the shared-memory layout the UMMA
+// descriptors in the kernels expect.  Rows beyond N read as zero.
 int encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *ptr, int bh,
-               int N, int d) {
+               int N, int d, unsigned box_rows = 128) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(bh)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void *>(ptr), dims, strides, box, estr,
@@ -341,6 +343,39 @@ int launch_decode(DeviceState &st, int variant, attn_b200::DecodeParams &p,
     return ATTN_ERR_CUDA;
   }
   kern<<<grid, attn_b200::kDecThreads, L::kBytes, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+// The tensor-core decode: one CTA per SM, an equal share of the key tiles of
+// all heads each (stream-K), the per-head part counters zeroed first.
+int launch_decode_mma(DeviceState &st, const CUtensorMap *maps,
+                      attn_b200::DecodeMmaParams &p, cudaStream_t stream) {
+  using L = attn_b200::DmSmem;
+  auto kern = attn_b200::attn_decode_mma_kernel;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!st.dm_attr_set) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(L::kAlloc)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      st.dm_attr_set = true;
+    }
+  }
+  int ctas = g_decode_max_ctas.load();
+  if (ctas <= 0) ctas = st.sm_count;
+  if (ctas > attn_b200::kDmMaxCtas) ctas = attn_b200::kDmMaxCtas;
+  const int grid0 = p.total < ctas ? p.total : ctas;
+  p.per_cta = (p.total + grid0 - 1) / grid0;
+  const int grid = (p.total + p.per_cta - 1) / p.per_cta;
+  if (cudaMemsetAsync(p.counters, 0, sizeof(int) * static_cast<size_t>(p.bh), stream) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  kern<<<grid, attn_b200::kDmThreads, L::kAlloc, stream>>>(maps[0], maps[1], maps[2], p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
@@ -868,12 +903,14 @@ size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
   if (B < 0 || H < 0 || Nq < 0 || Nq > ATTN_DECODE_MAX_Q || Nk < 0 ||
       (d != 64 && d != 128))
     return 0;
-  // launches serve at most 4 queries per head each and run one after another
-  // on the stream, so they share the partial slots
+  // the CUDA-core launches serve at most 4 queries per head each and run one
+  // after another on the stream, so they share the partial slots; 5..16
+  // queries at d = 128 take one tensor-core launch with all of them
+  static_assert(attn_b200::kDmMaxCtas <= attn_b200::kDecMaxCtas, "slot bound");
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t slots = bh + attn_b200::kDecMaxCtas;
   constexpr int kGroup = attn_b200::kDecMaxQ;  // queries per launch
-  const size_t g = Nq < kGroup ? static_cast<size_t>(Nq) : kGroup;
+  const size_t g = (Nq < kGroup || d == 128) ? static_cast<size_t>(Nq) : kGroup;
   return round256(slots * g * d * 4) + round256(slots * g * 4) + round256(bh * 4);
 }
 
@@ -919,10 +956,41 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
   for (const void *ptr : all)
     if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
   const size_t slots = static_cast<size_t>(bh64) + attn_b200::kDecMaxCtas;
-  constexpr int kGroup = attn_b200::kDecMaxQ;  // queries per launch
-  const size_t g = Nq < kGroup ? static_cast<size_t>(Nq) : kGroup;
+  constexpr int kGroup = attn_b200::kDecMaxQ;  // queries per CUDA-core launch
+  const bool mma = d == 128 && Nq > kGroup;    // one tensor-core launch instead
+  const size_t g = (Nq < kGroup || mma) ? static_cast<size_t>(Nq) : kGroup;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (mma) {
+    EncodeTiledFn enc;
+    if ((rc = get_encode_fn(&enc)) != ATTN_OK) return rc;
+    CUtensorMap maps[3];
+    const int bhi = static_cast<int>(bh64);
+    if ((rc = encode_map(enc, &maps[0], q, bhi, Nq, d, attn_b200::kDmQ)) != ATTN_OK ||
+        (rc = encode_map(enc, &maps[1], k, bhi, Nk, d)) != ATTN_OK ||
+        (rc = encode_map(enc, &maps[2], v, bhi, Nk, d)) != ATTN_OK)
+      return rc;
+    const int64_t nt = (Nk + attn_b200::kDmKeys - 1) / attn_b200::kDmKeys;
+    attn_b200::DecodeMmaParams p;
+    p.o = static_cast<uint16_t *>(o);
+    p.lse = lse;
+    p.part_o = reinterpret_cast<float *>(ws);
+    p.part_lse = reinterpret_cast<float *>(ws + round256(slots * g * d * 4));
+    p.counters = reinterpret_cast<int *>(ws + round256(slots * g * d * 4) +
+                                         round256(slots * g * 4));
+    p.status = st->status;
+    p.bh = bhi;
+    p.nq = Nq;
+    p.nk = Nk;
+    p.ntiles = static_cast<int>(nt);
+    p.total = static_cast<int>(bh64 * nt);
+    p.per_cta = 1;
+    p.causal = causal ? 1 : 0;
+    p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.timeout_ns = g_timeout_ns.load();
+    p.debug_flags = g_inject.load();
+    return launch_decode_mma(*st, maps, p, s);
+  }
   // groups of up to 4 queries, one launch each; under the causal mask a
   // group's last query sees keys 0 .. Nk - Nq + q0 + m - 1, so its launch
   // stops there (same visibility rule with Nk' = that count, Nq' = m)

@@ -204,6 +204,10 @@ DECODE_WORKLOADS = {
     "decode_tradingday_b16h12nq4nk23400d64": DecodeWorkload(
         "decode_tradingday_b16h12nq4nk23400d64", 16, 12, 4, 23400, 64, True,
         seed=2003),
+    # sixteen new positions per sequence at once (a chunk of new queries):
+    # one pass over K/V on the tensor cores serves all sixteen
+    "decode_b4h16nq16nk32768d128": DecodeWorkload(
+        "decode_b4h16nq16nk32768d128", 4, 16, 16, 32768, 128, True, seed=2004),
 }
 
 DECODE_HEADLINE = "decode_b1h8nq1nk262144d128"

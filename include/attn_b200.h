@@ -365,12 +365,17 @@ size_t attn_fwd_fp8_host_workspace_bytes(int B, int H, int N, int d);
  * Outputs and workspace must not overlap the inputs or each other.
  *
  * The key tiles of all heads are split into equal contiguous shares, one per
- * CTA (two CTAs per SM); a head split over several CTAs is combined exactly
- * by the CTA that finishes its last share.  One launch serves up to 4
- * queries per head; more are served in groups of 4 by successive launches
- * (each reads K/V again, up to the last key its group sees).  Queued on
- * `stream`; a wait that runs out of time shows in attn_status (outputs are
- * then invalid).
+ * CTA; a head split over several CTAs is combined exactly by the CTA that
+ * finishes its last share.  Two kernels:
+ *   - Nq <= 4, or d = 64: CUDA cores, two CTAs per SM, up to 4 queries per
+ *     head and launch; more are served in groups of 4 by successive
+ *     launches (each reads K/V again, up to the last key its group sees);
+ *   - 5 <= Nq <= 16 at d = 128: one launch on the tensor cores (S^T = K Q^T
+ *     and O^T = V^T P^T with tcgen05, one CTA per SM), K/V read once.  P is
+ *     rounded to bf16 for the P.V product, as in attn_fwd; the CUDA-core
+ *     kernel keeps it in fp32.
+ * Queued on `stream`; a wait that runs out of time shows in attn_status
+ * (outputs are then invalid).
  */
 #define ATTN_DECODE_MAX_Q 16
 #define ATTN_MAX_DECODE_KEYS (1 << 26)
@@ -379,8 +384,9 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
                 void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /* Workspace bytes attn_decode needs (0 on bad sizes): partial outputs and
- * log-sum-exps of min(Nq, 4) queries for B*H + 1024 parts, and B*H
- * counters, each rounded up to 256 bytes. */
+ * log-sum-exps of g queries for B*H + 1024 parts, and B*H counters, each
+ * rounded up to 256 bytes; g = Nq at d = 128 (one launch serves them all
+ * when Nq > 4), g = min(Nq, 4) at d = 64. */
 size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d);
 
 /* Test hook: cap the number of CTAs attn_decode launches (0 = two per SM),

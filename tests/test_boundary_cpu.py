@@ -247,6 +247,10 @@ def test_decode_entry_refuses_bad_arguments_without_a_device(attn):
         attn.decode_workspace_bytes(B, H, 4, 1000, d)
     assert attn.decode_workspace_bytes(B, H, 3, 1000, d) == \
         r(slots * 3 * d * 4) + r(slots * 3 * 4) + r(B * H * 4)
+    # at d = 128 more than 4 queries take one tensor-core launch that holds
+    # a part for every query
+    assert attn.decode_workspace_bytes(B, H, 13, 1000, 128) == \
+        r(slots * 13 * 128 * 4) + r(slots * 13 * 4) + r(B * H * 4)
 
 
 def test_merge_entries_refuse_bad_arguments_without_a_device(attn):

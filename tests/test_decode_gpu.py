@@ -6,7 +6,11 @@ fp32 scores and probabilities (no bf16 rounding of P); its outputs differ
 from the fp64 oracle on the same bf16 inputs by the bf16 rounding of O
 (2^-9 relative, taken as 2^-8) plus fp32 accumulation over up to Nk keys and
 ex2.approx (bounded here by 2e-3 absolute, far above what is observed); lse
-within 5e-3, the forward's bound.  Every shape runs with the default split (two CTAs
+within 5e-3, the forward's bound.  With 5..16 queries at d = 128 the kernel
+is the tensor-core one, which rounds P to bf16 for the P.V product as the
+forward does while the row sum adds the unrounded p: each weight then moves
+by at most 2^-9 of itself, so O moves by at most 2^-9 max|v| more, which is
+added to the absolute bound (lse is unaffected).  Every shape runs with the default split (two CTAs
 per SM over all key tiles) and with the CTA count forced low and high, so
 that heads split over many CTAs (merged in-kernel) and heads inside one CTA
 (written directly) are both exercised.
@@ -40,12 +44,23 @@ def _ref(oracle_mod, w, q, k, v):
     return oracle_mod.attention_decode(*f, w.causal, w.scale)
 
 
-def _check(got, ref, what):
+def _uses_mma(Nq, d):
+    return d == 128 and Nq > attn.DECODE_GROUP_Q
+
+
+def _o_atol(Nq, d, v):
+    """O_ATOL, plus the bf16 rounding of P where the tensor-core kernel runs."""
+    if not _uses_mma(Nq, d):
+        return O_ATOL
+    return O_ATOL + 2.0 ** -9 * float(v.float().abs().max())
+
+
+def _check(got, ref, what, atol=O_ATOL):
     o, lse = (t.float().cpu().numpy() for t in got)
     O_ref, l_ref = ref
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse)), what
     err = np.abs(o - O_ref)
-    assert np.all(err <= O_RTOL * np.abs(O_ref) + O_ATOL), \
+    assert np.all(err <= O_RTOL * np.abs(O_ref) + atol), \
         f"{what}: O error {err.max():.3e}"
     lerr = np.abs(lse - l_ref).max()
     assert lerr <= LSE_ATOL, f"{what}: lse error {lerr:.3e}"
@@ -54,7 +69,11 @@ def _check(got, ref, what):
 
 SHAPES = [(1, 1, 1, 1, 64), (1, 2, 1, 64, 128), (2, 1, 3, 65, 128),
           (1, 2, 4, 300, 64), (2, 3, 16, 1000, 128), (1, 1, 16, 16, 128),
-          (3, 2, 7, 4097, 64), (1, 4, 1, 20000, 128)]
+          (3, 2, 7, 4097, 64), (1, 4, 1, 20000, 128),
+          # the tensor-core kernel: 5..16 queries at d = 128, ragged and
+          # exact key tiles, one key tile and many
+          (1, 1, 5, 5, 128), (1, 3, 5, 129, 128), (2, 2, 8, 4096, 128),
+          (1, 2, 13, 20000, 128), (3, 1, 12, 128, 128), (1, 1, 16, 300, 128)]
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -68,7 +87,7 @@ def test_decode_parity(oracle_mod, B, H, Nq, Nk, d, causal):
         attn.set_decode_max_ctas(ctas)
         out = attn.attn_decode(qd, kd, vd, causal=causal, scale=w.scale)
         assert attn.status() == 0
-        e = _check(out, ref, f"{w.name} ctas={ctas}")
+        e = _check(out, ref, f"{w.name} ctas={ctas}", _o_atol(Nq, d, v))
     attn.set_decode_max_ctas(0)
     print(w.name, "max|dO| %.2e max|dlse| %.2e" % e)
 
@@ -116,8 +135,35 @@ def test_decode_full_workloads_every_row(oracle_mod, name):
     bits = [oracle_mod.bf16_bits(t) for t in (q, k, v)]
     rows = np.arange(w.B * w.H * w.Nq)
     O_ref, l_ref = oracle_mod.attention_decode_rows_bf16(*bits, w.causal, w.scale, rows)
-    e = _check((o.reshape(-1, w.d), lse.reshape(-1)), (O_ref, l_ref), name)
+    e = _check((o.reshape(-1, w.d), lse.reshape(-1)), (O_ref, l_ref), name,
+               _o_atol(w.Nq, w.d, v))
     print(name, "max|dO| %.2e max|dlse| %.2e" % e)
+
+
+@pytest.mark.parametrize("nq", [4, 16])
+def test_decode_rising_scores_move_the_reference_max(oracle_mod, nq):
+    """Scores that grow along the keys (and differ per query) make the lazy
+    reference maximum move many times inside every head part, and the parts
+    of a head split over many CTAs start from different maxima: the O
+    rescales and the merge are exercised.  16 queries run on the tensor-core
+    kernel, 4 on the CUDA-core one."""
+    B, H, Nk, d = 1, 2, 3000, 128
+    g = torch.Generator().manual_seed(91)
+    q = (torch.randn(B, H, nq, d, generator=g) * 0.1).to(torch.bfloat16)
+    q[..., 0] = torch.linspace(2.0, 6.0, nq).to(torch.bfloat16)
+    k = (torch.randn(B, H, Nk, d, generator=g) * 0.1)
+    k[..., 0] = torch.linspace(0.0, 48.0, Nk)
+    k = k.to(torch.bfloat16)
+    v = torch.randn(B, H, Nk, d, generator=g).to(torch.bfloat16)
+    scale = 1.0 / np.sqrt(d)
+    f = [oracle_mod.bf16_bits_to_f64(oracle_mod.bf16_bits(t)) for t in (q, k, v)]
+    ref = oracle_mod.attention_decode(*f, True, scale)
+    for ctas in (0, 7, 1000):
+        attn.set_decode_max_ctas(ctas)
+        out = attn.attn_decode(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=scale)
+        assert attn.status() == 0
+        _check(out, ref, f"nq={nq} ctas={ctas}", _o_atol(nq, d, v))
+    attn.set_decode_max_ctas(0)
 
 
 def test_decode_argument_errors_on_device():

@@ -62,12 +62,15 @@ def test_wait_timeout_is_reported_and_the_context_survives(d, causal):
     assert (o.float().abs().amax() <= v.float().abs().amax() * 1.01).item()
 
 
-def test_decode_wait_timeout_is_reported_and_the_context_survives():
-    """Decode: CTA 0's producer skips its first K/V tile; its compute warps'
-    bounded wait runs out, they agree to leave without writing, the producer
-    drains what it did copy.  The status reports the timeout, no drain ran
-    out, and the next launch is correct."""
-    w = W.decode_case(1, 8, 2, 20000, 128, True, seed=32)
+@pytest.mark.parametrize("nq", [2, 8])
+def test_decode_wait_timeout_is_reported_and_the_context_survives(nq):
+    """Decode: CTA 0's loader skips its first K/V tile.  With 2 queries (the
+    CUDA-core kernel) its compute warps' bounded wait runs out; with 8 (the
+    tensor-core kernel) the MMA thread's and the softmax warps' waits do.
+    The CTA leaves without writing and the loader drains what it did copy.
+    The status reports the timeout, no drain ran out, and the next launch is
+    correct."""
+    w = W.decode_case(1, 8, nq, 20000, 128, True, seed=32)
     q, k, v = (t.cuda() for t in W.make_decode_qkv(w))
     good, good_lse = attn.attn_decode(q, k, v, causal=True)
     assert attn.status() == 0
@@ -81,7 +84,7 @@ def test_decode_wait_timeout_is_reported_and_the_context_survives():
         attn.set_wait_timeout_ns(0)
     assert rc == 16, attn.strerror(rc)
     bits = attn.last_status_bits()
-    assert bits & 1 and bits & ((1 << 8) | (1 << 10))
+    assert bits & 1 and bits & ((1 << 8) | (1 << 9) | (1 << 10))
     assert not bits & (1 << 12)
     o, lse = attn.attn_decode(q, k, v, causal=True)
     assert attn.status() == 0
