@@ -242,3 +242,28 @@ def test_decode_query_groups_at_maximum_key_count():
         assert abs(lse[i] - 8.0 * marks[t]) <= 5e-3, (i, t, lse[i])
     del k, v
     torch.cuda.empty_cache()
+
+
+def test_decode_tensor_core_queries_at_maximum_key_count():
+    """13 causal queries at d = 128 (one tensor-core launch) against 2^26
+    keys: the same planted scores as the grouped test, so query i's output
+    is the value of the highest planted key it sees, in closed form."""
+    B, H, Nq, Nk, d = 1, 1, 13, 1 << 26, 128
+    q = torch.zeros((B, H, Nq, d), dtype=torch.bfloat16, device="cuda")
+    q[..., 0] = QV
+    k = torch.zeros((B, H, Nk, d), dtype=torch.bfloat16, device="cuda")
+    marks = {0: 32.0, 1 << 25: 48.0, Nk - 8: 64.0}
+    for t, a in marks.items():
+        k[0, 0, t, 0] = a
+    v = _randn_bf16((B, H, Nk, d), 23)
+    o, lse = attn.attn_decode(q, k, v, causal=True, scale=SCALE)
+    assert attn.status() == 0
+    o, lse = o.float().cpu().numpy()[0, 0], lse.cpu().numpy()[0, 0]
+    for i in range(Nq):
+        t = max(tt for tt in marks if tt <= Nk - Nq + i)
+        assert (t == Nk - 8) == (i >= 5)
+        vt = v[0, 0, t].float().cpu().numpy()
+        assert np.all(np.abs(o[i] - vt) <= 2.0 ** -8 * np.abs(vt) + 1e-6), (i, t)
+        assert abs(lse[i] - 8.0 * marks[t]) <= 5e-3, (i, t, lse[i])
+    del k, v
+    torch.cuda.empty_cache()
