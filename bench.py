@@ -707,9 +707,9 @@ def run_decode(args):
     peaks, peak_src = load_peaks()
     achieved = kv / (ms_per_step * 1e-3) / 1e9
     algo_bytes = kv + 2 * q.numel() * 2 + lse.numel() * 4
-    # 5..16 queries at d = 128: one tensor-core launch; otherwise one CUDA-core
-    # launch per group of 4 queries
-    mma = w.d == 128 and w.Nq > attn.DECODE_GROUP_Q
+    # the library's choice: one tensor-core launch for all queries, or one
+    # CUDA-core launch per group of 4
+    mma = attn.decode_kernel_for(w.Nq, w.d) == attn.DECODE_TENSOR_CORES
     launches = 1 if mma else -(-w.Nq // attn.DECODE_GROUP_Q)
     kernel = "attn_decode_mma_kernel" if mma else f"attn_decode_kernel<{w.d}>"
     cb = None

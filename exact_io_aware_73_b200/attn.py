@@ -465,12 +465,16 @@ def _decode_fns():
         L.attn_decode_workspace_bytes.restype = ctypes.c_size_t
         L.attn_set_decode_max_ctas.argtypes = [i]
         L.attn_set_decode_max_ctas.restype = None
+        L.attn_set_decode_kernel.argtypes = [i]
+        L.attn_set_decode_kernel.restype = None
+        L.attn_decode_kernel_for.argtypes = [i, i]
+        L.attn_decode_kernel_for.restype = i
     return L
 
 
 DECODE_MAX_Q = 16   # queries per (batch, head) and call
-DECODE_GROUP_Q = 4  # the CUDA-core kernel's queries per launch; 5..16 queries
-                    # at d = 128 take one tensor-core launch instead
+DECODE_GROUP_Q = 4  # the CUDA-core kernel's queries per launch (the
+                    # tensor-core kernel serves all of them in one)
 
 
 def decode_workspace_bytes(B, H, Nq, Nk, d) -> int:
@@ -478,8 +482,22 @@ def decode_workspace_bytes(B, H, Nq, Nk, d) -> int:
 
 
 def set_decode_max_ctas(n: int) -> None:
-    """Test hook: cap attn_decode's CTA count (0 restores two per SM)."""
+    """Test hook: cap attn_decode's CTA count (0 restores the default)."""
     _decode_fns().attn_set_decode_max_ctas(int(n))
+
+
+DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR_CORES = 0, 1, 2
+
+
+def set_decode_kernel(which: int) -> None:
+    """Test hook: force the CUDA-core (1) or tensor-core (2) decode kernel;
+    0 restores the library's choice."""
+    _decode_fns().attn_set_decode_kernel(int(which))
+
+
+def decode_kernel_for(Nq: int, d: int) -> int:
+    """The decode kernel attn_decode would run: 1 CUDA cores, 2 tensor cores."""
+    return int(_decode_fns().attn_decode_kernel_for(int(Nq), int(d)))
 
 
 def attn_decode_raw(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, ws,
@@ -492,8 +510,8 @@ def attn_decode_raw(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, ws,
 def attn_decode(q, k, v, causal: bool = True, scale: float | None = None,
                 workspace=None, out=None, lse=None, stream=None):
     """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16;
-    on the CUDA cores 4 per launch, or all in one tensor-core launch when
-    d = 128 and Nq > 4) against k, v bf16 [B, H, Nk, d]; returns (O bf16,
+    all in one tensor-core launch at d = 128 and at d = 64 from 4 queries,
+    else on the CUDA cores) against k, v bf16 [B, H, Nk, d]; returns (O bf16,
     lse fp32 [B, H, Nq])."""
     import torch
     _expect("q", q, torch.bfloat16)

@@ -36,7 +36,7 @@ struct DeviceState {
   bool smem_attr_set[6] = {false, false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
   bool dec_attr_set[2] = {false, false};  // decode kernel, d = 128 / 64
-  bool dm_attr_set = false;               // tensor-core decode kernel
+  bool dm_attr_set[2] = {false, false};   // tensor-core decode kernel, d = 128 / 64
 };
 
 std::mutex g_mu;
@@ -45,6 +45,7 @@ std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<uint32_t> g_inject{0};
 std::atomic<uint32_t> g_last_bits{0};
 std::atomic<int> g_decode_max_ctas{0};
+std::atomic<int> g_decode_kernel{0};  // 0 automatic, 1 CUDA cores, 2 tensor cores
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
                                   void *, const cuuint64_t *, const cuuint64_t *,
@@ -347,21 +348,31 @@ int launch_decode(DeviceState &st, int variant, attn_b200::DecodeParams &p,
   return ATTN_OK;
 }
 
+// Which decode kernel serves Nq queries per head at head size d when the
+// caller leaves the choice to the library.  Measured on B200 (both kernels
+// forced, B=16 H=12 Nk=23400): at d = 128 the tensor-core kernel streams
+// K/V faster for every Nq (6481 against 6082 GB/s at one query); at d = 64
+// the CUDA-core kernel wins up to 2 queries (5343 against 4405 GB/s) and
+// loses from 4 (4097 against 4386).
+bool decode_prefers_mma(int Nq, int d) { return d == 128 || Nq >= 4; }
+
 // The tensor-core decode: one CTA per SM, an equal share of the key tiles of
 // all heads each (stream-K), the per-head part counters zeroed first.
+template <int D>
 int launch_decode_mma(DeviceState &st, const CUtensorMap *maps,
                       attn_b200::DecodeMmaParams &p, cudaStream_t stream) {
-  using L = attn_b200::DmSmem;
-  auto kern = attn_b200::attn_decode_mma_kernel;
+  using L = attn_b200::DmSmem<D>;
+  auto kern = attn_b200::attn_decode_mma_kernel<D>;
+  constexpr int variant = D == 128 ? 0 : 1;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!st.dm_attr_set) {
+    if (!st.dm_attr_set[variant]) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(L::kAlloc)) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
       }
-      st.dm_attr_set = true;
+      st.dm_attr_set[variant] = true;
     }
   }
   int ctas = g_decode_max_ctas.load();
@@ -903,14 +914,13 @@ size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d) {
   if (B < 0 || H < 0 || Nq < 0 || Nq > ATTN_DECODE_MAX_Q || Nk < 0 ||
       (d != 64 && d != 128))
     return 0;
-  // the CUDA-core launches serve at most 4 queries per head each and run one
-  // after another on the stream, so they share the partial slots; 5..16
-  // queries at d = 128 take one tensor-core launch with all of them
+  // a tensor-core launch holds a part for every query; the CUDA-core
+  // launches serve at most 4 queries per head each, one after another on the
+  // stream, and reuse the same slots
   static_assert(attn_b200::kDmMaxCtas <= attn_b200::kDecMaxCtas, "slot bound");
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t slots = bh + attn_b200::kDecMaxCtas;
-  constexpr int kGroup = attn_b200::kDecMaxQ;  // queries per launch
-  const size_t g = (Nq < kGroup || d == 128) ? static_cast<size_t>(Nq) : kGroup;
+  const size_t g = static_cast<size_t>(Nq);
   return round256(slots * g * d * 4) + round256(slots * g * 4) + round256(bh * 4);
 }
 
@@ -957,8 +967,9 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
     if (!is_device_memory_of(ptr, dev)) return ATTN_ERR_NOT_DEVICE_MEMORY;
   const size_t slots = static_cast<size_t>(bh64) + attn_b200::kDecMaxCtas;
   constexpr int kGroup = attn_b200::kDecMaxQ;  // queries per CUDA-core launch
-  const bool mma = d == 128 && Nq > kGroup;    // one tensor-core launch instead
-  const size_t g = (Nq < kGroup || mma) ? static_cast<size_t>(Nq) : kGroup;
+  const int choice = g_decode_kernel.load();
+  const bool mma = choice == 2 || (choice == 0 && decode_prefers_mma(Nq, d));
+  const size_t g = static_cast<size_t>(Nq);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (mma) {
@@ -989,7 +1000,8 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
     p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.timeout_ns = g_timeout_ns.load();
     p.debug_flags = g_inject.load();
-    return launch_decode_mma(*st, maps, p, s);
+    return d == 128 ? launch_decode_mma<128>(*st, maps, p, s)
+                    : launch_decode_mma<64>(*st, maps, p, s);
   }
   // groups of up to 4 queries, one launch each; under the causal mask a
   // group's last query sees keys 0 .. Nk - Nq + q0 + m - 1, so its launch
@@ -1028,6 +1040,16 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
 }
 
 void attn_set_decode_max_ctas(int n) { g_decode_max_ctas.store(n > 0 ? n : 0); }
+
+void attn_set_decode_kernel(int which) {
+  g_decode_kernel.store(which == 1 || which == 2 ? which : 0);
+}
+
+int attn_decode_kernel_for(int Nq, int d) {
+  const int choice = g_decode_kernel.load();
+  if (choice != 0) return choice;
+  return decode_prefers_mma(Nq, d) ? 2 : 1;
+}
 
 int attn_merge_fold(float *acc_o, float *acc_lse, const void *part_o,
                     const float *part_lse, int64_t rows, int d, int first,

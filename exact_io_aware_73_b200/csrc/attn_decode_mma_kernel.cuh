@@ -1,12 +1,12 @@
-// attn_decode_mma_kernel.cuh -- multi-query split-KV decode on the tensor
-// cores for B200 (sm_100a), d = 128.
+// attn_decode_mma_kernel.cuh -- split-KV decode on the tensor cores for
+// B200 (sm_100a), d = 64 or 128, up to 16 queries per head.
 //
 // Source: the briefgpt.xyz summary page of FlashAttention-2 (arXiv
 // 2307.08691), entry "LeanAttention": the decode phase of long contexts is
 // computed in parallel over the key/value sequence.  Same result as
 // attn_decode_kernel (exact attention of Nq new queries, the last Nq
 // positions, against Nk keys; causal: query i sees keys 0 .. Nk - Nq + i),
-// for 5 <= Nq <= 16 at d = 128.
+// for Nq <= 16.
 //
 // The CUDA-core decode keeps at most 4 queries in registers and streams K/V
 // once per group of 4.  Here one pass over K/V serves up to 16 queries, and
@@ -27,17 +27,25 @@
 //     memory as a 16 x 128 K-major tile (128-byte swizzle); each thread adds
 //     its key's p to its own part of every query's row sum;
 //   * O^T += V^T P^T: M = d = 128 (the V tile read MN-major), N = 16, K = 128
-//     keys, accumulated in TMEM over the tiles of a head part;
+//     keys, accumulated in TMEM over the tiles of a head part.  At d = 64
+//     the tile's two 64-key halves stand side by side instead: M = 128 holds
+//     the 64 dimensions of the first half's keys and then of the second
+//     half's (the V tile's two halves, 8 KB apart), N = 32 holds P of the
+//     first half's keys for the 16 queries and then of the second half's
+//     (the same 4 KB of P read as 32 rows of 64 keys), K = 64 keys; the
+//     quadrants (dims 0-63, columns 0-15) and (dims 64-127, columns 16-31)
+//     are the two halves' sums, added at the end of the part, and the other
+//     two quadrants are not used;
 //   * at the end of a part the row-sum parts are added, O^T is read back
 //     (thread = dimension, so every query's row is stored coalesced) and
 //     written out, or recorded as a part and merged exactly by the CTA that
 //     finishes the head's last part: lse = log sum_s exp(lse_s),
 //     O = sum_s exp(lse_s - lse) O_s.
 // Work split: stream-K over the key tiles of all heads, an equal share per
-// CTA, one CTA per SM (the three-stage ring of 64 KB K/V tiles fills the
-// shared memory).  Roles: warps 0-3 softmax, warp 4 TMA loader (one lane),
+// CTA, one CTA per SM (the ring of K/V tiles, three stages of 64 KB at
+// d = 128 or six of 32 KB at d = 64, fills the shared memory).  Roles: warps 0-3 softmax, warp 4 TMA loader (one lane),
 // warp 5 MMA issuer (one lane) and TMEM owner.  TMEM: two S^T buffers of 16
-// columns and O^T (16 columns).  The MMA thread issues S^T of tile i + 1
+// columns and O^T (16 columns, or 32 at d = 64).  The MMA thread issues S^T of tile i + 1
 // before O^T of tile i, so the softmax of one tile overlaps the other's P.V.
 // Every wait is bounded; a wait that runs out flags the device status word,
 // the CTA drains its in-flight copies and MMAs, frees its TMEM and leaves
@@ -54,25 +62,27 @@ namespace attn_b200 {
 
 constexpr int kDmQ = 16;        // query columns per head (padded)
 constexpr int kDmKeys = 128;    // keys per tile
-constexpr int kDmD = 128;       // head dimension
 constexpr int kDmSoftmaxThreads = 128;
 constexpr int kDmThreads = kDmSoftmaxThreads + 64;  // + loader warp + MMA warp
 constexpr int kDmLoaderWarp = 4, kDmMmaWarp = 5;
-constexpr uint32_t kDmTmemCols = 64;  // S^T x 2 (16 each), O^T (16)
+constexpr uint32_t kDmTmemCols = 64;  // S^T x 2 (16 each), O^T (16 or 32)
 constexpr int kDmMaxCtas = 1024;      // bound on the grid (workspace sizing)
 constexpr float kDmLazy = 8.f;        // log2 units: p <= 2^8
 
+template <int D>
 struct DmSmem {
+  static constexpr int kSub = D / 64;                     // 128-byte panels per row
   static constexpr uint32_t kPanel = 128 * 128;           // 128 rows x 128 B
-  static constexpr uint32_t kTile = 2 * kPanel;           // a K or V tile (32 KB)
+  static constexpr uint32_t kTile = kSub * kPanel;        // a K or V tile (D x 256 B)
   static constexpr uint32_t kSmallPanel = kDmQ * 128;     // 16 rows x 128 B
-  static constexpr uint32_t kSmall = 2 * kSmallPanel;     // a Q or P tile (4 KB)
-  static constexpr int kStages = 3;
+  static constexpr uint32_t kQTile = kSub * kSmallPanel;  // Q: 16 rows x D
+  static constexpr uint32_t kPTile = 2 * kSmallPanel;     // P: 16 rows x 128 keys (4 KB)
+  static constexpr int kStages = (D == 64) ? 6 : 3;
   static constexpr uint32_t kK = 0;                       // K ring
   static constexpr uint32_t kV = kK + kStages * kTile;    // V ring
   static constexpr uint32_t kQ = kV + kStages * kTile;    // 2 Q buffers
-  static constexpr uint32_t kP = kQ + 2 * kSmall;         // 2 P buffers
-  static constexpr uint32_t kRed = kP + 2 * kSmall;       // [2][4 warps][16] tile maxima
+  static constexpr uint32_t kP = kQ + 2 * kQTile;         // 2 P buffers
+  static constexpr uint32_t kRed = kP + 2 * kPTile;       // [2][4 warps][16] tile maxima
   static constexpr uint32_t kStat = kRed + 2 * 4 * kDmQ * 4;  // [4 warps][16] row sums
   static constexpr uint32_t kBars = kStat + 4 * kDmQ * 4;
   static constexpr int KV_FULL = 0, KV_EMPTY = kStages, Q_FULL = 2 * kStages,
@@ -169,11 +179,12 @@ __device__ __forceinline__ uint32_t sw128_offset(int rows, int row, int col) {
 
 // ------------------------------------------------------------------ loader
 
+template <int D>
 __device__ __forceinline__ void dm_loader(uint32_t base, const CUtensorMap *tq,
                                           const CUtensorMap *tk, const CUtensorMap *tv,
                                           const DecodeMmaParams &p, const WaitCtx &wc,
                                           int g0, int g1) {
-  using L = DmSmem;
+  using L = DmSmem<D>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   int tc = 0, qc = 0;
   bool ok = true;
@@ -187,9 +198,9 @@ __device__ __forceinline__ void dm_loader(uint32_t base, const CUtensorMap *tq,
     const int qb = qc & 1;
     ok = mbar_wait(bar(L::Q_EMPTY + qb), ((qc >> 1) & 1) ^ 1, wc, kRoleProducer);
     if (!ok) break;
-    mbar_arrive_expect_tx(bar(L::Q_FULL + qb), L::kSmall);
-    for (int s = 0; s < 2; ++s)
-      tma_load_3d(base + L::kQ + qb * L::kSmall + s * L::kSmallPanel, tq,
+    mbar_arrive_expect_tx(bar(L::Q_FULL + qb), L::kQTile);
+    for (int s = 0; s < L::kSub; ++s)
+      tma_load_3d(base + L::kQ + qb * L::kQTile + s * L::kSmallPanel, tq,
                   bar(L::Q_FULL + qb), s * 64, 0, h);
     ++qc;
     for (int gg = g; gg < gend; ++gg) {
@@ -203,10 +214,10 @@ __device__ __forceinline__ void dm_loader(uint32_t base, const CUtensorMap *tq,
         continue;
       }
       mbar_arrive_expect_tx(bar(L::KV_FULL + st), 2 * L::kTile);
-      for (int s = 0; s < 2; ++s)
+      for (int s = 0; s < L::kSub; ++s)
         tma_load_3d_hint(base + L::kK + st * L::kTile + s * L::kPanel, tk,
                          bar(L::KV_FULL + st), s * 64, j * kDmKeys, h, pol_kv);
-      for (int s = 0; s < 2; ++s)
+      for (int s = 0; s < L::kSub; ++s)
         tma_load_3d_hint(base + L::kV + st * L::kTile + s * L::kPanel, tv,
                          bar(L::KV_FULL + st), s * 64, j * kDmKeys, h, pol_kv);
       ++tc;
@@ -231,8 +242,9 @@ __device__ __forceinline__ void dm_loader(uint32_t base, const CUtensorMap *tq,
 
 // ------------------------------------------------------------------ MMA
 
-// S^T[128 keys x 16] = K[128 x 128] Q[16 x 128]^T; both K-major, 128-byte
+// S^T[128 keys x 16] = K[128 x D] Q[16 x D]^T; both K-major, 128-byte
 // swizzle; one instruction per 16 dimensions.
+template <int D>
 __device__ __forceinline__ void dm_issue_s(uint32_t d_tmem, uint32_t k_smem,
                                            uint32_t q_smem) {
   constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
@@ -241,37 +253,52 @@ __device__ __forceinline__ void dm_issue_s(uint32_t d_tmem, uint32_t k_smem,
   const uint64_t kd = smem_desc_sw128(k_smem, 16, 1024);
   const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024);
 #pragma unroll
-  for (int kk = 0; kk < kDmD / 16; ++kk) {
-    const uint64_t ka = ((kk >> 2) * DmSmem::kPanel + (kk & 3) * 32) >> 4;
-    const uint64_t qa = ((kk >> 2) * DmSmem::kSmallPanel + (kk & 3) * 32) >> 4;
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t ka = ((kk >> 2) * DmSmem<D>::kPanel + (kk & 3) * 32) >> 4;
+    const uint64_t qa = ((kk >> 2) * DmSmem<D>::kSmallPanel + (kk & 3) * 32) >> 4;
     mma_bf16_ss(d_tmem, kd + ka, qd + qa, idesc, kk > 0);
   }
 }
 
-// O^T[128 dims x 16] (+)= V^T[128 x 128 keys] P^T[128 keys x 16]: A = the V
-// tile read MN-major (the dimension contiguous; 64-dimension panels
-// kPanel bytes apart, 8-key groups 1024 bytes apart), B = P K-major (16
-// query rows of 128 keys).  One instruction per 16 keys.
+// d = 128: O^T[128 dims x 16] (+)= V^T[128 x 128 keys] P^T[128 keys x 16]:
+// A = the V tile read MN-major (the dimension contiguous; 64-dimension
+// panels kPanel bytes apart, 8-key groups 1024 bytes apart), B = P K-major
+// (16 query rows of 128 keys, two 64-key panels).  One instruction per 16
+// keys.
+// d = 64: O2[128 x 32] (+)= A[128 x 64 keys] B[64 keys x 32] with A rows
+// 0-63 = the dimensions of keys 0-63 and rows 64-127 = those of keys
+// 64-127 (the V tile's two halves, 64 rows x 128 B = 8 KB apart, as the two
+// M panels), B columns 0-15 = P of keys 0-63 and 16-31 = P of keys 64-127
+// (P's two 64-key panels read as one 32-row panel: row 16 + q of the second
+// starts 2 KB after row q of the first and has the same swizzle phase).
+// One instruction per 16 keys of each half.
+template <int D>
 __device__ __forceinline__ void dm_issue_o(uint32_t d_tmem, uint32_t v_smem,
                                            uint32_t p_smem, bool accumulate) {
+  constexpr int kN = (D == 128) ? kDmQ : 2 * kDmQ;
   constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
                              (1u << 15)  // A: MN-major
-                             | ((uint32_t)(kDmQ >> 3) << 17) |
-                             ((uint32_t)(kDmD >> 4) << 24);
-  const uint64_t vd = smem_desc_sw128(v_smem, DmSmem::kPanel, 1024);
+                             | ((uint32_t)(kN >> 3) << 17) |
+                             ((uint32_t)(128 >> 4) << 24);
+  constexpr uint32_t kLbo = (D == 128) ? DmSmem<D>::kPanel : 64 * 128;
+  const uint64_t vd = smem_desc_sw128(v_smem, kLbo, 1024);
   const uint64_t pd = smem_desc_sw128(p_smem, 16, 1024);
+  constexpr int kSteps = (D == 128) ? kDmKeys / 16 : kDmKeys / 32;
 #pragma unroll
-  for (int kk = 0; kk < kDmKeys / 16; ++kk) {
+  for (int kk = 0; kk < kSteps; ++kk) {
     const uint64_t va = static_cast<uint64_t>((kk * 16 * 128) >> 4);
-    const uint64_t pa = ((kk >> 2) * DmSmem::kSmallPanel + (kk & 3) * 32) >> 4;
+    const uint64_t pa = (D == 128)
+        ? (((kk >> 2) * DmSmem<D>::kSmallPanel + (kk & 3) * 32) >> 4)
+        : static_cast<uint64_t>((kk * 32) >> 4);
     mma_bf16_ss(d_tmem, vd + va, pd + pa, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
+template <int D>
 __device__ __forceinline__ void dm_mma(uint32_t base, uint32_t tmem,
                                        const DecodeMmaParams &p, const WaitCtx &wc,
                                        int g0, int g1) {
-  using L = DmSmem;
+  using L = DmSmem<D>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   const uint32_t tO = tmem + 2 * kDmQ;
   int tc = 0, qc = 0;
@@ -283,7 +310,7 @@ __device__ __forceinline__ void dm_mma(uint32_t base, uint32_t tmem,
     if (!mbar_wait_spin(bar(L::P_FULL + pb), (t >> 1) & 1, wc, kRoleMma)) return false;
     tc_fence_after_sync();
     const int st = t % L::kStages;
-    dm_issue_o(tO, base + L::kV + st * L::kTile, base + L::kP + pb * L::kSmall, accumulate);
+    dm_issue_o<D>(tO, base + L::kV + st * L::kTile, base + L::kP + pb * L::kPTile, accumulate);
     mma_commit(bar(L::P_EMPTY + pb));
     mma_commit(bar(L::KV_EMPTY + st));
     return true;
@@ -302,8 +329,8 @@ __device__ __forceinline__ void dm_mma(uint32_t base, uint32_t tmem,
       ok = mbar_wait_spin(bar(L::S_EMPTY + sb), ((tc >> 1) & 1) ^ 1, wc, kRoleMma);
       if (!ok) break;
       tc_fence_after_sync();
-      dm_issue_s(tmem + sb * kDmQ, base + L::kK + st * L::kTile,
-                 base + L::kQ + qb * L::kSmall);
+      dm_issue_s<D>(tmem + sb * kDmQ, base + L::kK + st * L::kTile,
+                    base + L::kQ + qb * L::kQTile);
       mma_commit(bar(L::S_FULL + sb));
       if (i == n - 1) mma_commit(bar(L::Q_EMPTY + qb));  // last read of this Q
       if (i > 0) {
@@ -323,10 +350,11 @@ __device__ __forceinline__ void dm_mma(uint32_t base, uint32_t tmem,
 
 // ------------------------------------------------------------------ softmax
 
+template <int D>
 __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_t tmem,
                                            const DecodeMmaParams &p, const WaitCtx &wc,
                                            int g0, int g1, int warp, int lane) {
-  using L = DmSmem;
+  using L = DmSmem<D>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   const int tid = warp * 32 + lane;  // key of the tile / output dimension
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
@@ -415,7 +443,7 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
       fail = !__all_sync(0xffffffffu, mbar_wait(bar(L::P_EMPTY + pb), ((tc >> 1) & 1) ^ 1,
                                                 wc, kRoleSoftmax));
       if (fail) continue;  // the next barrier takes every thread out
-      uint8_t *pt = smem + L::kP + pb * L::kSmall;
+      uint8_t *pt = smem + L::kP + pb * L::kPTile;
 #pragma unroll
       for (int q = 0; q < kDmQ; ++q) {
         const float pq = (m[q] == -CUDART_INF_F) ? 0.f : ex2_approx(x[q] - m[q]);
@@ -430,12 +458,15 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
                                                   ((tc - 1) >> 1) & 1, wc, kRoleSoftmax));
         if (fail) continue;
         tc_fence_after_sync();
-        uint32_t o[16];
-        tmem_ld_32x32b_x16(tO, o);
-        tmem_wait_ld16(o);
 #pragma unroll
-        for (int q = 0; q < kDmQ; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
-        tmem_st_32x32b_x16(tO, o);
+        for (int c = 0; c < ((D == 128) ? 1 : 2); ++c) {  // column n holds query n % 16
+          uint32_t o[16];
+          tmem_ld_32x32b_x16(tO + c * kDmQ, o);
+          tmem_wait_ld16(o);
+#pragma unroll
+          for (int q = 0; q < kDmQ; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
+          tmem_st_32x32b_x16(tO + c * kDmQ, o);
+        }
         tmem_wait_st();
       }
       tc_fence_before_sync();
@@ -458,8 +489,27 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
     if (!dm_bar_and(!fail)) return;
     uint32_t o[16];
     tc_fence_after_sync();
-    tmem_ld_32x32b_x16(tO, o);
-    tmem_wait_ld16(o);
+    if constexpr (D == 128) {
+      tmem_ld_32x32b_x16(tO, o);  // O^T row `tid` = dimension tid
+      tmem_wait_ld16(o);
+    } else {
+      // dimension t: lane t, columns 0-15 (keys 0-63 of every tile) plus
+      // lane 64 + t, columns 16-31 (keys 64-127); warps 2-3 hand their
+      // quadrant over through the P buffers (free: every P.V is done)
+      tmem_ld_32x32b_x16(tO + (warp >= 2 ? kDmQ : 0), o);
+      tmem_wait_ld16(o);
+      float *xch = reinterpret_cast<float *>(smem + L::kP);  // [16][64]
+      if (warp >= 2) {
+#pragma unroll
+        for (int q = 0; q < kDmQ; ++q) xch[q * 64 + tid - 64] = __uint_as_float(o[q]);
+      }
+      dm_bar_and(true);
+      if (warp < 2) {
+#pragma unroll
+        for (int q = 0; q < kDmQ; ++q)
+          o[q] = __float_as_uint(__uint_as_float(o[q]) + xch[q * 64 + tid]);
+      }
+    }
     const int first = dm_first_cta(h, p), last = dm_last_cta(h, p);
     const bool whole = first == last;
     const int slot = h + static_cast<int>(blockIdx.x);
@@ -471,11 +521,12 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
       const bool any = lsum > 0.f;  // a part may see no key of a causal row
       const float val = any ? __uint_as_float(o[q]) * __frcp_rn(lsum) : 0.f;
       const float lse2 = any ? m[q] + lg2_approx(lsum) : -CUDART_INF_F;  // log2 units
+      if (tid >= D) continue;  // d = 64: warps 2-3 hold no dimension now
       if (whole) {
-        p.o[(row0 + q) * kDmD + tid] = static_cast<uint16_t>(pack_bf16x2(val, 0.f) & 0xFFFFu);
+        p.o[(row0 + q) * D + tid] = static_cast<uint16_t>(pack_bf16x2(val, 0.f) & 0xFFFFu);
         if (tid == q) p.lse[row0 + q] = lse2 * kLn2;
       } else {
-        p.part_o[(static_cast<int64_t>(slot) * p.nq + q) * kDmD + tid] = val;
+        p.part_o[(static_cast<int64_t>(slot) * p.nq + q) * D + tid] = val;
         if (tid == q)
           p.part_lse[static_cast<int64_t>(slot) * p.nq + q] = any ? lse2 * kLn2 : -CUDART_INF_F;
       }
@@ -488,15 +539,17 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
       if (*last_flag) {
         __threadfence();
         // One pass over the head's parts with a running maximum: thread t
-        // combines dimensions 4 (t % 32) .. + 3 of queries t / 32 + 4 r; the
-        // loads of one part (four lse values, four float4) are independent,
-        // so they are in flight together.
+        // combines dimensions 4 (t % C) .. + 3 of queries t / C + G r (C =
+        // D / 4 float4 per row, G = 128 / C query groups, R = 16 / G
+        // queries each); the loads of one part are independent, so they are
+        // in flight together.
+        constexpr int C = D / 4, G = kDmSoftmaxThreads / C, R = kDmQ / G;
         const int nseg = last - first + 1;
-        const int c4 = tid & 31, qg = tid >> 5;
-        float M[4], S[4];
-        float4 A[4];
+        const int c4 = tid % C, qg = tid / C;
+        float M[R], S[R];
+        float4 A[R];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < R; ++r) {
           M[r] = -CUDART_INF_F;
           S[r] = 0.f;
           A[r] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -504,20 +557,20 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
 #pragma unroll 2
         for (int sgi = 0; sgi < nseg; ++sgi) {
           const int64_t slot_row = static_cast<int64_t>(h + first + sgi) * p.nq;
-          float ls[4];
-          float4 po[4];
+          float ls[R];
+          float4 po[R];
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int q = qg + 4 * r;
+          for (int r = 0; r < R; ++r) {
+            const int q = qg + G * r;
             ls[r] = -CUDART_INF_F;
             po[r] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (q < p.nq) {
               ls[r] = __ldcg(p.part_lse + slot_row + q);
-              po[r] = __ldcg(reinterpret_cast<const float4 *>(p.part_o + (slot_row + q) * kDmD) + c4);
+              po[r] = __ldcg(reinterpret_cast<const float4 *>(p.part_o + (slot_row + q) * D) + c4);
             }
           }
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
+          for (int r = 0; r < R; ++r) {
             if (ls[r] == -CUDART_INF_F) continue;  // the part saw no key of the query
             if (ls[r] > M[r]) {
               const float sc = ex2_approx((M[r] - ls[r]) * 1.4426950408889634f);  // 0 at first
@@ -534,11 +587,11 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
           }
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int q = qg + 4 * r;
+        for (int r = 0; r < R; ++r) {
+          const int q = qg + G * r;
           if (q >= p.nq) continue;
           const float inv = __frcp_rn(S[r]);
-          reinterpret_cast<uint2 *>(p.o + (row0 + q) * kDmD)[c4] =
+          reinterpret_cast<uint2 *>(p.o + (row0 + q) * D)[c4] =
               make_uint2(pack_bf16x2(A[r].x * inv, A[r].y * inv),
                          pack_bf16x2(A[r].z * inv, A[r].w * inv));
           if (c4 == 0) p.lse[row0 + q] = M[r] + lg2_approx(S[r]) * kLn2;
@@ -552,12 +605,13 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
 
 // ------------------------------------------------------------------ kernel
 
+template <int D>
 __global__ void __launch_bounds__(kDmThreads, 1)
     attn_decode_mma_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const DecodeMmaParams p) {
-  using L = DmSmem;
+  using L = DmSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -600,12 +654,12 @@ __global__ void __launch_bounds__(kDmThreads, 1)
   const int g0 = blockIdx.x * p.per_cta;
   const int g1 = min(p.total, g0 + p.per_cta);
   if (warp < 4) {
-    dm_softmax(base, smem, tmem, p, wc, g0, g1, warp, lane);
+    dm_softmax<D>(base, smem, tmem, p, wc, g0, g1, warp, lane);
   } else if (warp == kDmLoaderWarp) {
-    if (lane == 0) dm_loader(base, &tm_q, &tm_k, &tm_v, p, wc, g0, g1);
+    if (lane == 0) dm_loader<D>(base, &tm_q, &tm_k, &tm_v, p, wc, g0, g1);
     __syncwarp();
   } else {
-    if (lane == 0) dm_mma(base, tmem, p, wc, g0, g1);
+    if (lane == 0) dm_mma<D>(base, tmem, p, wc, g0, g1);
     __syncwarp();
   }
   tc_fence_before_sync();

@@ -366,14 +366,16 @@ size_t attn_fwd_fp8_host_workspace_bytes(int B, int H, int N, int d);
  *
  * The key tiles of all heads are split into equal contiguous shares, one per
  * CTA; a head split over several CTAs is combined exactly by the CTA that
- * finishes its last share.  Two kernels:
- *   - Nq <= 4, or d = 64: CUDA cores, two CTAs per SM, up to 4 queries per
- *     head and launch; more are served in groups of 4 by successive
- *     launches (each reads K/V again, up to the last key its group sees);
- *   - 5 <= Nq <= 16 at d = 128: one launch on the tensor cores (S^T = K Q^T
- *     and O^T = V^T P^T with tcgen05, one CTA per SM), K/V read once.  P is
- *     rounded to bf16 for the P.V product, as in attn_fwd; the CUDA-core
- *     kernel keeps it in fp32.
+ * finishes its last share.  Two kernels, chosen by Nq and d (see
+ * attn_decode_kernel_for):
+ *   - tensor cores, at d = 128 and at d = 64 from 4 queries: one launch for
+ *     all queries (S^T = K Q^T and O^T = V^T P^T with tcgen05, one CTA per
+ *     SM), K/V read once.  P is rounded to bf16 for the P.V product, as in
+ *     attn_fwd;
+ *   - CUDA cores, at d = 64 up to 3 queries: two CTAs per SM, up to 4
+ *     queries per head and launch (more, when forced by
+ *     attn_set_decode_kernel, in groups of 4 by successive launches, each
+ *     reading K/V again); P stays fp32.
  * Queued on `stream`; a wait that runs out of time shows in attn_status
  * (outputs are then invalid).
  */
@@ -384,14 +386,26 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
                 void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /* Workspace bytes attn_decode needs (0 on bad sizes): partial outputs and
- * log-sum-exps of g queries for B*H + 1024 parts, and B*H counters, each
- * rounded up to 256 bytes; g = Nq at d = 128 (one launch serves them all
- * when Nq > 4), g = min(Nq, 4) at d = 64. */
+ * log-sum-exps of Nq queries for B*H + 1024 parts, and B*H counters, each
+ * rounded up to 256 bytes. */
 size_t attn_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d);
 
-/* Test hook: cap the number of CTAs attn_decode launches (0 = two per SM),
- * so that small problems can be split over many CTAs.  Process-wide. */
+/* Test hook: cap the number of CTAs attn_decode launches (0 = two per SM
+ * for the CUDA-core kernel, one per SM for the tensor-core one), so that
+ * small problems can be split over many CTAs.  Process-wide. */
 void attn_set_decode_max_ctas(int n);
+
+/* Test hook: which decode kernel attn_decode runs, for launches made after
+ * the call (process-wide): 1 = the CUDA-core kernel (groups of 4 queries),
+ * 2 = the tensor-core kernel (one launch for all queries), anything else =
+ * the library's choice by Nq and d (the default).  Both give the same
+ * result up to the bf16 rounding of P in the tensor-core kernel. */
+void attn_set_decode_kernel(int which);
+
+/* The decode kernel attn_decode runs for Nq queries per head at head size d
+ * under the current setting of attn_set_decode_kernel: 1 = CUDA cores,
+ * 2 = tensor cores.  No CUDA calls. */
+int attn_decode_kernel_for(int Nq, int d);
 
 /*
  * Merging partial attention results -- the softmax statistics kept per row

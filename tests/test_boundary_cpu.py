@@ -242,15 +242,10 @@ def test_decode_entry_refuses_bad_arguments_without_a_device(attn):
     slots = B * H + 1024
     assert attn.decode_workspace_bytes(B, H, Nq, 1000, d) == \
         r(slots * Nq * d * 4) + r(slots * Nq * 4) + r(B * H * 4)
-    # queries beyond 4 run as further groups of 4 that reuse the same slots
-    assert attn.decode_workspace_bytes(B, H, 16, 1000, d) == \
-        attn.decode_workspace_bytes(B, H, 4, 1000, d)
-    assert attn.decode_workspace_bytes(B, H, 3, 1000, d) == \
-        r(slots * 3 * d * 4) + r(slots * 3 * 4) + r(B * H * 4)
-    # at d = 128 more than 4 queries take one tensor-core launch that holds
-    # a part for every query
-    assert attn.decode_workspace_bytes(B, H, 13, 1000, 128) == \
-        r(slots * 13 * 128 * 4) + r(slots * 13 * 4) + r(B * H * 4)
+    # a part for every query (the tensor-core kernel serves them in one launch)
+    for nq, dd in ((3, 64), (16, 64), (13, 128)):
+        assert attn.decode_workspace_bytes(B, H, nq, 1000, dd) == \
+            r(slots * nq * dd * 4) + r(slots * nq * 4) + r(B * H * 4)
 
 
 def test_merge_entries_refuse_bad_arguments_without_a_device(attn):

@@ -36,6 +36,7 @@ def _gpu():
     attn.lib()
     yield
     attn.set_decode_max_ctas(0)
+    attn.set_decode_kernel(attn.DECODE_AUTO)
     assert attn.status() == 0
 
 
@@ -44,15 +45,14 @@ def _ref(oracle_mod, w, q, k, v):
     return oracle_mod.attention_decode(*f, w.causal, w.scale)
 
 
-def _uses_mma(Nq, d):
-    return d == 128 and Nq > attn.DECODE_GROUP_Q
-
-
 def _o_atol(Nq, d, v):
     """O_ATOL, plus the bf16 rounding of P where the tensor-core kernel runs."""
-    if not _uses_mma(Nq, d):
+    if attn.decode_kernel_for(Nq, d) != attn.DECODE_TENSOR_CORES:
         return O_ATOL
     return O_ATOL + 2.0 ** -9 * float(v.float().abs().max())
+
+
+KERNELS = (attn.DECODE_CUDA_CORES, attn.DECODE_TENSOR_CORES)
 
 
 def _check(got, ref, what, atol=O_ATOL):
@@ -70,26 +70,34 @@ def _check(got, ref, what, atol=O_ATOL):
 SHAPES = [(1, 1, 1, 1, 64), (1, 2, 1, 64, 128), (2, 1, 3, 65, 128),
           (1, 2, 4, 300, 64), (2, 3, 16, 1000, 128), (1, 1, 16, 16, 128),
           (3, 2, 7, 4097, 64), (1, 4, 1, 20000, 128),
-          # the tensor-core kernel: 5..16 queries at d = 128, ragged and
-          # exact key tiles, one key tile and many
+          # 5..16 queries: ragged and exact key tiles, one key tile and many
           (1, 1, 5, 5, 128), (1, 3, 5, 129, 128), (2, 2, 8, 4096, 128),
-          (1, 2, 13, 20000, 128), (3, 1, 12, 128, 128), (1, 1, 16, 300, 128)]
+          (1, 2, 13, 20000, 128), (3, 1, 12, 128, 128), (1, 1, 16, 300, 128),
+          (2, 2, 16, 3000, 64), (1, 1, 9, 127, 64)]
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("B,H,Nq,Nk,d", SHAPES)
-def test_decode_parity(oracle_mod, B, H, Nq, Nk, d, causal):
+def test_decode_parity(oracle_mod, B, H, Nq, Nk, d, causal, kernel):
+    """Each shape on both kernels (forced), each with the default split, 3
+    CTAs and 1000 CTAs."""
     w = W.decode_case(B, H, Nq, Nk, d, causal, seed=500 + Nk + Nq + d)
     q, k, v = W.make_decode_qkv(w)
     ref = _ref(oracle_mod, w, q, k, v)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
-    for ctas in (0, 3, 1000):
-        attn.set_decode_max_ctas(ctas)
-        out = attn.attn_decode(qd, kd, vd, causal=causal, scale=w.scale)
-        assert attn.status() == 0
-        e = _check(out, ref, f"{w.name} ctas={ctas}", _o_atol(Nq, d, v))
-    attn.set_decode_max_ctas(0)
-    print(w.name, "max|dO| %.2e max|dlse| %.2e" % e)
+    attn.set_decode_kernel(kernel)
+    try:
+        for ctas in (0, 3, 1000):
+            attn.set_decode_max_ctas(ctas)
+            out = attn.attn_decode(qd, kd, vd, causal=causal, scale=w.scale)
+            assert attn.status() == 0
+            e = _check(out, ref, f"{w.name} kernel={kernel} ctas={ctas}",
+                       _o_atol(Nq, d, v))
+    finally:
+        attn.set_decode_max_ctas(0)
+        attn.set_decode_kernel(attn.DECODE_AUTO)
+    print(w.name, kernel, "max|dO| %.2e max|dlse| %.2e" % e)
 
 
 def test_decode_repeated_calls_are_bitwise_equal():
@@ -140,14 +148,14 @@ def test_decode_full_workloads_every_row(oracle_mod, name):
     print(name, "max|dO| %.2e max|dlse| %.2e" % e)
 
 
-@pytest.mark.parametrize("nq", [4, 16])
-def test_decode_rising_scores_move_the_reference_max(oracle_mod, nq):
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("nq,d", [(4, 128), (16, 128), (16, 64)])
+def test_decode_rising_scores_move_the_reference_max(oracle_mod, nq, d, kernel):
     """Scores that grow along the keys (and differ per query) make the lazy
     reference maximum move many times inside every head part, and the parts
     of a head split over many CTAs start from different maxima: the O
-    rescales and the merge are exercised.  16 queries run on the tensor-core
-    kernel, 4 on the CUDA-core one."""
-    B, H, Nk, d = 1, 2, 3000, 128
+    rescales and the merge are exercised, on both kernels."""
+    B, H, Nk = 1, 2, 3000
     g = torch.Generator().manual_seed(91)
     q = (torch.randn(B, H, nq, d, generator=g) * 0.1).to(torch.bfloat16)
     q[..., 0] = torch.linspace(2.0, 6.0, nq).to(torch.bfloat16)
@@ -158,12 +166,16 @@ def test_decode_rising_scores_move_the_reference_max(oracle_mod, nq):
     scale = 1.0 / np.sqrt(d)
     f = [oracle_mod.bf16_bits_to_f64(oracle_mod.bf16_bits(t)) for t in (q, k, v)]
     ref = oracle_mod.attention_decode(*f, True, scale)
-    for ctas in (0, 7, 1000):
-        attn.set_decode_max_ctas(ctas)
-        out = attn.attn_decode(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=scale)
-        assert attn.status() == 0
-        _check(out, ref, f"nq={nq} ctas={ctas}", _o_atol(nq, d, v))
-    attn.set_decode_max_ctas(0)
+    attn.set_decode_kernel(kernel)
+    try:
+        for ctas in (0, 7, 1000):
+            attn.set_decode_max_ctas(ctas)
+            out = attn.attn_decode(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=scale)
+            assert attn.status() == 0
+            _check(out, ref, f"nq={nq} d={d} kernel={kernel} ctas={ctas}", _o_atol(nq, d, v))
+    finally:
+        attn.set_decode_max_ctas(0)
+        attn.set_decode_kernel(attn.DECODE_AUTO)
 
 
 def test_decode_argument_errors_on_device():

@@ -62,33 +62,37 @@ def test_wait_timeout_is_reported_and_the_context_survives(d, causal):
     assert (o.float().abs().amax() <= v.float().abs().amax() * 1.01).item()
 
 
-@pytest.mark.parametrize("nq", [2, 8])
-def test_decode_wait_timeout_is_reported_and_the_context_survives(nq):
-    """Decode: CTA 0's loader skips its first K/V tile.  With 2 queries (the
-    CUDA-core kernel) its compute warps' bounded wait runs out; with 8 (the
-    tensor-core kernel) the MMA thread's and the softmax warps' waits do.
-    The CTA leaves without writing and the loader drains what it did copy.
-    The status reports the timeout, no drain ran out, and the next launch is
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_decode_wait_timeout_is_reported_and_the_context_survives(kernel):
+    """Decode: CTA 0's loader skips its first K/V tile.  On the CUDA-core
+    kernel (1) its compute warps' bounded wait runs out; on the tensor-core
+    kernel (2) the MMA thread's and the softmax warps' waits do.  The CTA
+    leaves without writing and the loader drains what it did copy.  The
+    status reports the timeout, no drain ran out, and the next launch is
     correct."""
-    w = W.decode_case(1, 8, nq, 20000, 128, True, seed=32)
+    w = W.decode_case(1, 8, 6, 20000, 128, True, seed=32)
     q, k, v = (t.cuda() for t in W.make_decode_qkv(w))
-    good, good_lse = attn.attn_decode(q, k, v, causal=True)
-    assert attn.status() == 0
-    attn.set_wait_timeout_ns(50_000_000)
-    attn.set_fault_injection(2)
+    attn.set_decode_kernel(kernel)
     try:
-        attn.attn_decode(q, k, v, causal=True)
-        rc = attn.status()
+        good, good_lse = attn.attn_decode(q, k, v, causal=True)
+        assert attn.status() == 0
+        attn.set_wait_timeout_ns(50_000_000)
+        attn.set_fault_injection(2)
+        try:
+            attn.attn_decode(q, k, v, causal=True)
+            rc = attn.status()
+        finally:
+            attn.set_fault_injection(0)
+            attn.set_wait_timeout_ns(0)
+        assert rc == 16, attn.strerror(rc)
+        bits = attn.last_status_bits()
+        assert bits & 1 and bits & ((1 << 8) | (1 << 9) | (1 << 10))
+        assert not bits & (1 << 12)
+        o, lse = attn.attn_decode(q, k, v, causal=True)
+        assert attn.status() == 0
+        assert torch.equal(o, good) and torch.equal(lse, good_lse)
     finally:
-        attn.set_fault_injection(0)
-        attn.set_wait_timeout_ns(0)
-    assert rc == 16, attn.strerror(rc)
-    bits = attn.last_status_bits()
-    assert bits & 1 and bits & ((1 << 8) | (1 << 9) | (1 << 10))
-    assert not bits & (1 << 12)
-    o, lse = attn.attn_decode(q, k, v, causal=True)
-    assert attn.status() == 0
-    assert torch.equal(o, good) and torch.equal(lse, good_lse)
+        attn.set_decode_kernel(0)
 
 
 def _debug_lib():
