@@ -509,10 +509,10 @@ def attn_decode_raw(q, k, v, o, lse, B, H, Nq, Nk, d, causal, scale, ws,
 
 def attn_decode(q, k, v, causal: bool = True, scale: float | None = None,
                 workspace=None, out=None, lse=None, stream=None):
-    """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16;
-    all in one tensor-core launch at d = 128 and at d = 64 from 4 queries,
-    else on the CUDA cores) against k, v bf16 [B, H, Nk, d]; returns (O bf16,
-    lse fp32 [B, H, Nq])."""
+    """Split-KV decode: q bf16 [B, H, Nq, d] (the last Nq positions, Nq <= 16,
+    all in one tensor-core launch unless set_decode_kernel forces the
+    CUDA-core kernel) against k, v bf16 [B, H, Nk, d]; returns (O bf16, lse
+    fp32 [B, H, Nq])."""
     import torch
     _expect("q", q, torch.bfloat16)
     if q.dim() != 4 or k.dim() != 4:

@@ -350,11 +350,11 @@ int launch_decode(DeviceState &st, int variant, attn_b200::DecodeParams &p,
 
 // Which decode kernel serves Nq queries per head at head size d when the
 // caller leaves the choice to the library.  Measured on B200 (both kernels
-// forced, B=16 H=12 Nk=23400): at d = 128 the tensor-core kernel streams
-// K/V faster for every Nq (6481 against 6082 GB/s at one query); at d = 64
-// the CUDA-core kernel wins up to 2 queries (5343 against 4405 GB/s) and
-// loses from 4 (4097 against 4386).
-bool decode_prefers_mma(int Nq, int d) { return d == 128 || Nq >= 4; }
+// forced, B=16 H=12 Nk=23400, Nq = 1 .. 16): the tensor-core kernel streams
+// K/V faster for every Nq at both head sizes (d = 128: 6412 against 6351
+// GB/s at one query; d = 64: 6121 against 5708 at one query, 6098 against
+// 4097 at four), so it always serves unless a test forces the other.
+bool decode_prefers_mma(int, int) { return true; }
 
 // The tensor-core decode: one CTA per SM, an equal share of the key tiles of
 // all heads each (stream-K), the per-head part counters zeroed first.
@@ -981,7 +981,8 @@ int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse
         (rc = encode_map(enc, &maps[1], k, bhi, Nk, d)) != ATTN_OK ||
         (rc = encode_map(enc, &maps[2], v, bhi, Nk, d)) != ATTN_OK)
       return rc;
-    const int64_t nt = (Nk + attn_b200::kDmKeys - 1) / attn_b200::kDmKeys;
+    const int tile = d == 128 ? attn_b200::DmSmem<128>::kKeys : attn_b200::DmSmem<64>::kKeys;
+    const int64_t nt = (Nk + tile - 1) / tile;
     attn_b200::DecodeMmaParams p;
     p.o = static_cast<uint16_t *>(o);
     p.lse = lse;

@@ -61,23 +61,29 @@
 namespace attn_b200 {
 
 constexpr int kDmQ = 16;        // query columns per head (padded)
-constexpr int kDmKeys = 128;    // keys per tile
+constexpr int kDmBlock = 128;   // keys per S^T MMA (its M)
 constexpr int kDmSoftmaxThreads = 128;
 constexpr int kDmThreads = kDmSoftmaxThreads + 64;  // + loader warp + MMA warp
 constexpr int kDmLoaderWarp = 4, kDmMmaWarp = 5;
-constexpr uint32_t kDmTmemCols = 64;  // S^T x 2 (16 each), O^T (16 or 32)
+constexpr uint32_t kDmTmemCols = 128;  // S^T x 2 (16 or 32 each), O^T (16 or 32)
 constexpr int kDmMaxCtas = 1024;      // bound on the grid (workspace sizing)
 constexpr float kDmLazy = 8.f;        // log2 units: p <= 2^8
 
 template <int D>
 struct DmSmem {
+  // keys per tile: 32 KB of K (and of V) either way, so that the fixed cost
+  // of a tile (waits, barrier, reductions, commits) is spread over as many
+  // bytes at d = 64 as at d = 128
+  static constexpr int kKeys = (D == 64) ? 256 : 128;
+  static constexpr int kBlocks = kKeys / kDmBlock;        // S^T MMAs per tile
   static constexpr int kSub = D / 64;                     // 128-byte panels per row
   static constexpr uint32_t kPanel = 128 * 128;           // 128 rows x 128 B
-  static constexpr uint32_t kTile = kSub * kPanel;        // a K or V tile (D x 256 B)
+  static constexpr uint32_t kTile = kBlocks * kSub * kPanel;  // a K or V tile (32 KB)
   static constexpr uint32_t kSmallPanel = kDmQ * 128;     // 16 rows x 128 B
   static constexpr uint32_t kQTile = kSub * kSmallPanel;  // Q: 16 rows x D
-  static constexpr uint32_t kPTile = 2 * kSmallPanel;     // P: 16 rows x 128 keys (4 KB)
-  static constexpr int kStages = (D == 64) ? 6 : 3;
+  static constexpr uint32_t kPTile = (kKeys / 64) * kSmallPanel;  // P: 16 rows x kKeys
+  static constexpr int kScols = kBlocks * kDmQ;           // TMEM columns of one S^T
+  static constexpr int kStages = 3;
   static constexpr uint32_t kK = 0;                       // K ring
   static constexpr uint32_t kV = kK + kStages * kTile;    // V ring
   static constexpr uint32_t kQ = kV + kStages * kTile;    // 2 Q buffers
@@ -214,12 +220,16 @@ __device__ __forceinline__ void dm_loader(uint32_t base, const CUtensorMap *tq,
         continue;
       }
       mbar_arrive_expect_tx(bar(L::KV_FULL + st), 2 * L::kTile);
-      for (int s = 0; s < L::kSub; ++s)
-        tma_load_3d_hint(base + L::kK + st * L::kTile + s * L::kPanel, tk,
-                         bar(L::KV_FULL + st), s * 64, j * kDmKeys, h, pol_kv);
-      for (int s = 0; s < L::kSub; ++s)
-        tma_load_3d_hint(base + L::kV + st * L::kTile + s * L::kPanel, tv,
-                         bar(L::KV_FULL + st), s * 64, j * kDmKeys, h, pol_kv);
+      // block b (128 keys) of the tile, panel s (64 dimensions)
+      for (int b = 0; b < L::kBlocks; ++b)
+        for (int s = 0; s < L::kSub; ++s) {
+          const uint32_t off = st * L::kTile + (b * L::kSub + s) * L::kPanel;
+          const int row = j * L::kKeys + b * kDmBlock;
+          tma_load_3d_hint(base + L::kK + off, tk, bar(L::KV_FULL + st), s * 64, row, h,
+                           pol_kv);
+          tma_load_3d_hint(base + L::kV + off, tv, bar(L::KV_FULL + st), s * 64, row, h,
+                           pol_kv);
+        }
       ++tc;
     }
     g = gend;
@@ -249,7 +259,7 @@ __device__ __forceinline__ void dm_issue_s(uint32_t d_tmem, uint32_t k_smem,
                                            uint32_t q_smem) {
   constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
                              ((uint32_t)(kDmQ >> 3) << 17) |
-                             ((uint32_t)(kDmKeys >> 4) << 24);
+                             ((uint32_t)(kDmBlock >> 4) << 24);
   const uint64_t kd = smem_desc_sw128(k_smem, 16, 1024);
   const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024);
 #pragma unroll
@@ -283,7 +293,7 @@ __device__ __forceinline__ void dm_issue_o(uint32_t d_tmem, uint32_t v_smem,
   constexpr uint32_t kLbo = (D == 128) ? DmSmem<D>::kPanel : 64 * 128;
   const uint64_t vd = smem_desc_sw128(v_smem, kLbo, 1024);
   const uint64_t pd = smem_desc_sw128(p_smem, 16, 1024);
-  constexpr int kSteps = (D == 128) ? kDmKeys / 16 : kDmKeys / 32;
+  constexpr int kSteps = (D == 128) ? kDmBlock / 16 : kDmBlock / 32;
 #pragma unroll
   for (int kk = 0; kk < kSteps; ++kk) {
     const uint64_t va = static_cast<uint64_t>((kk * 16 * 128) >> 4);
@@ -300,17 +310,21 @@ __device__ __forceinline__ void dm_mma(uint32_t base, uint32_t tmem,
                                        int g0, int g1) {
   using L = DmSmem<D>;
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
-  const uint32_t tO = tmem + 2 * kDmQ;
+  const uint32_t tO = tmem + 2 * L::kScols;
   int tc = 0, qc = 0;
   bool ok = true;
-  // O^T of global tile `t` (the i-th of its part); releases P buffer t & 1
-  // and the tile's K/V stage.
+  // O^T of global tile `t` (the i-th of its part), one MMA group per
+  // 128-key block; releases P buffer t & 1 and the tile's K/V stage.
   auto issue_o = [&](int t, bool accumulate) -> bool {
     const int pb = t & 1;
     if (!mbar_wait_spin(bar(L::P_FULL + pb), (t >> 1) & 1, wc, kRoleMma)) return false;
     tc_fence_after_sync();
     const int st = t % L::kStages;
-    dm_issue_o<D>(tO, base + L::kV + st * L::kTile, base + L::kP + pb * L::kPTile, accumulate);
+#pragma unroll
+    for (int b = 0; b < L::kBlocks; ++b)
+      dm_issue_o<D>(tO, base + L::kV + st * L::kTile + b * L::kSub * L::kPanel,
+                    base + L::kP + pb * L::kPTile + b * 2 * L::kSmallPanel,
+                    accumulate || b > 0);
     mma_commit(bar(L::P_EMPTY + pb));
     mma_commit(bar(L::KV_EMPTY + st));
     return true;
@@ -329,8 +343,11 @@ __device__ __forceinline__ void dm_mma(uint32_t base, uint32_t tmem,
       ok = mbar_wait_spin(bar(L::S_EMPTY + sb), ((tc >> 1) & 1) ^ 1, wc, kRoleMma);
       if (!ok) break;
       tc_fence_after_sync();
-      dm_issue_s<D>(tmem + sb * kDmQ, base + L::kK + st * L::kTile,
-                    base + L::kQ + qb * L::kQTile);
+#pragma unroll
+      for (int b = 0; b < L::kBlocks; ++b)
+        dm_issue_s<D>(tmem + sb * L::kScols + b * kDmQ,
+                      base + L::kK + st * L::kTile + b * L::kSub * L::kPanel,
+                      base + L::kQ + qb * L::kQTile);
       mma_commit(bar(L::S_FULL + sb));
       if (i == n - 1) mma_commit(bar(L::Q_EMPTY + qb));  // last read of this Q
       if (i > 0) {
@@ -358,7 +375,8 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
   auto bar = [&](int i) { return base + L::kBars + 8u * i; };
   const int tid = warp * 32 + lane;  // key of the tile / output dimension
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tO = tmem + lane_base + 2 * kDmQ;
+  const uint32_t tO = tmem + lane_base + 2 * L::kScols;
+  constexpr int KB = L::kBlocks;  // keys of the tile this thread owns: tid + 128 b
   float *red = reinterpret_cast<float *>(smem + L::kRed);
   float *stat = reinterpret_cast<float *>(smem + L::kStat);
   volatile int *last_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 8);
@@ -378,35 +396,47 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
     for (int gg = g; gg < gend; ++gg, ++tc) {
       const int j = gg - h * p.ntiles;
       const int sb = tc & 1;
-      // 1. this key's 16 scores
-      uint32_t sr[16];
+      // 1. the 16 scores of each of this thread's keys
+      uint32_t sr[KB][16];
 #pragma unroll
-      for (int q = 0; q < kDmQ; ++q) sr[q] = 0u;
+      for (int b = 0; b < KB; ++b)
+#pragma unroll
+        for (int q = 0; q < kDmQ; ++q) sr[b][q] = 0u;
       if (!fail)
         fail = !__all_sync(0xffffffffu, mbar_wait(bar(L::S_FULL + sb), (tc >> 1) & 1, wc,
                                                   kRoleSoftmax));
       if (!fail) {
         tc_fence_after_sync();
-        tmem_ld_32x32b_x16(tmem + lane_base + sb * kDmQ, sr);
-        tmem_wait_ld16(sr);
+#pragma unroll
+        for (int b = 0; b < KB; ++b) {
+          tmem_ld_32x32b_x16(tmem + lane_base + sb * L::kScols + b * kDmQ, sr[b]);
+          tmem_wait_ld16(sr[b]);
+        }
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::S_EMPTY + sb));
       }
-      const int key = j * kDmKeys + tid;
-      const bool tail = (j + 1) * kDmKeys > p.nk - (p.causal ? p.nq : 0);  // uniform
-      float x[kDmQ];
+      const int key0 = j * L::kKeys + tid;
+      const bool tail = (j + 1) * L::kKeys > p.nk - (p.causal ? p.nq : 0);  // uniform
+      float x[KB][kDmQ];
 #pragma unroll
-      for (int q = 0; q < kDmQ; ++q) {
-        x[q] = __uint_as_float(sr[q]) * p.c_log2;
-        if (tail && (key >= p.nk || (p.causal && key > p.nk - p.nq + q)))
-          x[q] = -CUDART_INF_F;
+      for (int b = 0; b < KB; ++b) {
+        const int key = key0 + b * kDmBlock;
+#pragma unroll
+        for (int q = 0; q < kDmQ; ++q) {
+          x[b][q] = __uint_as_float(sr[b][q]) * p.c_log2;
+          if (tail && (key >= p.nk || (p.causal && key > p.nk - p.nq + q)))
+            x[b][q] = -CUDART_INF_F;
+        }
       }
-      // 2. per query, the tile's maximum over the 128 keys
+      // 2. per query, the tile's maximum over its keys
       float *rb = red + sb * (4 * kDmQ);
 #pragma unroll
       for (int q = 0; q < kDmQ; ++q) {
-        const float wm = warp_max_f32(x[q]);
+        float xm = x[0][q];
+#pragma unroll
+        for (int b = 1; b < KB; ++b) xm = fmaxf(xm, x[b][q]);
+        const float wm = warp_max_f32(xm);
         if (lane == q) rb[warp * kDmQ + q] = wm;
       }
       if (!dm_bar_and(!fail)) {
@@ -445,12 +475,14 @@ __device__ __forceinline__ void dm_softmax(uint32_t base, uint8_t *smem, uint32_
       if (fail) continue;  // the next barrier takes every thread out
       uint8_t *pt = smem + L::kP + pb * L::kPTile;
 #pragma unroll
-      for (int q = 0; q < kDmQ; ++q) {
-        const float pq = (m[q] == -CUDART_INF_F) ? 0.f : ex2_approx(x[q] - m[q]);
-        l[q] += pq;
-        *reinterpret_cast<uint16_t *>(pt + sw128_offset(kDmQ, q, tid)) =
-            static_cast<uint16_t>(pack_bf16x2(pq, 0.f) & 0xFFFFu);
-      }
+      for (int b = 0; b < KB; ++b)
+#pragma unroll
+        for (int q = 0; q < kDmQ; ++q) {
+          const float pq = (m[q] == -CUDART_INF_F) ? 0.f : ex2_approx(x[b][q] - m[q]);
+          l[q] += pq;
+          *reinterpret_cast<uint16_t *>(pt + sw128_offset(kDmQ, q, tid + b * kDmBlock)) =
+              static_cast<uint16_t>(pack_bf16x2(pq, 0.f) & 0xFFFFu);
+        }
       fence_proxy_async_smem();
       if (rescale) {  // uniform: every thread took the same decision
         // O^T must hold the previous tile's P.V before it is rescaled

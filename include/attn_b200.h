@@ -366,16 +366,13 @@ size_t attn_fwd_fp8_host_workspace_bytes(int B, int H, int N, int d);
  *
  * The key tiles of all heads are split into equal contiguous shares, one per
  * CTA; a head split over several CTAs is combined exactly by the CTA that
- * finishes its last share.  Two kernels, chosen by Nq and d (see
- * attn_decode_kernel_for):
- *   - tensor cores, at d = 128 and at d = 64 from 4 queries: one launch for
- *     all queries (S^T = K Q^T and O^T = V^T P^T with tcgen05, one CTA per
- *     SM), K/V read once.  P is rounded to bf16 for the P.V product, as in
- *     attn_fwd;
- *   - CUDA cores, at d = 64 up to 3 queries: two CTAs per SM, up to 4
- *     queries per head and launch (more, when forced by
- *     attn_set_decode_kernel, in groups of 4 by successive launches, each
- *     reading K/V again); P stays fp32.
+ * finishes its last share.  Two kernels (see attn_decode_kernel_for):
+ *   - tensor cores, the default: one launch for all queries (S^T = K Q^T and
+ *     O^T = V^T P^T with tcgen05, one CTA per SM), K/V read once.  P is
+ *     rounded to bf16 for the P.V product, as in attn_fwd;
+ *   - CUDA cores, when attn_set_decode_kernel(1) asks for it: two CTAs per
+ *     SM, up to 4 queries per head and launch, more in groups of 4 by
+ *     successive launches (each reading K/V again); P stays fp32.
  * Queued on `stream`; a wait that runs out of time shows in attn_status
  * (outputs are then invalid).
  */
