@@ -159,12 +159,22 @@ def test_forward_at_maximum_head_count():
     assert np.abs(got - want).max() <= 5e-3
 
 
+def _decode_with(kernel, *args, **kw):
+    """attn_decode on the given kernel (1 CUDA cores, 2 tensor cores)."""
+    attn.set_decode_kernel(kernel)
+    try:
+        return attn.attn_decode(*args, **kw)
+    finally:
+        attn.set_decode_kernel(0)
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
 @pytest.mark.parametrize("causal", [False, True])
-def test_decode_needles_at_maximum_key_count(causal):
+def test_decode_needles_at_maximum_key_count(causal, kernel):
     """Nk = 2^26 keys (the library's limit), d = 64: K and V are 8.6 GB
     each.  Planted scores 256 (key 0), 384 (key 2^25, a tile boundary) and
     512 (the last key): with the causal mask only the last of the 4 queries
-    sees the last key."""
+    sees the last key.  Both decode kernels."""
     B, H, Nq, Nk, d = 1, 1, 4, 1 << 26, 64
     q = torch.zeros((B, H, Nq, d), dtype=torch.bfloat16, device="cuda")
     q[..., 0] = QV
@@ -173,7 +183,7 @@ def test_decode_needles_at_maximum_key_count(causal):
     for t, a in marks.items():
         k[0, 0, t, 0] = a
     v = _randn_bf16((B, H, Nk, d), 21)
-    o, lse = attn.attn_decode(q, k, v, causal=causal, scale=SCALE)
+    o, lse = _decode_with(kernel, q, k, v, causal=causal, scale=SCALE)
     assert attn.status() == 0
     o, lse = o.float().cpu().numpy()[0, 0], lse.cpu().numpy()[0, 0]
     for i in range(Nq):
@@ -218,8 +228,9 @@ def test_backward_needles_long(causal):
 
 
 def test_decode_query_groups_at_maximum_key_count():
-    """13 queries (four launches of up to 4, the last ragged) against 2^26
-    keys under the causal mask: query i sees keys up to Nk - 13 + i.  Planted
+    """13 queries on the CUDA-core kernel (four launches of up to 4, the last
+    ragged) against 2^26 keys under the causal mask: query i sees keys up to
+    Nk - 13 + i.  Planted
     scores 256 (key 0), 384 (key 2^25) and 512 (key Nk - 8, seen by queries
     5 and later only), so a group's key limit or its query offset being wrong
     shows in whole rows."""
@@ -231,7 +242,7 @@ def test_decode_query_groups_at_maximum_key_count():
     for t, a in marks.items():
         k[0, 0, t, 0] = a
     v = _randn_bf16((B, H, Nk, d), 22)
-    o, lse = attn.attn_decode(q, k, v, causal=True, scale=SCALE)
+    o, lse = _decode_with(1, q, k, v, causal=True, scale=SCALE)
     assert attn.status() == 0
     o, lse = o.float().cpu().numpy()[0, 0], lse.cpu().numpy()[0, 0]
     for i in range(Nq):
@@ -256,7 +267,7 @@ def test_decode_tensor_core_queries_at_maximum_key_count():
     for t, a in marks.items():
         k[0, 0, t, 0] = a
     v = _randn_bf16((B, H, Nk, d), 23)
-    o, lse = attn.attn_decode(q, k, v, causal=True, scale=SCALE)
+    o, lse = _decode_with(2, q, k, v, causal=True, scale=SCALE)
     assert attn.status() == 0
     o, lse = o.float().cpu().numpy()[0, 0], lse.cpu().numpy()[0, 0]
     for i in range(Nq):
