@@ -193,9 +193,11 @@ struct Smem {
   static constexpr uint32_t kV = kK + kKStages * kTileBytes;  // V ring
   static constexpr uint32_t kBars = kV + kVStages * kTileBytes;
   // barrier indices
+  // P_HALF: the first 64 keys of a tile's P are in TMEM (bf16 only);
+  // P_FULL: all of it
   static constexpr int Q_FULL = 0, Q_EMPTY = 2, S_FULL = 4, P_FULL = 6,
-                       O_FULL = 8, O_EMPTY = 10, DRAIN = 12,
-                       K_FULL = 13, K_EMPTY = K_FULL + kKStages,
+                       O_FULL = 8, O_EMPTY = 10, DRAIN = 12, P_HALF = 13,
+                       K_FULL = 15, K_EMPTY = K_FULL + kKStages,
                        V_FULL = K_EMPTY + kKStages, V_EMPTY = V_FULL + kVStages,
                        NUM_BARS = V_EMPTY + kVStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;  // tmem slot, abort
@@ -459,7 +461,7 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem,
   }
 }
 
-template <int D, bool FP8 = false>
+template <int D, bool FP8 = false, int KK0 = 0, int KK1 = kBlockN / (FP8 ? 32 : 16)>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
                                          uint32_t v_smem, bool accumulate) {
   // O[128 x D] (+)= P[128 x 128] V[128 x D]; P in TMEM (K-major: bf16 two per
@@ -475,7 +477,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
   constexpr int kKeys = FP8 ? 32 : 16;
   const uint64_t vd = smem_desc_sw128(v_smem, Smem<D, FP8>::kPanelBytes, 1024);
 #pragma unroll
-  for (int kk = 0; kk < kBlockN / kKeys; ++kk) {
+  for (int kk = KK0; kk < KK1; ++kk) {
     const uint64_t bdesc = vd + static_cast<uint64_t>((kk * kKeys * 128) >> 4);
     if constexpr (FP8)
       mma_f8_ts(d_tmem, p_tmem + kk * 8, bdesc, idesc, (accumulate || kk > 0) ? 1u : 0u);
@@ -529,8 +531,10 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
       bool k_ready = false;
       for (int t = 0; t < 2; ++t) {
         if (j >= nt[t]) continue;
-        ok = mbar_wait_spin(bar(L::P_FULL + t), pcnt[t] & 1, wc, kRoleMma);
-        ++pcnt[t];
+        // bf16: the P.V of the tile's first 64 keys starts while the softmax
+        // still computes the second half's probabilities
+        ok = mbar_wait_spin(bar((FP8 ? L::P_FULL : L::P_HALF) + t), pcnt[t] & 1, wc,
+                            kRoleMma);
         if (!ok) break;
         if (j == 0 && oocc[t] > 0) {
           // previous unit's epilogue must have read O out of TMEM
@@ -538,7 +542,17 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
           if (!ok) break;
         }
         tc_fence_after_sync();
-        issue_pv<D, FP8>(tO[t], tS[t], base + L::kV + vs * L::kTileBytes, j > 0);
+        const uint32_t vt = base + L::kV + vs * L::kTileBytes;
+        if constexpr (FP8) {
+          issue_pv<D, FP8>(tO[t], tS[t], vt, j > 0);
+        } else {
+          issue_pv<D, FP8, 0, 4>(tO[t], tS[t], vt, j > 0);
+          ok = mbar_wait_spin(bar(L::P_FULL + t), pcnt[t] & 1, wc, kRoleMma);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_pv<D, FP8, 4, 8>(tO[t], tS[t], vt, true);
+        }
+        ++pcnt[t];
         mma_commit(bar(L::O_FULL + t));
         if (j + 1 < nt[t]) {
           if (!k_ready) {
@@ -621,15 +635,16 @@ __device__ __forceinline__ float row_max_raw(const uint32_t (&s)[4][32]) {
 // p = 2^(s * scale * log2 e - m) for the whole row: one packed FMA per pair,
 // the exponential on the MUFU unit or (kEmuPer8 pairs in 8) the FMA pipe,
 // packed row sums, bf16x2 packing for the P.V MMA.  Returns the row sum.
-template <int D, int HALF>
+template <int D, int HALF, int CC0 = 0, int CC1 = 32>
 __device__ __forceinline__ float exp_row(const uint32_t (&s)[4][32], float cl2,
                                          float m, uint32_t (&pk)[32]) {
-  // columns 64 HALF .. 64 HALF + 63: pairs c = 32 HALF .. 32 HALF + 31
+  // columns 64 HALF .. 64 HALF + 63: pairs c = 32 HALF .. 32 HALF + 31, of
+  // which this call computes cc in [CC0, CC1) into pk[cc]
   const uint64_t c2 = f32x2(cl2, cl2);
   const uint64_t nm2 = f32x2(-m, -m);
   uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
 #pragma unroll
-  for (int cc = 0; cc < 32; ++cc) {
+  for (int cc = CC0; cc < CC1; ++cc) {
     const int c = 32 * HALF + cc;
     const float s0 = __uint_as_float(s[(2 * c) >> 5][(2 * c) & 31]);
     const float s1 = __uint_as_float(s[(2 * c + 1) >> 5][(2 * c + 1) & 31]);
@@ -762,17 +777,30 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
         row_sum = exp_row_fp8(s, c, m_run - 8.f, pk);
         tmem_st_32x32b_x32(tS + 0, pk);
       } else {
-        // the first half's P is stored while the second half is computed
+        // The first half's P is stored while the second half is computed,
+        // and announced (P_HALF) a quarter of the way through it, so that the
+        // P.V of the first 64 keys overlaps the rest.  O is rescaled before
+        // that announcement: the P.V then adds to the rescaled O.  O holds
+        // the earlier P.V products only; the S_FULL commit for this tile was
+        // issued after the previous P.V, so that MMA has completed.
         uint32_t pk[2][32];
         row_sum = exp_row<D, 0>(s, c, m_run, pk[0]);
         tmem_st_32x32b_x32(tS + 0, pk[0]);
-        row_sum += exp_row<D, 1>(s, c, m_run, pk[1]);
+        if (update) rescale_o<D>(tO, alpha);
+        row_sum += exp_row<D, 1, 0, 8>(s, c, m_run, pk[1]);
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::P_HALF + t));
+        row_sum += exp_row<D, 1, 8, 32>(s, c, m_run, pk[1]);
         tmem_st_32x32b_x32(tS + 32, pk[1]);
       }
       l_run += row_sum;
-      // O holds the earlier P.V products; the S_FULL commit for this tile was
-      // issued after the previous P.V, so that MMA has completed.
-      if (update) rescale_o<D>(tO, alpha);
+      if constexpr (FP8) {
+        // O holds the earlier P.V products; the S_FULL commit for this tile
+        // was issued after the previous P.V, so that MMA has completed.
+        if (update) rescale_o<D>(tO, alpha);
+      }
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
@@ -906,6 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(b0 + 8 * (L::Q_EMPTY + t), 1);
       mbar_init(b0 + 8 * (L::S_FULL + t), 1);
       mbar_init(b0 + 8 * (L::P_FULL + t), 4);
+      mbar_init(b0 + 8 * (L::P_HALF + t), 4);
       mbar_init(b0 + 8 * (L::O_FULL + t), 1);
       mbar_init(b0 + 8 * (L::O_EMPTY + t), 4);
     }
