@@ -274,3 +274,21 @@ def test_fwd_merge_refuses_bad_modes_without_a_device(attn):
     assert f(*(args[:3] + [None] + args[4:]), 2, None) == 1   # accumulator missing
     assert f(*(args[:3] + [4 * far + 8] + args[4:]), 2, None) == 4
     assert f(*(args[:3] + [far + 64] + args[4:]), 2, None) == 6  # acc over q
+
+
+def test_decode_kernel_choice_without_a_device(attn):
+    """The library's decode kernel choice and the test hook that forces one
+    (host logic only, no CUDA call): tensor cores by default at both head
+    sizes, either kernel when forced, the default back for any other value."""
+    try:
+        for nq in (1, 4, 16):
+            for d in (64, 128):
+                assert attn.decode_kernel_for(nq, d) == attn.DECODE_TENSOR_CORES
+        attn.set_decode_kernel(attn.DECODE_CUDA_CORES)
+        assert attn.decode_kernel_for(3, 64) == attn.DECODE_CUDA_CORES
+        attn.set_decode_kernel(attn.DECODE_TENSOR_CORES)
+        assert attn.decode_kernel_for(3, 64) == attn.DECODE_TENSOR_CORES
+        attn.set_decode_kernel(7)  # not a kernel: the library's choice
+        assert attn.decode_kernel_for(3, 64) == attn.DECODE_TENSOR_CORES
+    finally:
+        attn.set_decode_kernel(attn.DECODE_AUTO)
