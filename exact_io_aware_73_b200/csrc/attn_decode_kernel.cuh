@@ -6,6 +6,11 @@
 // attention for Nq <= 16 new queries (the last Nq positions) against Nk keys:
 // with the causal mask query i sees keys 0 .. Nk - Nq + i.
 //
+// attn_decode runs this kernel when attn_set_decode_kernel(1) selects it; by
+// default the tensor-core kernel (attn_decode_mma_kernel.cuh) serves, which
+// streamed K/V faster at every Nq and head size measured.  This one keeps P
+// in fp32 instead of rounding it to bf16 for a P.V product.
+//
 // Decode is a matrix-vector product per (batch, head): every key and value
 // byte is used for a handful of queries, so the bound is HBM bandwidth, not
 // the tensor cores.  One launch serves up to 4 queries per head (their
