@@ -13,43 +13,47 @@
 // both contractions run on tcgen05 with the roles of the operands turned
 // around, so that the M = 128 side of the MMA is the key tile (and the head
 // dimension), never the handful of queries:
-//   * S^T = K Q^T: M = 128 keys of the tile, N = 16 query columns (Q rows
-//     beyond Nq are zero), K = d; A = the K tile and B = Q, both K-major
-//     with the 128-byte swizzle, exactly as the TMA writes them.  Softmax
-//     thread t (warp t / 32 reads TMEM lanes 32 (t / 32) ..) owns key t of
-//     the tile and holds its 16 scores;
-//   * per query, the tile maximum over the 128 keys (a warp max reduction,
-//     then the four warps through shared memory); the reference maximum
-//     moves lazily as in the forward kernel (only when a score exceeds it by
-//     more than 2^8, which every thread decides identically), O^T is then
+//   * a tile is 32 KB of K and 32 KB of V: 128 keys at d = 128, 256 at
+//     d = 64 (so that a tile's fixed cost -- waits, barrier, reductions,
+//     commits -- is spread over as many bytes as at d = 128);
+//   * S^T = K Q^T per 128-key block of the tile: M = 128 keys, N = 16 query
+//     columns (Q rows beyond Nq are zero), K = d; A = the K block and B = Q,
+//     both K-major with the 128-byte swizzle, exactly as the TMA writes
+//     them.  Softmax thread t (warp t / 32 reads TMEM lanes 32 (t / 32) ..)
+//     owns key t of each block and holds its 16 scores per block;
+//   * per query, the tile maximum over its keys (a warp max reduction, then
+//     the four warps through shared memory); the reference maximum moves
+//     lazily as in the forward kernel (only when a score exceeds it by more
+//     than 2^8, which every thread decides identically), O^T is then
 //     rescaled in TMEM;
 //   * p = 2^(s scale log2(e) - m) rounded to bf16 and written to shared
-//     memory as a 16 x 128 K-major tile (128-byte swizzle); each thread adds
-//     its key's p to its own part of every query's row sum;
-//   * O^T += V^T P^T: M = d = 128 (the V tile read MN-major), N = 16, K = 128
-//     keys, accumulated in TMEM over the tiles of a head part.  At d = 64
-//     the tile's two 64-key halves stand side by side instead: M = 128 holds
-//     the 64 dimensions of the first half's keys and then of the second
-//     half's (the V tile's two halves, 8 KB apart), N = 32 holds P of the
-//     first half's keys for the 16 queries and then of the second half's
-//     (the same 4 KB of P read as 32 rows of 64 keys), K = 64 keys; the
-//     quadrants (dims 0-63, columns 0-15) and (dims 64-127, columns 16-31)
-//     are the two halves' sums, added at the end of the part, and the other
-//     two quadrants are not used;
+//     memory as a 16-row K-major tile of the tile's keys (64-key panels,
+//     128-byte swizzle); each thread adds its keys' p to its own part of
+//     every query's row sum;
+//   * O^T += V^T P^T per 128-key block: at d = 128, M = d (the V block read
+//     MN-major), N = 16, K = 128 keys.  At d = 64 the block's two 64-key
+//     halves stand side by side instead: M = 128 holds the 64 dimensions of
+//     the first half's keys and then of the second half's (the V block's
+//     two halves, 8 KB apart), N = 32 holds P of the first half's keys for
+//     the 16 queries and then of the second half's (the block's 4 KB of P
+//     read as 32 rows of 64 keys), K = 64 keys; the quadrants (dims 0-63,
+//     columns 0-15) and (dims 64-127, columns 16-31) are the two halves'
+//     sums, added at the end of the part, and the other two quadrants are
+//     not used.  O^T accumulates in TMEM over the tiles of a head part;
 //   * at the end of a part the row-sum parts are added, O^T is read back
 //     (thread = dimension, so every query's row is stored coalesced) and
 //     written out, or recorded as a part and merged exactly by the CTA that
 //     finishes the head's last part: lse = log sum_s exp(lse_s),
 //     O = sum_s exp(lse_s - lse) O_s.
 // Work split: stream-K over the key tiles of all heads, an equal share per
-// CTA, one CTA per SM (the ring of K/V tiles, three stages of 64 KB at
-// d = 128 or six of 32 KB at d = 64, fills the shared memory).  Roles: warps 0-3 softmax, warp 4 TMA loader (one lane),
-// warp 5 MMA issuer (one lane) and TMEM owner.  TMEM: two S^T buffers of 16
-// columns and O^T (16 columns, or 32 at d = 64).  The MMA thread issues S^T of tile i + 1
-// before O^T of tile i, so the softmax of one tile overlaps the other's P.V.
-// Every wait is bounded; a wait that runs out flags the device status word,
-// the CTA drains its in-flight copies and MMAs, frees its TMEM and leaves
-// without writing.
+// CTA, one CTA per SM (the three-stage ring of 64 KB K/V tiles fills the
+// shared memory).  Roles: warps 0-3 softmax, warp 4 TMA loader (one lane),
+// warp 5 MMA issuer (one lane) and TMEM owner.  TMEM: two S^T buffers (16
+// columns per 128-key block) and O^T (16 columns, or 32 at d = 64).  The MMA
+// thread issues S^T of tile i + 1 before O^T of tile i, so the softmax of one
+// tile overlaps the other's P.V.  Every wait is bounded; a wait that runs
+// out flags the device status word, the CTA drains its in-flight copies and
+// MMAs, frees its TMEM and leaves without writing.
 #pragma once
 
 #include <cstdint>
