@@ -395,8 +395,9 @@ void attn_set_decode_max_ctas(int n);
 /* Test hook: which decode kernel attn_decode runs, for launches made after
  * the call (process-wide): 1 = the CUDA-core kernel (groups of 4 queries),
  * 2 = the tensor-core kernel (one launch for all queries), anything else =
- * the library's choice by Nq and d (the default).  Both give the same
- * result up to the bf16 rounding of P in the tensor-core kernel. */
+ * the library's choice (the default; currently the tensor-core kernel for
+ * every Nq and d).  Both give the same result up to the bf16 rounding of P
+ * in the tensor-core kernel. */
 void attn_set_decode_kernel(int which);
 
 /* The decode kernel attn_decode runs for Nq queries per head at head size d
