@@ -711,7 +711,7 @@ def run_decode(args):
     # CUDA-core launch per group of 4
     mma = attn.decode_kernel_for(w.Nq, w.d) == attn.DECODE_TENSOR_CORES
     launches = 1 if mma else -(-w.Nq // attn.DECODE_GROUP_Q)
-    kernel = "attn_decode_mma_kernel" if mma else f"attn_decode_kernel<{w.d}>"
+    kernel = f"attn_decode_mma_kernel<{w.d}>" if mma else f"attn_decode_kernel<{w.d}>"
     cb = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         cb = cpu_baseline_decode(w, qkv_host, args.cpu_budget_s)
