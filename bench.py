@@ -87,6 +87,32 @@ def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
+# The exponential roof: the softmax evaluates one exp2 per visible score, B H
+# N^2 of them (halved under the causal mask, the FLOP convention's count), on
+# the MUFU unit at 16 per clock per SM.  The d = 64 kernel evaluates a quarter
+# of them on the FMA pipe instead, so its MUFU share is 3/4 of the count.
+MUFU_EX2_PER_CLK_PER_SM = 16
+DEFAULT_SM_MHZ = 1965.0
+
+
+def exp_roof(flops: float, d: int, ms_per_step: float, sm_count: int,
+             sm_mhz) -> dict:
+    """The forward's second roof beside the tensor cores: algorithmic exp2
+    per launch (flops / (4 d)) over the launch time, against the MUFU rate
+    of all SMs at the SM clock sampled during the timed region (the maximum
+    clock when no sample exists)."""
+    mhz = float(sm_mhz) if sm_mhz else DEFAULT_SM_MHZ
+    count = flops / (4.0 * d)
+    achieved = count / (ms_per_step * 1e-3) / 1e9
+    peak = MUFU_EX2_PER_CLK_PER_SM * sm_count * mhz * 1e6 / 1e9
+    return {"unit": "Gexp2/s", "achieved": achieved, "peak": peak,
+            "frac": achieved / peak, "exp2_per_launch": count,
+            "peak_basis": (f"{MUFU_EX2_PER_CLK_PER_SM} ex2 per clock per SM x "
+                           f"{sm_count} SMs x {mhz:.0f} MHz (median SM clock in "
+                           "the timed region)"),
+            "mufu_share": 0.75 if d == 64 else 1.0}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -1013,6 +1039,9 @@ def main():
                        "parallelism": (f"{world} independent replicas (one "
                                        "workload per GPU, no collective)")},
             "roofline": roofline,
+            "exp_roof": exp_roof(flops, w.d, ms_per_step,
+                                 torch.cuda.get_device_properties(dev).multi_processor_count,
+                                 (clk or {}).get("sm_mhz")),
             "cpu_baseline": cb,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

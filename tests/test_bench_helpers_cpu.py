@@ -61,3 +61,18 @@ def test_clock_record_of_a_short_region_takes_the_nearest_samples():
     assert rec["window"].startswith("the region's own samples plus")
     # the last sample before and the first after: 1965 and 1955 (hw_slowdown)
     assert rec["sm_mhz"] == 1960.0 and rec["reasons"] == ["hw_slowdown"]
+
+
+def test_exp_roof_counts_one_exp2_per_visible_score():
+    # the headline's count: 32 heads x 16384^2 scores, one exp2 each
+    flops = 4.0 * 1 * 32 * 16384 ** 2 * 128
+    r = bench.exp_roof(flops, 128, 3.5, 148, 1965.0)
+    assert r["exp2_per_launch"] == 32 * 16384 ** 2
+    assert abs(r["peak"] - 16 * 148 * 1965e6 / 1e9) < 1e-6
+    assert abs(r["achieved"] - 32 * 16384 ** 2 / 3.5e-3 / 1e9) < 1e-3
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+    assert r["mufu_share"] == 1.0
+    # no clock sample: the maximum clock; d = 64 puts a quarter on the FMA pipe
+    r64 = bench.exp_roof(flops / 2, 64, 1.0, 148, None)
+    assert r64["peak"] == r["peak"] and r64["mufu_share"] == 0.75
+    assert r64["exp2_per_launch"] == flops / 2 / 256
