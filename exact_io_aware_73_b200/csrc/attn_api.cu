@@ -47,6 +47,15 @@ std::atomic<uint32_t> g_last_bits{0};
 std::atomic<int> g_decode_max_ctas{0};
 std::atomic<int> g_decode_kernel{0};  // 0 automatic, 1 CUDA cores, 2 tensor cores
 
+// Error code for a nonzero device status word: a wait that ran out of time
+// wins over a failed index check of the debug build; any other bit is a
+// generic failure.
+int status_bits_to_code(uint32_t bits) {
+  if (bits & attn_b200::kStatusTimeout) return ATTN_ERR_DEVICE_TIMEOUT;
+  if (bits & attn_b200::kStatusBounds) return ATTN_ERR_DEVICE_BOUNDS;
+  return ATTN_ERR_CUDA;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
                                   void *, const cuuint64_t *, const cuuint64_t *,
                                   const cuuint32_t *, const cuuint32_t *,
@@ -1145,9 +1154,7 @@ int attn_status(attn_stream_t stream) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
-  if (bits & attn_b200::kStatusTimeout) return ATTN_ERR_DEVICE_TIMEOUT;
-  if (bits & attn_b200::kStatusBounds) return ATTN_ERR_DEVICE_BOUNDS;
-  return ATTN_ERR_CUDA;
+  return status_bits_to_code(bits);
 }
 
 uint32_t attn_last_status_bits(void) { return g_last_bits.load(); }
@@ -1324,8 +1331,7 @@ extern "C" int attn_fwd_host_noalloc(const void *q, const void *k,
   }
   if (bits != 0) {
     g_last_bits.store(bits);
-    return (bits & attn_b200::kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT
-                                              : ATTN_ERR_CUDA;
+    return status_bits_to_code(bits);
   }
   return ATTN_OK;
 }
