@@ -52,6 +52,40 @@ DECODE_MMA_SOURCES = ("attn_decode_mma_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_
 BWD_SOURCES = ("attn_bwd_kernel.cuh", "attn_fwd_kernel.cuh", "ptx_sm100.cuh")
 
 
+def cpu_model() -> str:
+    """Model name of the host CPU (first entry of /proc/cpuinfo), recorded
+    beside the core count of every CPU baseline."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def pages_context(w) -> dict:
+    """The pages' own figures for this path, quoted beside the result for
+    context.  They are not targets: none was measured on a B200."""
+    n_scores = w.B * w.H * w.N * w.N
+    return {
+        "note": "figures printed on the pages, for context only (not targets)",
+        "hopper_fa2_vs_ampere_fa2": (
+            "+20-50% FLOPs/s for the CUTLASS FlashAttention-2 forward on one "
+            "H100 PCIe over the Ampere-tuned kernel (briefgpt.xyz keyword page "
+            "'attention algorithm', abstract)"),
+        "standard_attention_scores_fp16_gb_printed": 12.9,
+        "standard_attention_scores_fp16_gb_computed": round(
+            23400 * 23400 * 12 * 2 / 1e9, 2),
+        "standard_attention_scores_source": (
+            "23,400 one-second steps x 12 heads, fp16 S, under standard "
+            "attention (marketmaker.cc post, introduction)"),
+        "this_workload_scores_fp16_gb": round(n_scores * 2 / 1e9, 3),
+    }
+
+
 def _code_only(text: str) -> str:
     """C++ source without comments and with whitespace runs collapsed, so
     that editing a comment does not change the hash of the code."""
@@ -265,7 +299,7 @@ def cpu_baseline(w, qkv, budget_s: float, seed: int = 11):
         if budget_s - elapsed < 0.5:
             break
     return {"value": done_flops / elapsed / 1e12, "unit": "TFLOP/s",
-            "cores": threads, "kind": "oracle",
+            "cores": threads, "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"{done_rows} random query rows of {w.name} "
                       f"({done_rows / total_rows:.2e} of the workload), fp64 "
                       f"two-pass oracle, {elapsed:.1f} s"}
@@ -322,6 +356,7 @@ def cpu_baseline_bwd(w, budget_s: float):
     dt = time.perf_counter() - t0
     flops = 2.5 * sub.flops()
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "cpu_model": cpu_model(),
             "kind": "oracle",
             "sample": f"fp64 backward of {H} heads x N={n}, d={w.d} "
                       f"({'causal' if w.causal else 'non-causal'}), {dt:.1f} s"}
@@ -455,6 +490,7 @@ def cpu_baseline_fp8(w, qkv, signs, budget_s: float, seed: int = 13):
             break
     total = elapsed + t_quant * rows_done / w.N
     return {"value": flops / total / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "cpu_model": cpu_model(),
             "kind": "oracle",
             "sample": f"head (0,0) of {w.name}: quantized in {t_quant:.1f} s "
                       f"(amortised over the rows), {rows_done} random query "
@@ -638,6 +674,7 @@ def cpu_baseline_decode(w, qkv, budget_s: float):
     heads = done / w.Nq
     kv = heads * 2 * w.Nk * w.d * 2
     return {"value": kv / elapsed / 1e9, "unit": "GB/s", "cores": threads,
+            "cpu_model": cpu_model(),
             "kind": "oracle",
             "sample": f"{done} of {rows_total} query rows of {w.name} "
                       f"(fp64 oracle, {elapsed:.1f} s)"}
@@ -1047,6 +1084,7 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "steps": e2e_steps,
                     "api": "attn_fwd_host (pinned host buffers)"},
+            "context": pages_context(w),
             "gpu_launches": args.steps,
             "clocks": clk,
         }
