@@ -17,6 +17,7 @@ from .oracle import (  # noqa: F401
     attention_backward,
     attention_blocked,
     attention_rows_bf16,
+    attention_full_bf16,
     attend_scores,
     softmax_row,
     bf16_bits,

@@ -373,3 +373,58 @@ def quantize_qkv_fp8(qbits, kbits, vbits, rotate: bool, signs=None):
     v8, vs = fp8_quantize(vbits, False, None, vbits.shape[-2])
     return dict(q8=q8, qs=qs, k8=k8, ks=ks, v8=v8, vs=vs,
                 gain=(1.0 / d) if rotate else 1.0)
+
+
+def attention_full_bf16(qbits, kbits, vbits, causal: bool, scale: float,
+                        threads=None, panel: int = 256):
+    """The definition over EVERY row of bf16 bit-pattern inputs [B, H, N, d],
+    with the score block of a panel of query rows formed by a library matrix
+    product (float64 BLAS) instead of the C oracle's scalar loops; for the
+    full-output checks of the largest workloads, where the row oracle would
+    take many minutes.
+
+    Per head and panel of `panel` query rows, the steps are those of the C
+    oracle, in the same order ([MM] "Mengapa perhatian terikat pada
+    memori"; the masked path of "Integrasinya delapan baris"):
+        S = scale * Q_panel K^T          (keys up to the panel's last row
+                                          when causal; later keys are masked)
+        S[i, j] = -inf for j > i         (causal)
+        m = rowmax S;  E = exp(S - m);  l = rowsum E
+        O = (E V) / l;  lse = m + ln l
+    Panels run on a thread pool with one BLAS thread each.  Returns float64
+    (O [B, H, N, d], lse [B, H, N])."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from threadpoolctl import threadpool_limits
+
+    shape = tuple(qbits.shape)
+    B, H, N, d = shape
+    BH = B * H
+    heads = [tuple(bf16_bits_to_f64(np.asarray(x).reshape(BH, N, d)[h])
+                   for x in (qbits, kbits, vbits)) for h in range(BH)]
+    O = np.empty((BH, N, d))
+    lse = np.empty((BH, N))
+
+    def one_panel(job):
+        h, r0 = job
+        q, k, v = heads[h]
+        r1 = min(N, r0 + panel)
+        n_keys = r1 if causal else N
+        S = scale * (q[r0:r1] @ k[:n_keys].T)
+        if causal:
+            S[np.arange(n_keys)[None, :] > np.arange(r0, r1)[:, None]] = -np.inf
+        m = S.max(axis=1)
+        E = np.exp(S - m[:, None])
+        l = E.sum(axis=1)
+        O[h, r0:r1] = (E @ v[:n_keys]) / l[:, None]
+        lse[h, r0:r1] = m + np.log(l)
+
+    jobs = [(h, r0) for h in range(BH) for r0 in range(0, N, panel)]
+    # heaviest panels first under the causal mask, so the pool ends together
+    if causal:
+        jobs.sort(key=lambda j: -j[1])
+    with threadpool_limits(limits=1, user_api="blas"):
+        with ThreadPoolExecutor(max_workers=_threads(threads)) as ex:
+            for _ in ex.map(one_panel, jobs):
+                pass
+    return O.reshape(shape), lse.reshape(shape[:-1])

@@ -358,3 +358,54 @@ def test_bad_arguments_are_rejected(oracle_mod):
     qb = np.zeros((1, 1, 4, 2), dtype=np.uint16)
     with pytest.raises(RuntimeError):
         oracle_mod.attention_rows_bf16(qb, qb, qb, False, 1.0, np.array([4]))
+
+
+# --------------------------------------------------------------------------
+# the full-output entry point (score blocks by BLAS products)
+# --------------------------------------------------------------------------
+
+def _bf16(shape, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * std).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,panel", [(1, 256), (45, 16), (300, 128), (777, 256)])
+def test_full_bf16_matches_row_oracle(oracle_mod, causal, N, panel):
+    """The panelled BLAS form of the definition equals the scalar C oracle to
+    rounding on every row, with ragged last panels and panels that straddle
+    the causal diagonal."""
+    shape = (2, 2, N, 16)
+    q, k, v = (_bf16(shape, s, 2.0) for s in (11, 12, 13))
+    qb, kb, vb = (oracle_mod.bf16_bits(t) for t in (q, k, v))
+    O, lse = oracle_mod.attention(oracle_mod.bf16_bits_to_f64(qb),
+                                  oracle_mod.bf16_bits_to_f64(kb),
+                                  oracle_mod.bf16_bits_to_f64(vb), causal, 0.3)
+    Of, lf = oracle_mod.attention_full_bf16(qb, kb, vb, causal, 0.3, panel=panel)
+    np.testing.assert_allclose(Of, O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lf, lse, rtol=0, atol=1e-12)
+
+
+def test_full_bf16_closed_forms(oracle_mod):
+    """N = 1 gives V and the dot product; Q = 0 gives the (prefix) mean of V
+    with lse = ln N (ln(i + 1) when causal)."""
+    one = [oracle_mod.bf16_bits(_bf16((1, 3, 1, 8), s)) for s in (21, 22, 23)]
+    for causal in (False, True):
+        O, lse = oracle_mod.attention_full_bf16(*one, causal, 0.5)
+        f = [oracle_mod.bf16_bits_to_f64(b) for b in one]
+        assert np.array_equal(O, f[2])
+        np.testing.assert_allclose(lse, 0.5 * np.einsum("bhnd,bhnd->bhn", f[0], f[1]),
+                                   rtol=1e-15, atol=1e-15)
+    N = 333
+    k, v = (oracle_mod.bf16_bits(_bf16((1, 2, N, 8), s)) for s in (24, 25))
+    q = np.zeros_like(k)
+    vf = oracle_mod.bf16_bits_to_f64(v)
+    O, lse = oracle_mod.attention_full_bf16(q, k, v, False, 1.0, panel=100)
+    np.testing.assert_allclose(O, np.broadcast_to(vf.mean(axis=2, keepdims=True),
+                                                  O.shape), atol=1e-14)
+    np.testing.assert_allclose(lse, math.log(N), rtol=1e-15)
+    O, lse = oracle_mod.attention_full_bf16(q, k, v, True, 1.0, panel=100)
+    np.testing.assert_allclose(O, np.cumsum(vf, axis=2) /
+                               np.arange(1, N + 1).reshape(1, 1, N, 1), atol=1e-14)
+    np.testing.assert_allclose(lse, np.broadcast_to(np.log(np.arange(1, N + 1)),
+                                                    lse.shape), rtol=1e-15)
