@@ -221,8 +221,19 @@ int launch(DeviceState &st, int variant, const CUtensorMap *maps,
       st.smem_attr_set[variant] = true;
     }
   }
+  // O (bf16 [B*H, N, D]) as the epilogue's TMA store sees it: boxes of 64
+  // columns x 32 rows, one per softmax warp and half row.  The merge modes
+  // write through the accumulator instead and leave the map unused.
+  CUtensorMap map_o;
+  std::memset(&map_o, 0, sizeof map_o);
+  if (p.merge_mode == attn_b200::kMergeNone) {
+    EncodeTiledFn enc;
+    int rc = get_encode_fn(&enc);
+    if (rc == ATTN_OK) rc = encode_map(enc, &map_o, p.o, p.bh, p.n, D, 32);
+    if (rc != ATTN_OK) return rc;
+  }
   const int grid = p.num_units < st.sm_count ? p.num_units : st.sm_count;
-  kern<<<grid, attn_b200::kThreads, smem, stream>>>(maps[0], maps[1], maps[2], p);
+  kern<<<grid, attn_b200::kThreads, smem, stream>>>(maps[0], maps[1], maps[2], map_o, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }

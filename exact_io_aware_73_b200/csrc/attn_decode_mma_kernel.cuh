@@ -152,12 +152,6 @@ __device__ __forceinline__ float warp_max_f32(float v) {
   return r;
 }
 
-// Generic-proxy writes to shared memory become visible to the tensor cores
-// (async proxy) after this fence and a synchronisation.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "

@@ -37,9 +37,10 @@
 //   * S = Q K^T: tcgen05.mma kind::f16, M=128 N=128 K=d, A and B K-major in
 //     128B-swizzled shared memory (exactly the layout the TMA writes);
 //     O += P V: M=128 N=d K=128, A from TMEM, B (V) MN-major in shared memory;
-//   * each softmax thread writes its own output row straight from TMEM to
-//     HBM (16-byte stores); Q tiles are released by a tcgen05.commit after
-//     their last S MMA, so the next unit's Q load overlaps this epilogue;
+//   * the epilogue stages each warp's 32 output rows in shared memory and
+//     writes them with TMA tensor stores (whole 128-byte row segments); Q
+//     tiles are released by a tcgen05.commit after their last S MMA, so the
+//     next unit's Q load overlaps this epilogue;
 //   * the row max is rescaled lazily: the output is only corrected when a
 //     row's running max grows by more than 2^8 (in exp2 units); P then stays
 //     below 256, and O / l is unchanged because m and l always move together;
@@ -191,7 +192,11 @@ struct Smem {
   static constexpr uint32_t kQ = 0;                           // 2 Q tiles
   static constexpr uint32_t kK = kQ + 2 * kTileBytes;         // K ring
   static constexpr uint32_t kV = kK + kKStages * kTileBytes;  // V ring
-  static constexpr uint32_t kBars = kV + kVStages * kTileBytes;
+  // O staging for the TMA store of the epilogue: one buffer of 32 rows x 64
+  // bf16 columns (128-byte rows, 128B-swizzled) per softmax warp
+  static constexpr uint32_t kOutWarpBytes = 32 * 128;
+  static constexpr uint32_t kOut = kV + kVStages * kTileBytes;
+  static constexpr uint32_t kBars = kOut + 8 * kOutWarpBytes;
   // barrier indices
   // P_HALF: the first 64 keys of a tile's P are in TMEM (bf16 only);
   // P_FULL: all of it
@@ -705,6 +710,7 @@ __device__ __forceinline__ float exp_row_fp8(const uint32_t (&s)[4][32], float c
 
 template <int D, bool CAUSAL, bool FP8>
 __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
+                                             const CUtensorMap *tmo,
                                              const FwdParams &p,
                                              const WaitCtx &wc, int warp,
                                              int lane) {
@@ -831,22 +837,52 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     const float lse_this = (m_run - (FP8 ? 8.f : 0.f) + lg2_approx(l_run)) * kLn2;
     float lse_out = lse_this;
     if (p.merge_mode == kMergeNone) {
-      uint4 *orow = reinterpret_cast<uint4 *>(p.o + grow * D);
+      // The row of O leaves TMEM first, so that its columns go back to the
+      // next unit's P.V as early as possible.  It then reaches HBM through
+      // shared memory: each warp stages its 32 rows x 64 columns in the
+      // 128B-swizzled layout of the O tensor map, and one lane issues a TMA
+      // tensor store, so the global writes are whole 128-byte row segments
+      // rather than 16-byte pieces 2 D bytes apart.  The tensor map clips
+      // rows at or past N.
+      uint32_t ov[D / 32][32];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld_32x32b_x32(tO + c * 32, o);
-        tmem_wait_ld(o);
-        uint32_t h[16];
+      for (int c = 0; c < D / 32; ++c) tmem_ld_32x32b_x32(tO + c * 32, ov[c]);
+      tmem_wait_ld(ov[0]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
-                             __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (row_ok) {
+      for (int c = 1; c < D / 32; ++c) reg_fence(ov[c]);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::O_EMPTY + t));  // O columns reusable
+      const uint32_t buf = base + L::kOut + static_cast<uint32_t>(warp) * L::kOutWarpBytes;
+      const int y0 = qs + wq * 32;
+      int zc = w.bh;
+      if constexpr (kDebugBounds) {
+        // the injected index error of the debug build (see grow above)
+        if ((p.debug_flags & 4u) && blockIdx.x == 0 && k == 0 && t == 0 && wq == 0)
+          zc += p.bh;
+      }
+      const bool store_ok =
+          y0 < p.n && in_bounds(zc, p.bh, p.status) && in_bounds(y0, p.n, p.status);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            orow[c * 4 + i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2],
-                                         h[4 * i + 3]);
+      for (int h = 0; h < D / 64; ++h) {
+        uint32_t wv[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = 64 * h + 2 * i;
+          wv[i] = pack_bf16x2(__uint_as_float(ov[col >> 5][col & 31]) * inv_l,
+                              __uint_as_float(ov[(col + 1) >> 5][(col + 1) & 31]) * inv_l);
+        }
+        if (lane == 0) bulk_wait_group_read0();  // the previous store has read the buffer
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(buf + lane * 128 + ((c ^ (lane & 7)) << 4), wv[4 * c],
+                       wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && store_ok) {
+          tma_store_3d(tmo, buf, 64 * h, y0, zc);
+          bulk_commit_group();
         }
       }
     } else {
@@ -897,10 +933,10 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
             arow[c * 8 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
       }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::O_EMPTY + t));  // O columns reusable
     }
-    tc_fence_before_sync();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar(L::O_EMPTY + t));  // O columns reusable
     if (row_ok) {
       if (p.merge_mode == kMergeFirst || p.merge_mode == kMergeInto)
         p.acc_lse[grow] = lse_out;
@@ -908,6 +944,8 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
         p.lse[grow] = lse_out;
     }
   }
+  // every TMA store this warp issued must be complete before the CTA exits
+  if (lane == 0) bulk_wait_group0();
 }
 
 // ------------------------------------------------------------------ kernel
@@ -917,6 +955,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o,
                           const FwdParams p) {
   using L = Smem<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
@@ -958,6 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
+    if (p.merge_mode == kMergeNone) prefetch_tensormap(&tm_o);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -967,7 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role<D, CAUSAL, FP8>(base, tmem, p, wc, warp, lane);
+    softmax_role<D, CAUSAL, FP8>(base, tmem, &tm_o, p, wc, warp, lane);
   } else {
     setmaxnreg_dec<kControlRegs>();
     if (warp == kProducerWarp) {
