@@ -232,8 +232,27 @@ int launch(DeviceState &st, int variant, const CUtensorMap *maps,
     if (rc == ATTN_OK) rc = encode_map(enc, &map_o, p.o, p.bh, p.n, D, 32);
     if (rc != ATTN_OK) return rc;
   }
-  const int grid = p.num_units < st.sm_count ? p.num_units : st.sm_count;
-  kern<<<grid, attn_b200::kThreads, smem, stream>>>(maps[0], maps[1], maps[2], map_o, p);
+  // Non-causal units are pairs of Q tiles of equal cost.  When the last
+  // round of pairs would fill at most half of the CTAs (or every pair fits
+  // in half of them), those pairs run as single Q tiles on twice as many
+  // CTAs: a lone tile shares neither the tensor pipe nor the exponential
+  // unit, so it takes well under the time of a pair.
+  FwdParams q = p;
+  if (!CAUSAL) {
+    const int64_t S = st.sm_count, U2 = p.num_units;
+    if (2 * U2 <= S) {
+      q.tail_start = 0;
+      q.num_units = static_cast<int>(2 * U2);
+    } else {
+      const int64_t G = U2 < S ? U2 : S, R = U2 / G, r = U2 % G;
+      if (r > 0 && 2 * r <= G && U2 + r <= 0x7fffffffLL) {
+        q.tail_start = static_cast<int>(G * R);
+        q.num_units = static_cast<int>(G * R + 2 * r);
+      }
+    }
+  }
+  const int grid = q.num_units < st.sm_count ? q.num_units : st.sm_count;
+  kern<<<grid, attn_b200::kThreads, smem, stream>>>(maps[0], maps[1], maps[2], map_o, q);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }

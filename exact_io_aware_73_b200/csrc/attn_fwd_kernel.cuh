@@ -163,6 +163,11 @@ struct FwdParams {
   float *acc_o = nullptr;
   float *acc_lse = nullptr;
   int merge_mode = 0;
+  // Non-causal only: units from tail_start on are single Q tiles, unit
+  // tail_start + s being tile s % 2 of the pair tail_start + s / 2 (a last
+  // round of pairs that would fill few CTAs runs as twice as many single
+  // tiles instead).
+  int tail_start = 0x7fffffff;
 };
 constexpr int kMergeNone = 0, kMergeFirst = 1, kMergeInto = 2, kMergeLast = 3;
 
@@ -212,17 +217,30 @@ struct Smem {
 };
 
 // One work unit: rows [q0, q0 + 256) of head bh, as two Q tiles; n0 / n1 =
-// number of K/V tiles each Q tile visits (0 = tile lies beyond N).
+// number of K/V tiles each Q tile visits (0 = tile lies beyond N).  A
+// single-tile unit has n1 = 0.
 struct Unit {
   int bh, q0, n0, n1;
 };
 
 template <bool CAUSAL>
-__device__ __forceinline__ Unit decode_unit(int u, int bh_count, int n) {
+__device__ __forceinline__ Unit decode_unit(int u, int bh_count, int n,
+                                            int tail_start) {
   const int qpairs = (n + 255) >> 8;
   const int tiles = (n + 127) >> 7;
   Unit w;
   int qp;
+  if (!CAUSAL && u >= tail_start) {
+    // a single Q tile of one of the last pairs; it runs in the first tile's
+    // slot (softmax warpgroup 0, S0 / O0)
+    const int s = u - tail_start;
+    const int pr = tail_start + (s >> 1);
+    w.bh = pr / qpairs;
+    w.q0 = (pr % qpairs) * 256 + 128 * (s & 1);
+    w.n0 = (w.q0 < n) ? tiles : 0;
+    w.n1 = 0;
+    return w;
+  }
   if (CAUSAL) {
     // heaviest units (last query rows) first, heads interleaved
     qp = qpairs - 1 - u / bh_count;
@@ -366,7 +384,7 @@ __device__ __forceinline__ void producer_role(uint32_t base,
   const uint64_t pol_q = policy_evict_first();
 
   for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
-    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
+    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
     const int nt[2] = {w.n0, w.n1};
     for (int t = 0; MODE != kLoadV && t < 2; ++t) {
       if (nt[t] == 0) continue;
@@ -504,9 +522,10 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
   bool ok = true;
 
   for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
-    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
+    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
     const int nt[2] = {w.n0, w.n1};
     const int nmax = max(nt[0], nt[1]);
+    if (nmax == 0) continue;  // a single tile beyond N: nothing to compute
     for (int t = 0; t < 2 && ok; ++t)
       if (nt[t] > 0) {
         ok = mbar_wait_spin(bar(L::Q_FULL + t), qocc[t] & 1, wc, kRoleMma);
@@ -727,7 +746,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
   bool ok = true;
 
   for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
-    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n);
+    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
     const int n = t ? w.n1 : w.n0;
     if (n == 0) continue;
     const int qs = w.q0 + kBlockM * t;
