@@ -915,6 +915,11 @@ def main():
                          "fp8: the FP8 forward with incoherent processing; "
                          "decode: split-KV decode (decode_* workloads); "
                          "seqpar: one sequence sharded over ranks")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="forward on N GPUs: replicas (default: every rank "
+                         "its own seeded problem, weak scaling) or heads (the "
+                         "B*H heads of one problem split into contiguous "
+                         "ranges over the ranks, strong scaling)")
     ap.add_argument("--shards", type=int, default=1,
                     help="seqpar on one process: shards emulated on one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -951,12 +956,20 @@ def main():
     def barrier():
         R.barrier(world)
 
-    # ---- inputs (seeded per rank), resident in HBM before timing
-    seed = R.rank_seed(w.seed, rank)
+    # ---- inputs, resident in HBM before timing: a problem of its own per
+    # rank (seeded per rank), or this rank's range of the heads of one problem
+    heads = args.split == "heads"
+    seed = w.seed if heads else R.rank_seed(w.seed, rank)
     qkv_host = W.make_qkv(w, seed=seed)
+    Bs, Hs = w.B, w.H
+    if heads:
+        h0, nh = R.head_shard(w.B * w.H, world, rank)
+        qkv_host = tuple(t.reshape(w.B * w.H, w.N, w.d)[h0:h0 + nh]
+                         .reshape(1, nh, w.N, w.d).contiguous() for t in qkv_host)
+        Bs, Hs = 1, nh
     q, k, v = (t.to(dev) for t in qkv_host)
     o = torch.empty_like(q)
-    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    lse = torch.empty((Bs, Hs, w.N), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     in_bytes = 3 * q.numel() * 2
@@ -965,7 +978,7 @@ def main():
 
     def step():
         rc = attn.attn_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                               o.data_ptr(), lse.data_ptr(), w.B, w.H, w.N,
+                               o.data_ptr(), lse.data_ptr(), Bs, Hs, w.N,
                                w.d, w.causal, w.scale, sh)
         if rc != 0:
             raise attn.AttnError(rc, "attn_fwd")
@@ -1014,14 +1027,17 @@ def main():
 
     max_ms = R.max_over_ranks(kernel_ms, world, dev)
     ms_per_step = max_ms / args.steps
-    flops = w.flops()
-    value = R.job_throughput(flops, world, ms_per_step * 1e-3) / 1e12
+    # FLOPs of this rank's launch; the job's are every rank's (replicas) or
+    # the one problem's (heads)
+    flops = w.flops() * (Bs * Hs) / (w.B * w.H)
+    job_flops = w.flops() if heads else world * w.flops()
+    value = job_flops / (ms_per_step * 1e-3) / 1e12
 
     # ---- end to end through the host-buffer C entry point
     qh, kh, vh = (x.pin_memory() for x in qkv_host)
     oh = torch.empty_like(qh).pin_memory()
-    lh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
-    ws = torch.empty(attn.host_workspace_bytes(w.B, w.H, w.N, w.d),
+    lh = torch.empty((Bs, Hs, w.N), dtype=torch.float32).pin_memory()
+    ws = torch.empty(attn.host_workspace_bytes(Bs, Hs, w.N, w.d),
                      dtype=torch.uint8, device=dev)
     del q, k, v, o, lse
     e2e_steps = max(3, min(args.steps, 10))
@@ -1041,7 +1057,7 @@ def main():
     if rc != 0:
         raise attn.AttnError(rc, "e2e region")
     e2e_ms = R.max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
-    e2e_value = R.job_throughput(flops, world, e2e_ms * 1e-3) / 1e12
+    e2e_value = job_flops / (e2e_ms * 1e-3) / 1e12
     h2d = 3 * qh.numel() * 2
     d2h = oh.numel() * 2 + lh.numel() * 4
 
@@ -1068,13 +1084,17 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "strong" if heads else "weak", "vs_baseline": None,
+            "dtype": "bf16",
             "data": "synthetic (seeded Gaussian/uniform bf16 inputs)",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N,
                        "d": w.d, "causal": w.causal, "scale": w.scale,
                        "l2": l2_note,
-                       "parallelism": (f"{world} independent replicas (one "
-                                       "workload per GPU, no collective)")},
+                       "parallelism": (
+                           f"the {w.B * w.H} heads of one problem split over "
+                           f"{world} GPUs (contiguous ranges, no collective)"
+                           if heads else f"{world} independent replicas (one "
+                           "workload per GPU, no collective)")},
             "roofline": roofline,
             "exp_roof": exp_roof(flops, w.d, ms_per_step,
                                  torch.cuda.get_device_properties(dev).multi_processor_count,

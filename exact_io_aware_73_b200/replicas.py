@@ -1,9 +1,11 @@
 """Multi-GPU scaffolding: independent replicas, one process per GPU.
 
 Every (batch, head, query-tile) unit of attention is independent, so
-running on N GPUs needs no data exchange: each rank computes a whole
-problem of its own (its own seeded inputs) and the job's throughput is the
-sum of the ranks' work over the slowest rank's time.  ``torch.distributed``
+running on N GPUs needs no data exchange.  By default each rank computes a
+whole problem of its own (its own seeded inputs) and the job's throughput is
+the sum of the ranks' work over the slowest rank's time.  Alternatively the
+B*H heads of one problem are split into contiguous ranges (head_shard), each
+rank computing its range with K and V of its heads only.  ``torch.distributed``
 is used only for a barrier and for the max-over-ranks of the device timings.
 Nothing here touches tensors of the attention itself.
 """
@@ -51,6 +53,18 @@ def max_over_ranks(x: float, world: int, device="cpu") -> float:
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def head_shard(bh: int, world: int, rank: int):
+    """The contiguous range of the B*H heads of one problem that a rank
+    computes when one problem is split over ranks: (first head, count).
+    Heads are independent (no key or value crosses heads), so the ranks'
+    outputs tile the single-GPU output exactly; the first bh % world ranks
+    take one head more."""
+    bh, world, rank = int(bh), int(world), int(rank)
+    base, extra = divmod(bh, world)
+    first = rank * base + min(rank, extra)
+    return first, base + (1 if rank < extra else 0)
 
 
 def job_throughput(units_per_rank: float, world: int, max_seconds: float) -> float:

@@ -98,3 +98,66 @@ def test_reference_arm_under_torchrun_prints_on_rank0_only(tmp_path):
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["value"] > 0
+
+
+# --------------------------------------------------------------------------
+# one problem split by heads over ranks (bench.py --split heads)
+# --------------------------------------------------------------------------
+
+def test_head_shard_tiles_every_head_exactly_once():
+    from exact_io_aware_73_b200 import replicas as R
+    for bh in (1, 2, 5, 12, 32, 48, 97):
+        for world in (1, 2, 3, 4, 8):
+            ranges = [R.head_shard(bh, world, r) for r in range(world)]
+            covered = [h for h0, n in ranges for h in range(h0, h0 + n)]
+            assert covered == list(range(bh)), (bh, world, ranges)
+            counts = [n for _, n in ranges]
+            assert max(counts) - min(counts) <= 1
+
+
+def _head_worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+                      WORLD_SIZE=str(world), RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import oracle
+    from exact_io_aware_73_b200 import replicas as R
+    from exact_io_aware_73_b200 import workloads as W
+    R.init("gloo", world, timeout_s=60)
+    # every rank draws the same problem and computes its own range of heads;
+    # the oracle stands in for the kernel (each head is computed alone)
+    w = W.shape_case(2, 3, 50, 64, True, seed=321)
+    f = [oracle.bf16_bits_to_f64(oracle.bf16_bits(t)) for t in W.make_qkv(w)]
+    h0, nh = R.head_shard(w.B * w.H, world, rank)
+    part = [x.reshape(w.B * w.H, w.N, w.d)[h0:h0 + nh][None] for x in f]
+    O, L = oracle.attention(*part, w.causal, w.scale)
+    # test-side gather of the shards (the benchmark itself exchanges nothing)
+    outs = [None] * world
+    torch.distributed.all_gather_object(outs, (h0, nh, O[0], L[0]))
+    R.finish(world)
+    if rank == 0:
+        O_all = np.concatenate([o for _, _, o, _ in outs])
+        L_all = np.concatenate([l for _, _, _, l in outs])
+        O_ref, L_ref = oracle.attention(*f, w.causal, w.scale)
+        np.save(os.path.join(out_dir, "o.npy"), O_all)
+        np.save(os.path.join(out_dir, "o_ref.npy"), O_ref.reshape(O_all.shape))
+        np.save(os.path.join(out_dir, "l.npy"), L_all)
+        np.save(os.path.join(out_dir, "l_ref.npy"), L_ref.reshape(L_all.shape))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_heads_split_over_gloo_ranks_reassemble_the_whole_problem(tmp_path, world):
+    import numpy as np
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_head_worker, args=(r, world, port, str(tmp_path)))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    o, o_ref = np.load(tmp_path / "o.npy"), np.load(tmp_path / "o_ref.npy")
+    l, l_ref = np.load(tmp_path / "l.npy"), np.load(tmp_path / "l_ref.npy")
+    assert np.array_equal(o, o_ref) and np.array_equal(l, l_ref)
