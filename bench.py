@@ -901,20 +901,192 @@ def run_seqpar(args, w):
     return 0
 
 
+METRIC_SPARSE = "block-sparse attention fwd TFLOP/s (bf16; FLOPs of the computed blocks)"
+
+
+def cpu_baseline_sparse(w, qkv, mask, budget_s: float, seed: int = 17):
+    """The block-sparse fp64 oracle on random rows of the workload, all host
+    cores; TFLOP/s over the FLOPs those rows' kept keys take."""
+    import numpy as np
+    import oracle
+    bits = [oracle.bf16_bits(t) for t in qkv]
+    m = mask.numpy()
+    threads = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(seed)
+    T = (w.N + 127) // 128
+    keep = m.reshape(-1, T, T)[0].astype(np.int64)
+
+    def row_flops(rows):
+        i = rows % w.N
+        kept = np.zeros(len(rows))
+        for a, r in enumerate(i):
+            js = np.arange((r + 1) if w.causal else w.N)
+            kept[a] = keep[r // 128][js // 128].sum()
+        return float(np.sum(4.0 * kept * w.d))
+
+    done, flops, elapsed, batch = 0, 0.0, 0.0, max(threads, 8)
+    while elapsed < budget_s:
+        rows = rng.integers(0, w.B * w.H * w.N, size=batch)
+        t0 = time.perf_counter()
+        oracle.attention_block_sparse_rows_bf16(*bits, w.causal, w.scale, m, rows,
+                                                threads)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        done += batch
+        flops += row_flops(rows)
+        batch = int(min(max(threads, batch / max(dt, 1e-6) * (budget_s - elapsed) * 0.9),
+                        w.B * w.H * w.N))
+        if budget_s - elapsed < 0.5:
+            break
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "cpu_model": cpu_model(), "kind": "oracle",
+            "sample": f"{done} random query rows of {w.name} with its block mask, "
+                      f"fp64 block-sparse oracle, {elapsed:.1f} s"}
+
+
+def run_sparse(args):
+    """Block-sparse forward: the named workload's shape with its seeded block
+    mask (a sliding window of key tiles plus random ones, one mask for every
+    head).  A step is one attn_fwd_block_sparse launch; FLOPs count the
+    computed blocks only."""
+    import torch
+    from exact_io_aware_73_b200 import attn
+    name = args.workload if args.workload in W.SPARSE_WORKLOADS else \
+        "sparse_long_b1h32n16384d128"
+    w, density, local = W.SPARSE_WORKLOADS[name]
+    world, rank, local_rank = R.env_ranks()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    R.init("nccl", world, device=dev)
+    qkv_host = W.make_qkv(w, seed=R.rank_seed(w.seed, rank))
+    mask = W.block_mask_for(name)
+    q, k, v = (t.to(dev) for t in qkv_host)
+    md = mask.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    flops = W.sparse_flops(w, mask)
+    kept = float(mask.float().mean())
+    in_bytes = 3 * q.numel() * 2
+    flush = None if in_bytes > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8,
+                                                         device=dev)
+
+    def step():
+        rc = attn.attn_fwd_block_sparse_raw(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+            w.B, w.H, w.N, w.d, w.causal, w.scale, md.data_ptr(), False, sh)
+        if rc != 0:
+            raise attn.AttnError(rc, "attn_fwd_block_sparse")
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    if attn.status() != 0:
+        raise RuntimeError("device status after warm-up")
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.begin()
+    evs = []
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        evs.append((a, b))
+    R.barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.end()
+    clk = clocks.stop()
+    if attn.status() != 0:
+        raise RuntimeError("device status after the timed region")
+    ms = R.max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
+    ms_per_step = ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    # end to end: inputs from pinned host memory, the call, outputs back
+    qh, kh, vh = (t.pin_memory() for t in qkv_host)
+    mh = mask.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for src, dst in ((qh, q), (kh, k), (vh, v), (mh, md)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if attn.status() != 0:
+        raise RuntimeError("device status after the e2e region")
+    e2e_ms = R.max_over_ranks(e0.elapsed_time(e1), world, dev) / n_e2e
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    cb = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb = cpu_baseline_sparse(w, qkv_host, mask, args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC_SPARSE, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian bf16 inputs, seeded block mask)",
+            "config": {"workload": name, "pass": "sparse", "B": w.B, "H": w.H,
+                       "N": w.N, "d": w.d, "causal": w.causal,
+                       "blocks_kept": round(kept, 4), "window_tiles": local,
+                       "random_density": density,
+                       "l2": "inputs larger than L2" if flush is None else
+                             "L2 flushed between steps (outside the events)",
+                       "parallelism": f"{world} independent replicas"},
+            "roofline": {"bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+                         "traffic": load_traffic(name),
+                         "algorithmic_flops_per_launch": flops,
+                         "kernel": KERNEL_NAME},
+            "cpu_baseline": cb,
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": in_bytes + mask.numel(),
+                    "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4,
+                    "ms_per_step": e2e_ms, "steps": n_e2e,
+                    "api": "attn_fwd_block_sparse with torch copies from pinned host memory"},
+            "gpu_launches": args.steps, "clocks": clk}), flush=True)
+    R.finish(world)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=W.HEADLINE,
-                    choices=sorted(W.WORKLOADS) + sorted(W.DECODE_WORKLOADS))
+                    choices=sorted(W.WORKLOADS) + sorted(W.DECODE_WORKLOADS) +
+                    sorted(W.SPARSE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--pass", dest="pass_", default="fwd",
-                    choices=["fwd", "bwd", "fp8", "decode", "seqpar"],
+                    choices=["fwd", "bwd", "fp8", "decode", "seqpar", "sparse"],
                     help="fwd (default): the forward hot path; bwd: attn_bwd; "
                          "fp8: the FP8 forward with incoherent processing; "
                          "decode: split-KV decode (decode_* workloads); "
-                         "seqpar: one sequence sharded over ranks")
+                         "seqpar: one sequence sharded over ranks; "
+                         "sparse: block-sparse forward (sparse_* workloads)")
     ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
                     help="forward on N GPUs: replicas (default: every rank "
                          "its own seeded problem, weak scaling) or heads (the "
@@ -931,8 +1103,13 @@ def main():
         if args.impl == "reference":
             ap.error("the reference arm times the forward oracle")
         return run_decode(args)
+    if args.pass_ == "sparse":
+        if args.impl == "reference":
+            ap.error("the reference arm times the forward oracle")
+        return run_sparse(args)
     if args.workload not in W.WORKLOADS:
-        ap.error(f"{args.workload} is a decode workload: use --pass decode")
+        ap.error(f"{args.workload} is a decode or block-sparse workload: use "
+                 "--pass decode or --pass sparse")
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

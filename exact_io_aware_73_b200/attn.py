@@ -141,6 +141,57 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None,
     return out, lse
 
 
+def _sparse_fn():
+    f = lib().attn_fwd_block_sparse
+    if f.argtypes is None:
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        f.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, ctypes.c_float, vp, i, vp]
+        f.restype = i
+    return f
+
+
+def attn_fwd_block_sparse_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d,
+                              causal, scale, mask_ptr, mask_per_head,
+                              stream_handle) -> int:
+    """Direct call with integer pointers; returns the library's code."""
+    return _sparse_fn()(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, int(B), int(H),
+                        int(N), int(d), int(bool(causal)), float(scale),
+                        mask_ptr, int(bool(mask_per_head)), stream_handle)
+
+
+def attn_fwd_block_sparse(q, k, v, block_mask, causal: bool = False,
+                          scale: float | None = None, out=None, lse=None,
+                          stream=None):
+    """O, lse of block-sparse attention: attn_fwd with the (128-query,
+    128-key) blocks that block_mask zeroes left out.  block_mask: uint8 CUDA
+    tensor [T, T] for every head, or [B, H, T, T] / [B*H, T, T] per head,
+    T = ceil(N / 128).  Rows with no key left get O = 0, lse = -inf."""
+    import torch
+    _expect_qkv(q, k, v)
+    B, H, N, d = q.shape
+    T = -(-N // 128)
+    if not isinstance(block_mask, torch.Tensor) or block_mask.dtype != torch.uint8:
+        raise TypeError("block_mask must be a uint8 CUDA tensor")
+    if block_mask.numel() not in (T * T, B * H * T * T):
+        raise ValueError(f"block_mask must hold {T}x{T} bytes or one such mask per head")
+    _expect("block_mask", block_mask, torch.uint8, device=q.device)
+    per_head = block_mask.numel() != T * T
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _expect("out", out, torch.bfloat16, q.shape, device=q.device)
+    _expect("lse", lse, torch.float32, (B, H, N), device=q.device)
+    rc = attn_fwd_block_sparse_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                   out.data_ptr(), lse.data_ptr(), B, H, N, d,
+                                   causal, scale, block_mask.data_ptr(), per_head,
+                                   _stream_handle(stream))
+    _check(rc, "attn_fwd_block_sparse")
+    return out, lse
+
+
 def attn_fwd_host(q, k, v, out, lse, causal: bool, scale: float, workspace,
                   stream=None):
     """End-to-end call on host (ideally pinned) bf16 tensors; `workspace` is a

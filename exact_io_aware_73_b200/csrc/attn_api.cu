@@ -33,7 +33,9 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   uint32_t *status = nullptr;  // 4-byte device status word, lazily allocated
-  bool smem_attr_set[6] = {false, false, false, false, false, false};
+  // forward variants: 0-3 bf16 (d, causal), 4-5 E4M3, 6-9 block-sparse bf16
+  bool smem_attr_set[10] = {false, false, false, false, false,
+                            false, false, false, false, false};
   bool bwd_attr_set[4] = {false, false, false, false};
   bool dec_attr_set[2] = {false, false};  // decode kernel, d = 128 / 64
   bool dm_attr_set[2] = {false, false};   // tensor-core decode kernel, d = 128 / 64
@@ -205,10 +207,10 @@ int encode_map_u8(EncodeTiledFn enc, CUtensorMap *map, const void *ptr, int bh,
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_TENSOR_MAP;
 }
 
-template <int D, bool CAUSAL, bool FP8 = false>
+template <int D, bool CAUSAL, bool FP8 = false, bool SPARSE = false>
 int launch(DeviceState &st, int variant, const CUtensorMap *maps,
            const FwdParams &p, cudaStream_t stream) {
-  auto kern = attn_b200::attn_fwd_sm100_kernel<D, CAUSAL, FP8>;
+  auto kern = attn_b200::attn_fwd_sm100_kernel<D, CAUSAL, FP8, SPARSE>;
   const uint32_t smem = Smem<D, FP8>::kAlloc;
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -238,7 +240,7 @@ int launch(DeviceState &st, int variant, const CUtensorMap *maps,
   // CTAs: a lone tile shares neither the tensor pipe nor the exponential
   // unit, so it takes well under the time of a pair.
   FwdParams q = p;
-  if (!CAUSAL) {
+  if (!CAUSAL && !SPARSE) {
     const int64_t S = st.sm_count, U2 = p.num_units;
     if (2 * U2 <= S) {
       q.tail_start = 0;
@@ -585,6 +587,58 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                   : launch<128, false>(*st, 1, maps, p, s);
   return causal ? launch<64, true>(*st, 2, maps, p, s)
                 : launch<64, false>(*st, 3, maps, p, s);
+}
+
+int attn_fwd_block_sparse(const void *q, const void *k, const void *v, void *o,
+                          float *lse, int B, int H, int N, int d, int causal,
+                          float scale, const uint8_t *block_mask,
+                          int mask_per_head, attn_stream_t stream) {
+  int rc = check_args(q, k, v, o, lse, B, H, N, d, scale, true);
+  if (rc != ATTN_OK || B == 0 || H == 0 || N == 0) return rc;
+  if (!block_mask) return ATTN_ERR_NULL_POINTER;
+  const int bh = B * H;
+  const int tiles = (N + 127) / 128;
+  const int64_t units = static_cast<int64_t>(bh) * tiles;
+  if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_SIZE;
+  const size_t mask_bytes = static_cast<size_t>(mask_per_head ? bh : 1) * tiles * tiles;
+  const size_t tb = static_cast<size_t>(bh) * N * d * 2, lb = static_cast<size_t>(bh) * N * 4;
+  if (overlaps(o, tb, block_mask, mask_bytes) || overlaps(lse, lb, block_mask, mask_bytes))
+    return ATTN_ERR_ALIAS;
+
+  int dev;
+  DeviceState *st;
+  if ((rc = current_device(&dev, &st)) != ATTN_OK) return rc;
+  if (!is_device_memory_of(q, dev) || !is_device_memory_of(k, dev) ||
+      !is_device_memory_of(v, dev) || !is_device_memory_of(o, dev) ||
+      !is_device_memory_of(lse, dev) || !is_device_memory_of(block_mask, dev))
+    return ATTN_ERR_NOT_DEVICE_MEMORY;
+
+  EncodeTiledFn enc;
+  if ((rc = get_encode_fn(&enc)) != ATTN_OK) return rc;
+  CUtensorMap maps[3];
+  if ((rc = encode_map(enc, &maps[0], q, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[1], k, bh, N, d)) != ATTN_OK) return rc;
+  if ((rc = encode_map(enc, &maps[2], v, bh, N, d)) != ATTN_OK) return rc;
+
+  FwdParams p;
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.status = st->status;
+  p.bh = bh;
+  p.n = N;
+  p.num_units = static_cast<int>(units);  // one Q tile per unit
+  p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.timeout_ns = g_timeout_ns.load();
+  p.debug_flags = 0;
+  p.block_mask = block_mask;
+  p.mask_head_stride = mask_per_head ? static_cast<int64_t>(tiles) * tiles : 0;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch<128, true, false, true>(*st, 6, maps, p, s)
+                  : launch<128, false, false, true>(*st, 7, maps, p, s);
+  return causal ? launch<64, true, false, true>(*st, 8, maps, p, s)
+                : launch<64, false, false, true>(*st, 9, maps, p, s);
 }
 
 int attn_fwd_merge(const void *q, const void *k, const void *v, float *acc_o,

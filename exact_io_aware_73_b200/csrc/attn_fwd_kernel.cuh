@@ -168,6 +168,12 @@ struct FwdParams {
   // round of pairs that would fill few CTAs runs as twice as many single
   // tiles instead).
   int tail_start = 0x7fffffff;
+  // Block-sparse variant only: one byte per (Q tile, K tile) pair of a head,
+  // row-major [tiles x tiles]; nonzero = the pair is computed.  A head's
+  // mask starts mask_head_stride bytes after the previous one's (0: one
+  // mask for every head).
+  const uint8_t *block_mask = nullptr;
+  int64_t mask_head_stride = 0;
 };
 constexpr int kMergeNone = 0, kMergeFirst = 1, kMergeInto = 2, kMergeLast = 3;
 
@@ -269,6 +275,43 @@ __device__ __forceinline__ int unit_at(int k) {
   return k * g + ((CAUSAL && (k & 1)) ? g - 1 - c : c);
 }
 
+// Block-sparse units (the block-sparse extension of the tiled algorithm,
+// briefgpt.xyz summary page of arXiv 2307.08691, FlashAttention entry): one
+// Q tile each, head-major, and only the K tiles its mask row marks; the
+// causal mask further excludes K tiles past the diagonal.  Every role walks
+// the same list with sparse_next, so the K/V ring stays in step.
+__device__ __forceinline__ const uint8_t *sparse_row(const FwdParams &p, int bh, int qt,
+                                                    int tiles) {
+  return p.block_mask + static_cast<int64_t>(bh) * p.mask_head_stride +
+         static_cast<int64_t>(qt) * tiles;
+}
+
+// The first computed K tile at or after kj (kend when there is none).
+__device__ __forceinline__ int sparse_next(const uint8_t *row, int kj, int kend) {
+  while (kj < kend && __ldg(row + kj) == 0) ++kj;
+  return kj;
+}
+
+template <bool CAUSAL, bool SPARSE>
+__device__ __forceinline__ Unit get_unit(int u, const FwdParams &p) {
+  if constexpr (!SPARSE) {
+    return decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
+  } else {
+    const int tiles = (p.n + 127) >> 7;
+    Unit w;
+    w.bh = u / tiles;
+    const int qt = u - w.bh * tiles;
+    w.q0 = qt * kBlockM;
+    const uint8_t *row = sparse_row(p, w.bh, qt, tiles);
+    const int kend = CAUSAL ? qt + 1 : tiles;
+    int cnt = 0;
+    for (int kj = 0; kj < kend; ++kj) cnt += (__ldg(row + kj) != 0);
+    w.n0 = cnt;
+    w.n1 = 0;
+    return w;
+  }
+}
+
 // Index checks of the debug build (compiled with ATTN_DEBUG_BOUNDS): an index
 // the kernel is about to use for a global access must lie in [0, limit);
 // when it does not, the status word is flagged and the caller skips the
@@ -366,7 +409,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr,
 // P.V MMAs).
 constexpr int kLoadQK = 1, kLoadV = 2;
 
-template <int D, bool CAUSAL, int MODE, bool FP8>
+template <int D, bool CAUSAL, int MODE, bool FP8, bool SPARSE>
 __device__ __forceinline__ void producer_role(uint32_t base,
                                               const CUtensorMap *tq,
                                               const CUtensorMap *tk,
@@ -384,8 +427,15 @@ __device__ __forceinline__ void producer_role(uint32_t base,
   const uint64_t pol_q = policy_evict_first();
 
   for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
-    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
+    const Unit w = get_unit<CAUSAL, SPARSE>(u, p);
     const int nt[2] = {w.n0, w.n1};
+    const uint8_t *srow = nullptr;
+    int kend = 0, kj = -1;  // block-sparse: the K tile of step j
+    if constexpr (SPARSE) {
+      const int tiles = (p.n + 127) >> 7, qt = w.q0 >> 7;
+      srow = sparse_row(p, w.bh, qt, tiles);
+      kend = CAUSAL ? qt + 1 : tiles;
+    }
     for (int t = 0; MODE != kLoadV && t < 2; ++t) {
       if (nt[t] == 0) continue;
       if (qocc[t] > 0) {
@@ -408,6 +458,8 @@ __device__ __forceinline__ void producer_role(uint32_t base,
     if (!ok) break;
     const int nmax = max(nt[0], nt[1]);
     for (int j = 0; j < nmax; ++j) {
+      if constexpr (SPARSE) kj = sparse_next(srow, kj + 1, kend);
+      else kj = j;
       if (MODE != kLoadV) {
         const int ks = k_issued % L::kKStages;
         ok = mbar_wait(bar(L::K_EMPTY + ks), ((k_issued / L::kKStages) & 1) ^ 1,
@@ -417,7 +469,7 @@ __device__ __forceinline__ void producer_role(uint32_t base,
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d_hint(base + L::kK + ks * L::kTileBytes + s * L::kPanelBytes,
                            tk, bar(L::K_FULL + ks), s * L::kPanelElems,
-                           j * kBlockN, w.bh,
+                           kj * kBlockN, w.bh,
                            pol_kv);
         ++k_issued;
       }
@@ -430,7 +482,7 @@ __device__ __forceinline__ void producer_role(uint32_t base,
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d_hint(base + L::kV + vs * L::kTileBytes + s * L::kPanelBytes,
                            tv, bar(L::V_FULL + vs), s * L::kPanelElems,
-                           j * kBlockN, w.bh,
+                           kj * kBlockN, w.bh,
                            pol_kv);
         ++v_issued;
       }
@@ -509,7 +561,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
   }
 }
 
-template <int D, bool CAUSAL, bool FP8>
+template <int D, bool CAUSAL, bool FP8, bool SPARSE>
 __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
                                          const FwdParams &p, const WaitCtx &wc) {
   using L = Smem<D, FP8>;
@@ -522,10 +574,10 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
   bool ok = true;
 
   for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
-    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
+    const Unit w = get_unit<CAUSAL, SPARSE>(u, p);
     const int nt[2] = {w.n0, w.n1};
     const int nmax = max(nt[0], nt[1]);
-    if (nmax == 0) continue;  // a single tile beyond N: nothing to compute
+    if (nmax == 0) continue;  // a single tile beyond N, or no K tile: nothing to compute
     for (int t = 0; t < 2 && ok; ++t)
       if (nt[t] > 0) {
         ok = mbar_wait_spin(bar(L::Q_FULL + t), qocc[t] & 1, wc, kRoleMma);
@@ -727,7 +779,7 @@ __device__ __forceinline__ float exp_row_fp8(const uint32_t (&s)[4][32], float c
   return (a0 + a1) + (b0 + b1);
 }
 
-template <int D, bool CAUSAL, bool FP8>
+template <int D, bool CAUSAL, bool FP8, bool SPARSE>
 __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
                                              const CUtensorMap *tmo,
                                              const FwdParams &p,
@@ -746,10 +798,40 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
   bool ok = true;
 
   for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
-    const Unit w = decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
+    const Unit w = get_unit<CAUSAL, SPARSE>(u, p);
     const int n = t ? w.n1 : w.n0;
-    if (n == 0) continue;
     const int qs = w.q0 + kBlockM * t;
+    if constexpr (SPARSE) {
+      if (n == 0 && t == 0 && qs < p.n) {
+        // No K tile computed for these rows: every score is masked, and the
+        // output is written as O = 0, lse = -inf (a reading: the softmax of
+        // an empty row is undefined).
+        const uint32_t buf = base + L::kOut + static_cast<uint32_t>(warp) * L::kOutWarpBytes;
+        const int y0 = qs + wq * 32;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) st_shared_v4(buf + lane * 128 + c * 16, 0u, 0u, 0u, 0u);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && y0 < p.n) {
+            tma_store_3d(tmo, buf, 64 * h, y0, w.bh);
+            bulk_commit_group();
+          }
+        }
+        if (qs + r < p.n) p.lse[static_cast<int64_t>(w.bh) * p.n + qs + r] = -CUDART_INF_F;
+      }
+    }
+    if (n == 0) continue;
+    const uint8_t *srow = nullptr;
+    int kend = 0, kj = -1;  // block-sparse: the K tile of step j
+    if constexpr (SPARSE) {
+      const int tiles = (p.n + 127) >> 7, qt = qs >> 7;
+      srow = sparse_row(p, w.bh, qt, tiles);
+      kend = CAUSAL ? qt + 1 : tiles;
+    }
     float m_run = -CUDART_INF_F;  // running max, log2 units (x = s * scale * log2 e)
     float l_run = 0.f;            // running sum of exp2(x - m_run)
     // FP8: the Q tile's scale joins the score multiplier; V's is applied at
@@ -770,8 +852,18 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
       if (!ok) break;
       tc_fence_after_sync();
 
-      const bool mask = (j == n - 1) && (CAUSAL || (p.n & (kBlockN - 1)));
-      const int limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
+      bool mask;
+      int limit;
+      if constexpr (SPARSE) {
+        // the causal diagonal tile, or the ragged last K tile
+        kj = sparse_next(srow, kj + 1, kend);
+        const bool diag = CAUSAL && kj == (qs >> 7);
+        mask = diag || (kj == ((p.n - 1) >> 7) && (p.n & (kBlockN - 1)));
+        limit = diag ? r : (p.n - 1 - kj * kBlockN);
+      } else {
+        mask = (j == n - 1) && (CAUSAL || (p.n & (kBlockN - 1)));
+        limit = CAUSAL ? r : (p.n - 1 - j * kBlockN);
+      }
       uint32_t s[4][32];
       load_scores(tS, s, mask, limit);
 
@@ -969,7 +1061,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
 
 // ------------------------------------------------------------------ kernel
 
-template <int D, bool CAUSAL, bool FP8 = false>
+template <int D, bool CAUSAL, bool FP8 = false, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -1026,17 +1118,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role<D, CAUSAL, FP8>(base, tmem, &tm_o, p, wc, warp, lane);
+    softmax_role<D, CAUSAL, FP8, SPARSE>(base, tmem, &tm_o, p, wc, warp, lane);
   } else {
     setmaxnreg_dec<kControlRegs>();
     if (warp == kProducerWarp) {
       if (lane == 0)
-        producer_role<D, CAUSAL, kLoadQK, FP8>(base, &tm_q, &tm_k, &tm_v, p, wc);
+        producer_role<D, CAUSAL, kLoadQK, FP8, SPARSE>(base, &tm_q, &tm_k, &tm_v, p, wc);
     } else if (warp == kVLoaderWarp) {
       if (lane == 0)
-        producer_role<D, CAUSAL, kLoadV, FP8>(base, &tm_q, &tm_k, &tm_v, p, wc);
+        producer_role<D, CAUSAL, kLoadV, FP8, SPARSE>(base, &tm_q, &tm_k, &tm_v, p, wc);
     } else if (warp == kMmaWarp) {
-      if (lane == 0) mma_role<D, CAUSAL, FP8>(base, tmem, p, wc);
+      if (lane == 0) mma_role<D, CAUSAL, FP8, SPARSE>(base, tmem, p, wc);
     }
     __syncwarp();
   }

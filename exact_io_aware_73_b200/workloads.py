@@ -134,6 +134,65 @@ def sample_rows(w: Workload, count: int, seed: int = 7):
     return sorted(picks)
 
 
+# ------------------------------------------------------------ block masks
+
+def make_block_mask(seed: int, T: int, density: float, heads: int = 0,
+                    local: int = 0) -> torch.Tensor:
+    """A block mask for the block-sparse variant: uint8 [T, T] (or
+    [heads, T, T] when heads > 0), 1 = the (128-query, 128-key) block is kept.
+    Each block is kept with probability ``density`` (seeded draw), and the
+    ``local`` blocks on and below the diagonal of every row are always kept
+    (a sliding window of local * 128 keys)."""
+    shape = (heads, T, T) if heads > 0 else (T, T)
+    m = (torch.rand(shape, generator=_gen(seed)) < float(density)).to(torch.uint8)
+    if local > 0:
+        i = torch.arange(T)[:, None]
+        j = torch.arange(T)[None, :]
+        m |= ((j <= i) & (j > i - int(local))).to(torch.uint8)
+    return m
+
+
+# Block-sparse workloads: the long headline shape with a sliding window of
+# 8 key tiles (1,024 keys) plus 25 % of the other key tiles at random, one
+# mask for every head, and the trading day with a 30-minute window (15 key
+# tiles of 128 one-second steps) plus 10 % random tiles, causal.
+SPARSE_WORKLOADS = {
+    "sparse_long_b1h32n16384d128": (WORKLOADS["long_b1h32n16384d128"], 0.25, 8),
+    "sparse_tradingday_b1h12n23400d64_causal": (
+        WORKLOADS["tradingday_b1h12n23400d64_causal"], 0.10, 15),
+}
+
+
+def block_mask_for(name: str) -> torch.Tensor:
+    """The [T, T] mask of a named block-sparse workload (seed 4242)."""
+    w, density, local = SPARSE_WORKLOADS[name]
+    return make_block_mask(4242, (w.N + 127) // 128, density, local=local)
+
+
+def sparse_flops(w: Workload, mask: torch.Tensor) -> float:
+    """FLOPs of the two GEMMs over the computed blocks only: 4 d per visible
+    score, with the causal mask and the ragged last key tile counted
+    exactly (scores of masked-out blocks are not computed)."""
+    T = (w.N + 127) // 128
+    m = mask.reshape(-1, T, T).to(torch.int64)
+    qlen = torch.full((T,), 128, dtype=torch.int64)
+    qlen[-1] = w.N - 128 * (T - 1)
+    klen = qlen.clone()
+    pairs = qlen[:, None] * klen[None, :]
+    if w.causal:
+        # rows of tile i see keys <= row: full tiles below the diagonal, and
+        # r + 1 keys of the diagonal tile for its row r
+        i = torch.arange(T)[:, None]
+        j = torch.arange(T)[None, :]
+        diag = qlen * (qlen + 1) // 2
+        pairs = torch.where(j < i, pairs, torch.zeros_like(pairs))
+        pairs = pairs + torch.diag(diag)
+    per_head = (m * pairs[None]).sum(dim=(1, 2)).to(torch.float64)
+    heads = w.B * w.H
+    total = per_head.sum() * (heads if m.shape[0] == 1 else 1)
+    return float(4.0 * w.d * total)
+
+
 # ------------------------------------------------------------ FP8 inputs
 
 def make_signs(seed: int, d: int) -> torch.Tensor:

@@ -406,6 +406,36 @@ void attn_set_decode_kernel(int which);
 int attn_decode_kernel_for(int Nq, int d);
 
 /*
+ * attn_fwd_block_sparse -- attn_fwd restricted to the (query tile, key tile)
+ * blocks a mask selects: the block-sparse extension of the tiled exact
+ * algorithm (briefgpt.xyz summary page of FlashAttention-2, arXiv
+ * 2307.08691, FlashAttention entry: the method "extends to block-sparse
+ * attention"; the entry on sparse FlashAttention for key/query dropping).
+ *
+ *   S[i, j] = -inf when block_mask[i / 128][j / 128] == 0 (and, if causal,
+ *             when j > i); O = softmax_rows(S) V; lse[i] = ln sum_j exp S[i, j].
+ *   A row whose every score is masked gets O = 0 and lse = -inf (the softmax
+ *   of an empty row is undefined; this is the reading taken).
+ *
+ * q, k, v, o, lse: as attn_fwd (device memory, [B, H, N, d] bf16 and
+ * [B, H, N] fp32, the same alignment and aliasing rules).  block_mask: device
+ * bytes, row-major [T, T] with T = ceil(N / 128), one byte per pair of a
+ * 128-row query tile and a 128-key key tile, nonzero = computed; shared by
+ * every head (mask_per_head = 0) or one [T, T] mask per head in [B, H] order
+ * (mask_per_head != 0; B * H * T * T bytes).  Owned by the caller, only read.
+ * Under the causal mask, blocks above the diagonal are never computed
+ * whatever their mask byte.  Work is one query tile per CTA step over the
+ * selected key tiles only, so time scales with the number of selected
+ * blocks.  Errors as attn_fwd, plus ATTN_ERR_NULL_POINTER for a NULL mask
+ * and ATTN_ERR_NOT_DEVICE_MEMORY for a mask outside the current device.
+ * Asynchronous on `stream`.
+ */
+int attn_fwd_block_sparse(const void *q, const void *k, const void *v, void *o,
+                          float *lse, int B, int H, int N, int d, int causal,
+                          float scale, const uint8_t *block_mask,
+                          int mask_per_head, attn_stream_t stream);
+
+/*
  * Merging partial attention results -- the softmax statistics kept per row
  * (the marketmaker.cc post's section "Backward pass", folded into lse) make
  * attention over disjoint key sets exactly combinable:

@@ -18,6 +18,8 @@ from .oracle import (  # noqa: F401
     attention_blocked,
     attention_rows_bf16,
     attention_full_bf16,
+    attention_block_sparse_rows_bf16,
+    attention_block_sparse_bf16,
     attend_scores,
     softmax_row,
     bf16_bits,

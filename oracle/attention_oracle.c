@@ -333,6 +333,75 @@ int oracle_attention_rows_bf16(const uint16_t *Q, const uint16_t *K,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Block-sparse attention.                                                  */
+/* ------------------------------------------------------------------------ */
+
+/* The block-sparse extension of the tiled method (briefgpt.xyz summary page
+ * of FlashAttention-2, arXiv 2307.08691, FlashAttention entry): scores of
+ * the (query block, key block) pairs a mask leaves out are -inf, so those
+ * keys drop out of the row; the rest is the definition above.  Blocks are
+ * 128 rows of queries by 128 keys; mask is row-major [T, T] bytes, T =
+ * ceil(N / 128), nonzero = kept; one mask for every head (mask_per_head = 0)
+ * or one per head in [B, H] order.  With the causal mask, key j > i is also
+ * dropped.  A row with no key left has no softmax; the reading taken is
+ * O = 0 and lse = -inf.  Selected rows (flat bh * N + i) of bf16 bit
+ * patterns, widened exactly, as in oracle_attention_rows_bf16. */
+int oracle_attention_block_sparse_rows_bf16(
+    const uint16_t *Q, const uint16_t *K, const uint16_t *V, int64_t B,
+    int64_t H, int64_t N, int64_t d, int causal, double scale,
+    const uint8_t *mask, int mask_per_head, const int64_t *rows, int64_t nrows,
+    double *O_out, double *lse_out, int nthreads) {
+  if (!Q || !K || !V || !mask || !rows || !O_out || !lse_out || B < 0 ||
+      H < 0 || N < 1 || d < 1 || nrows < 0)
+    return ORACLE_EBADARG;
+  for (int64_t a = 0; a < nrows; ++a)
+    if (rows[a] < 0 || rows[a] >= B * H * N) return ORACLE_EBADARG;
+  const int64_t T = (N + 127) / 128;
+  int err = ORACLE_OK;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *qi = (double *)malloc(sizeof(double) * (size_t)d);
+    double *vv = (double *)malloc(sizeof(double) * (size_t)(N * d));
+    if (!s || !qi || !vv) {
+#pragma omp atomic write
+      err = ORACLE_ENOMEM;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t a = 0; a < nrows; ++a) {
+      if (!s || !qi || !vv) continue;
+      const int64_t r = rows[a], bh = r / N, i = r % N;
+      const uint16_t *Kh = K + bh * N * d, *Vh = V + bh * N * d;
+      const uint8_t *mrow = mask + (mask_per_head ? bh * T * T : 0) + (i / 128) * T;
+      for (int64_t t = 0; t < d; ++t) qi[t] = bf16_bits_to_double(Q[r * d + t]);
+      /* the kept keys of row i, in ascending order */
+      int64_t n = 0;
+      const int64_t jend = visible_keys(i, N, causal);
+      for (int64_t j = 0; j < jend; ++j) {
+        if (mrow[j / 128] == 0) continue;
+        double acc = 0.0;
+        for (int64_t t = 0; t < d; ++t)
+          acc += qi[t] * bf16_bits_to_double(Kh[j * d + t]);
+        s[n] = scale * acc;
+        for (int64_t t = 0; t < d; ++t)
+          vv[n * d + t] = bf16_bits_to_double(Vh[j * d + t]);
+        ++n;
+      }
+      if (n == 0) {
+        for (int64_t t = 0; t < d; ++t) O_out[a * d + t] = 0.0;
+        lse_out[a] = -INFINITY;
+        continue;
+      }
+      attend_row(s, n, vv, d, O_out + a * d, lse_out + a, NULL);
+    }
+    free(s);
+    free(qi);
+    free(vv);
+  }
+  return err;
+}
+
+/* ------------------------------------------------------------------------ */
 /* The pages' blocked algorithm, as a second opinion on the oracle.         */
 /* ------------------------------------------------------------------------ */
 

@@ -49,6 +49,11 @@ def _load():
         lib.oracle_attention_decode_rows_bf16.argtypes = [
             u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_int, ctypes.c_double,
             i64p, i64, dp, dp, ctypes.c_int]
+        lib.oracle_attention_block_sparse_rows_bf16.argtypes = [
+            u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_int, ctypes.c_double,
+            ctypes.POINTER(ctypes.c_uint8), ctypes.c_int, i64p, i64, dp, dp,
+            ctypes.c_int]
+        lib.oracle_attention_block_sparse_rows_bf16.restype = ctypes.c_int
         lib.oracle_attention_backward_rows_bf16.argtypes = [
             u16p, u16p, u16p, u16p, i64, i64, ctypes.c_int, ctypes.c_double,
             i64p, i64, dp, i64p, i64, dp, dp, ctypes.c_int]
@@ -428,3 +433,46 @@ def attention_full_bf16(qbits, kbits, vbits, causal: bool, scale: float,
             for _ in ex.map(one_panel, jobs):
                 pass
     return O.reshape(shape), lse.reshape(shape[:-1])
+
+
+def attention_block_sparse_rows_bf16(qbits, kbits, vbits, causal: bool,
+                                     scale: float, block_mask, rows,
+                                     threads=None):
+    """Block-sparse attention ([MM]'s definition with the scores of the
+    (128-query, 128-key) blocks the mask leaves out set to -inf; rows with no
+    key left give O = 0, lse = -inf) on selected flat rows (bh * N + i) of
+    bf16 bit patterns [B, H, N, d].  block_mask: uint8 [T, T] shared by all
+    heads or [B, H, T, T] (or [B * H, T, T]) per head, T = ceil(N / 128).
+    Returns (O [len(rows), d], lse [len(rows)])."""
+    qbits = np.ascontiguousarray(qbits, dtype=np.uint16)
+    kbits = np.ascontiguousarray(kbits, dtype=np.uint16)
+    vbits = np.ascontiguousarray(vbits, dtype=np.uint16)
+    B, H, N, d = qbits.shape
+    T = -(-N // 128)
+    m = np.ascontiguousarray(block_mask, dtype=np.uint8)
+    per_head = int(m.size != T * T)
+    if m.size not in (T * T, B * H * T * T):
+        raise ValueError("block_mask must hold T*T or B*H*T*T bytes")
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    O = np.empty((rows.size, d))
+    lse = np.empty(rows.size)
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    _check(_load().oracle_attention_block_sparse_rows_bf16(
+        qbits.ctypes.data_as(u16p), kbits.ctypes.data_as(u16p),
+        vbits.ctypes.data_as(u16p), B, H, N, d, int(bool(causal)),
+        float(scale), m.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+        per_head, rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        rows.size, _dptr(O), _dptr(lse), _threads(threads)),
+        "attention_block_sparse_rows_bf16")
+    return O, lse
+
+
+def attention_block_sparse_bf16(qbits, kbits, vbits, causal: bool, scale: float,
+                                block_mask, threads=None):
+    """attention_block_sparse_rows_bf16 over every row; O [B, H, N, d],
+    lse [B, H, N]."""
+    B, H, N, d = qbits.shape
+    rows = np.arange(B * H * N, dtype=np.int64)
+    O, lse = attention_block_sparse_rows_bf16(qbits, kbits, vbits, causal, scale,
+                                              block_mask, rows, threads)
+    return O.reshape(B, H, N, d), lse.reshape(B, H, N)

@@ -1,0 +1,118 @@
+"""GPU parity of block-sparse attention (attn_fwd_block_sparse) against the
+fp64 block-sparse oracle.
+
+The block-sparse extension of the tiled method (briefgpt.xyz summary page of
+FlashAttention-2, arXiv 2307.08691, FlashAttention entry): the (128-query,
+128-key) blocks a mask leaves out are skipped, which is the same as setting
+their scores to -inf.  Tolerances are the forward's: max |O - O_ref| <= 2e-2,
+max |lse - lse_ref| <= 5e-3; rows that keep no key must be exactly O = 0 and
+lse = -inf.  With every block kept (or, under the causal mask, every block
+on and below the diagonal) the result must equal attn_fwd's bit for bit: the
+kernel is the forward kernel walking a list of K tiles.
+"""
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_73_b200 import attn
+from exact_io_aware_73_b200 import workloads as W
+
+O_TOL = 2e-2
+LSE_TOL = 5e-3
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    if torch.cuda.get_device_capability() != (10, 0):
+        pytest.skip("needs a B200 (sm_100)")
+    attn.lib()
+    yield
+    assert attn.status() == 0
+
+
+def _compare(o, lse, o_ref, lse_ref, what):
+    o = o.reshape(o_ref.shape)
+    lse = lse.reshape(lse_ref.shape)
+    empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), empty), what
+    assert np.all(o[empty] == 0), what
+    keep = ~empty
+    assert np.all(np.isfinite(o[keep])) and np.all(np.isfinite(lse[keep])), what
+    eo = float(np.max(np.abs(o[keep] - o_ref[keep]))) if keep.any() else 0.0
+    el = float(np.max(np.abs(lse[keep] - lse_ref[keep]))) if keep.any() else 0.0
+    assert eo <= O_TOL, f"{what}: max|dO| {eo}"
+    assert el <= LSE_TOL, f"{what}: max|dlse| {el}"
+    return eo, el
+
+
+SHAPES = [(1, 1, 1, 128), (1, 3, 129, 64), (1, 2, 300, 64), (2, 1, 1000, 128),
+          (1, 1, 1536, 128), (2, 2, 777, 64)]
+
+
+@pytest.mark.parametrize("per_head", [False, True])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,H,N,d", SHAPES)
+def test_block_sparse_parity(oracle_mod, B, H, N, d, causal, per_head):
+    w = W.shape_case(B, H, N, d, causal, seed=300 + N + d + B + H)
+    q, k, v = W.make_qkv(w)
+    T = (N + 127) // 128
+    m = W.make_block_mask(17 + N, T, 0.5, heads=B * H if per_head else 0)
+    if T > 1:
+        # one query tile keeps no block at all (its rows: O = 0, lse = -inf)
+        m.reshape(-1, T, T)[:, 1, :] = 0
+    o, lse = attn.attn_fwd_block_sparse(q.cuda(), k.cuda(), v.cuda(), m.cuda(),
+                                        causal=causal, scale=w.scale)
+    assert attn.status() == 0
+    bits = [oracle_mod.bf16_bits(t) for t in (q, k, v)]
+    o_ref, l_ref = oracle_mod.attention_block_sparse_bf16(*bits, causal, w.scale,
+                                                          m.numpy())
+    _compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(300, 64), (1000, 128), (1536, 128)])
+def test_full_mask_equals_dense_forward_bit_for_bit(N, d, causal):
+    w = W.shape_case(2, 3, N, d, causal, seed=400 + N)
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    T = (N + 127) // 128
+    full = torch.ones(T, T, dtype=torch.uint8)
+    if causal:
+        full = torch.tril(full)   # blocks above the diagonal never count
+    o, lse = attn.attn_fwd_block_sparse(q, k, v, full.cuda(), causal=causal,
+                                        scale=w.scale)
+    od, ld = attn.attn_fwd(q, k, v, causal=causal, scale=w.scale)
+    assert attn.status() == 0
+    assert torch.equal(o, od) and torch.equal(lse, ld)
+
+
+def test_empty_mask_gives_zero_and_minus_infinity():
+    w = W.shape_case(1, 2, 400, 128, False, seed=51)
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    m = torch.zeros(4, 4, dtype=torch.uint8, device="cuda")
+    o = torch.full_like(q, 7.0)
+    lse = torch.zeros(1, 2, 400, device="cuda")
+    attn.attn_fwd_block_sparse(q, k, v, m, out=o, lse=lse)
+    assert attn.status() == 0
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+@pytest.mark.parametrize("name", sorted(W.SPARSE_WORKLOADS))
+def test_block_sparse_workloads_sampled_rows(oracle_mod, name):
+    """The benchmark's block-sparse workloads, in the launch the benchmark
+    times, on sampled rows (first, tile edges, last, ragged tail, random)."""
+    w, _, _ = W.SPARSE_WORKLOADS[name]
+    q, k, v = W.make_qkv(w)
+    m = W.block_mask_for(name)
+    o, lse = attn.attn_fwd_block_sparse(q.cuda(), k.cuda(), v.cuda(), m.cuda(),
+                                        causal=w.causal, scale=w.scale)
+    assert attn.status() == 0
+    rows = np.array(W.sample_rows(w, 256))
+    bits = [oracle_mod.bf16_bits(t) for t in (q, k, v)]
+    o_ref, l_ref = oracle_mod.attention_block_sparse_rows_bf16(
+        *bits, w.causal, w.scale, m.numpy(), rows)
+    _compare(o.float().cpu().numpy().reshape(-1, w.d)[rows],
+             lse.cpu().numpy().reshape(-1)[rows], o_ref, l_ref, name)

@@ -292,3 +292,27 @@ def test_decode_kernel_choice_without_a_device(attn):
         assert attn.decode_kernel_for(3, 64) == attn.DECODE_TENSOR_CORES
     finally:
         attn.set_decode_kernel(attn.DECODE_AUTO)
+
+
+def test_block_sparse_refuses_bad_arguments_without_a_device(attn):
+    """attn_fwd_block_sparse checks its arguments (those of attn_fwd, plus the
+    mask pointer and the mask's overlap with the outputs) before any CUDA
+    call; fake pointers are never dereferenced."""
+    far = 1 << 40
+    f = attn._sparse_fn()
+    ok = dict(q=far, k=2 * far, v=3 * far, o=4 * far, lse=5 * far, B=1, H=2,
+              N=300, d=64, causal=0, scale=0.125, mask=6 * far, per_head=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"],
+                 a["d"], a["causal"], a["scale"], a["mask"], a["per_head"], None)
+
+    assert call(mask=None) == 1                 # ATTN_ERR_NULL_POINTER
+    assert call(N=-1) == 2                      # ATTN_ERR_INVALID_SIZE
+    assert call(d=96) == 3                      # head size
+    assert call(q=far + 8) == 4                 # misaligned
+    assert call(scale=0.0) == 5
+    assert call(o=far) == 6                     # o over q
+    assert call(mask=4 * far + 64) == 6         # mask inside o
+    assert call(mask=None, B=0) == 0            # empty problem: nothing to do

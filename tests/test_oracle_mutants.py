@@ -24,6 +24,7 @@ PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 BACKWARD_PINS = os.path.join(ROOT, "tests", "test_oracle_backward_pins.py")
 FP8_PINS = os.path.join(ROOT, "tests", "test_oracle_fp8_pins.py")
 DECODE_PINS = os.path.join(ROOT, "tests", "test_oracle_decode_pins.py")
+SPARSE_PINS = os.path.join(ROOT, "tests", "test_oracle_sparse_pins.py")
 
 MUTANTS = {
     "mask_hides_diagonal": ("return causal ? (i + 1) : N;",
@@ -94,13 +95,32 @@ DECODE_MUTANTS = {
                                      "for (int64_t t = 0; t < d; ++t) vv[j * d + t] = bf16_bits_to_double(Kh[j * d + t]);"),
 }
 
+# planted mistakes in the block-sparse oracle; each must fail a sparse pin
+SPARSE_MUTANTS = {
+    "sparse_mask_transposed": (
+        "if (mrow[j / 128] == 0) continue;",
+        "if (mask[(mask_per_head ? bh * T * T : 0) + (j / 128) * T + i / 128] == 0) continue;"),
+    "sparse_heads_share_first_mask": (
+        "const uint8_t *mrow = mask + (mask_per_head ? bh * T * T : 0) + (i / 128) * T;",
+        "const uint8_t *mrow = mask + (i / 128) * T;"),
+    "sparse_blocks_of_64_keys": (
+        "if (mrow[j / 128] == 0) continue;",
+        "if (mrow[j / 64 < T ? j / 64 : T - 1] == 0) continue;"),
+    "sparse_empty_row_not_special": (
+        "      if (n == 0) {\n        for (int64_t t = 0; t < d; ++t) O_out[a * d + t] = 0.0;",
+        "      if (n < 0) {\n        for (int64_t t = 0; t < d; ++t) O_out[a * d + t] = 0.0;"),
+    "sparse_causal_ignored": (
+        "const int64_t jend = visible_keys(i, N, causal);\n      for (int64_t j = 0; j < jend; ++j) {\n        if (mrow",
+        "const int64_t jend = N;\n      for (int64_t j = 0; j < jend; ++j) {\n        if (mrow"),
+}
+
 
 def _build_mutant(name, tmpdir):
     if name in FP8_MUTANTS:
         old, new = FP8_MUTANTS[name]
         target, other = FP8_SRC, SRC
     else:
-        old, new = {**MUTANTS, **BACKWARD_MUTANTS, **DECODE_MUTANTS}[name]
+        old, new = {**MUTANTS, **BACKWARD_MUTANTS, **DECODE_MUTANTS, **SPARSE_MUTANTS}[name]
         target, other = SRC, FP8_SRC
     src = open(target).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
@@ -153,3 +173,9 @@ def test_every_planted_decode_mistake_fails_a_decode_pin():
     with tempfile.TemporaryDirectory() as tmp:
         survivors = _run_against(DECODE_MUTANTS, DECODE_PINS, tmp)
         assert not survivors, f"decode pins did not catch: {survivors}"
+
+
+def test_every_planted_sparse_mistake_fails_a_sparse_pin():
+    with tempfile.TemporaryDirectory() as tmp:
+        survivors = _run_against(SPARSE_MUTANTS, SPARSE_PINS, tmp)
+        assert not survivors, f"block-sparse pins did not catch: {survivors}"
