@@ -598,7 +598,7 @@ int attn_fwd_block_sparse(const void *q, const void *k, const void *v, void *o,
   if (!block_mask) return ATTN_ERR_NULL_POINTER;
   const int bh = B * H;
   const int tiles = (N + 127) / 128;
-  const int64_t units = static_cast<int64_t>(bh) * tiles;
+  const int64_t units = static_cast<int64_t>(bh) * ((tiles + 1) / 2);
   if (units > 0x7fffffffLL) return ATTN_ERR_INVALID_SIZE;
   const size_t mask_bytes = static_cast<size_t>(mask_per_head ? bh : 1) * tiles * tiles;
   const size_t tb = static_cast<size_t>(bh) * N * d * 2, lb = static_cast<size_t>(bh) * N * 4;
@@ -626,7 +626,7 @@ int attn_fwd_block_sparse(const void *q, const void *k, const void *v, void *o,
   p.status = st->status;
   p.bh = bh;
   p.n = N;
-  p.num_units = static_cast<int>(units);  // one Q tile per unit
+  p.num_units = static_cast<int>(units);  // two consecutive Q tiles per unit
   p.c_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.timeout_ns = g_timeout_ns.load();
   p.debug_flags = 0;

@@ -29,11 +29,14 @@
 //   * a persistent CTA per SM walks "units" = two 128-row Q tiles of one
 //     (batch, head) that share every K/V tile it loads;
 //   * warps 0-3 / 4-7: softmax warpgroups for Q tile 0 / 1 (one TMEM lane =
-//     one query row per thread); warp 8: TMA loader; warp 9: tcgen05 MMA
-//     issuer (one thread) and TMEM owner;
+//     one query row per thread); warps 8 and 10: TMA loaders (Q and K, V);
+//     warp 9: tcgen05 MMA issuer (one thread) and TMEM owner; at d = 64 and
+//     for block-sparse units warp 9 issues for Q tile 0 and warp 11 for
+//     Q tile 1;
 //   * TMEM (512 columns x 128 lanes x 32 bit): S0 | S1 | O0 | O1.  The
-//     softmax writes P (bf16) back over the first 64 columns of its S tile;
-//     the P.V MMA reads it from TMEM as its A operand;
+//     softmax writes P (bf16) back over the first 64 columns of its S tile
+//     (at d = 64, dense: into 64 columns of its own after O1); the P.V MMA
+//     reads it from TMEM as its A operand;
 //   * S = Q K^T: tcgen05.mma kind::f16, M=128 N=128 K=d, A and B K-major in
 //     128B-swizzled shared memory (exactly the layout the TMA writes);
 //     O += P V: M=128 N=d K=128, A from TMEM, B (V) MN-major in shared memory;
@@ -73,7 +76,8 @@ constexpr int kBlockN = 128;   // keys per K/V tile
 constexpr int kThreads = 384;  // 12 warps = 3 warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kVLoaderWarp = 10;  // warp 11 only completes warpgroup 2
+constexpr int kVLoaderWarp = 10;
+constexpr int kMmaWarp2 = 11;  // tile 1's MMA issuer (see mma_role_tile)
 // Register split.  With 12 warps every thread is launched with 168
 // registers (an SM sub-partition holds 3 warps of the CTA); warpgroup 2 (the
 // loader / MMA / idle warps) hands registers back and the two softmax
@@ -210,14 +214,18 @@ struct Smem {
   static constexpr uint32_t kBars = kOut + 8 * kOutWarpBytes;
   // barrier indices
   // P_HALF: the first 64 keys of a tile's P are in TMEM (bf16 only);
-  // P_FULL: all of it
+  // P_FULL: all of it; S_FREE (d = 64 only): the softmax has read its S
+  // tile out of TMEM
   static constexpr int Q_FULL = 0, Q_EMPTY = 2, S_FULL = 4, P_FULL = 6,
                        O_FULL = 8, O_EMPTY = 10, DRAIN = 12, P_HALF = 13,
-                       K_FULL = 15, K_EMPTY = K_FULL + kKStages,
+                       S_FREE = 15,
+                       K_FULL = 17, K_EMPTY = K_FULL + kKStages,
                        V_FULL = K_EMPTY + kKStages, V_EMPTY = V_FULL + kVStages,
                        NUM_BARS = V_EMPTY + kVStages;
   static constexpr uint32_t kMisc = kBars + NUM_BARS * 8;  // tmem slot, abort
-  static constexpr uint32_t kBytes = kMisc + 16;
+  // the ring index each K / V slot was last claimed for (see slot_claimed)
+  static constexpr uint32_t kSlotPos = kMisc + 16;
+  static constexpr uint32_t kBytes = kSlotPos + 4 * (kKStages + kVStages);
   static constexpr uint32_t kAlloc = kBytes + 1024;  // slack for alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
@@ -226,7 +234,8 @@ struct Smem {
 // number of K/V tiles each Q tile visits (0 = tile lies beyond N).  A
 // single-tile unit has n1 = 0.
 struct Unit {
-  int bh, q0, n0, n1;
+  int bh, q0, n0, n1;  // n0, n1: K tiles Q tile 0 / 1 computes
+  int nu;              // K/V tiles the unit loads (the union of both lists)
 };
 
 template <bool CAUSAL>
@@ -245,6 +254,7 @@ __device__ __forceinline__ Unit decode_unit(int u, int bh_count, int n,
     w.q0 = (pr % qpairs) * 256 + 128 * (s & 1);
     w.n0 = (w.q0 < n) ? tiles : 0;
     w.n1 = 0;
+    w.nu = w.n0;
     return w;
   }
   if (CAUSAL) {
@@ -260,6 +270,7 @@ __device__ __forceinline__ Unit decode_unit(int u, int bh_count, int n,
   const int qt0 = w.q0 >> 7;
   w.n0 = CAUSAL ? min(tiles, qt0 + 1) : tiles;
   w.n1 = (w.q0 + 128 < n) ? (CAUSAL ? min(tiles, qt0 + 2) : tiles) : 0;
+  w.nu = max(w.n0, w.n1);
   return w;
 }
 
@@ -276,10 +287,13 @@ __device__ __forceinline__ int unit_at(int k) {
 }
 
 // Block-sparse units (the block-sparse extension of the tiled algorithm,
-// briefgpt.xyz summary page of arXiv 2307.08691, FlashAttention entry): one
-// Q tile each, head-major, and only the K tiles its mask row marks; the
-// causal mask further excludes K tiles past the diagonal.  Every role walks
-// the same list with sparse_next, so the K/V ring stays in step.
+// briefgpt.xyz summary page of arXiv 2307.08691, FlashAttention entry): two
+// consecutive Q tiles of one (batch, head), like the dense units, each
+// computing only the K tiles its mask row marks (and, under the causal mask,
+// none past its diagonal).  The unit loads the union of the two lists, in
+// order; a K/V tile that only one of the tiles uses is computed by that
+// tile alone.  Every role walks the same union with KWalk, so the K/V ring
+// stays in step.
 __device__ __forceinline__ const uint8_t *sparse_row(const FwdParams &p, int bh, int qt,
                                                     int tiles) {
   return p.block_mask + static_cast<int64_t>(bh) * p.mask_head_stride +
@@ -297,20 +311,71 @@ __device__ __forceinline__ Unit get_unit(int u, const FwdParams &p) {
   if constexpr (!SPARSE) {
     return decode_unit<CAUSAL>(u, p.bh, p.n, p.tail_start);
   } else {
-    const int tiles = (p.n + 127) >> 7;
+    const int tiles = (p.n + 127) >> 7, pairs = (tiles + 1) >> 1;
     Unit w;
-    w.bh = u / tiles;
-    const int qt = u - w.bh * tiles;
-    w.q0 = qt * kBlockM;
-    const uint8_t *row = sparse_row(p, w.bh, qt, tiles);
-    const int kend = CAUSAL ? qt + 1 : tiles;
-    int cnt = 0;
-    for (int kj = 0; kj < kend; ++kj) cnt += (__ldg(row + kj) != 0);
-    w.n0 = cnt;
-    w.n1 = 0;
+    int pq;
+    if (CAUSAL) {  // heaviest pairs (last query rows) first, heads interleaved
+      pq = pairs - 1 - u / p.bh;
+      w.bh = u % p.bh;
+    } else {
+      w.bh = u / pairs;
+      pq = u % pairs;
+    }
+    const int qt0 = 2 * pq, qt1 = qt0 + 1;
+    w.q0 = qt0 * kBlockM;
+    const uint8_t *r0 = sparse_row(p, w.bh, qt0, tiles);
+    const uint8_t *r1 = sparse_row(p, w.bh, qt1 < tiles ? qt1 : qt0, tiles);
+    const int kend0 = CAUSAL ? qt0 + 1 : tiles;
+    const int kend1 = qt1 < tiles ? (CAUSAL ? qt1 + 1 : tiles) : 0;
+    int c0 = 0, c1 = 0, cu = 0;
+    for (int kj = 0; kj < max(kend0, kend1); ++kj) {
+      const bool m0 = kj < kend0 && __ldg(r0 + kj) != 0;
+      const bool m1 = kj < kend1 && __ldg(r1 + kj) != 0;
+      c0 += m0;
+      c1 += m1;
+      cu += (m0 || m1);
+    }
+    w.n0 = c0;
+    w.n1 = c1;
+    w.nu = cu;
     return w;
   }
 }
+
+// The K/V tiles one unit loads, in order: next() steps to the following
+// one and returns its K tile index, with bit t of `use` set when Q tile t
+// computes it.  Dense units load K tiles 0 .. nu-1, and tile t uses the
+// first n_t of them.
+template <bool CAUSAL, bool SPARSE>
+struct KWalk {
+  const uint8_t *r0, *r1;
+  int kend0, kend1, kj, n0, n1;
+  __device__ __forceinline__ KWalk(const FwdParams &p, const Unit &w)
+      : r0(nullptr), r1(nullptr), kend0(0), kend1(0), kj(-1), n0(w.n0), n1(w.n1) {
+    if constexpr (SPARSE) {
+      const int tiles = (p.n + 127) >> 7, qt0 = w.q0 >> 7, qt1 = qt0 + 1;
+      r0 = sparse_row(p, w.bh, qt0, tiles);
+      r1 = sparse_row(p, w.bh, qt1 < tiles ? qt1 : qt0, tiles);
+      kend0 = CAUSAL ? qt0 + 1 : tiles;
+      kend1 = qt1 < tiles ? (CAUSAL ? qt1 + 1 : tiles) : 0;
+    }
+  }
+  __device__ __forceinline__ int next(int &use) {
+    ++kj;
+    if constexpr (SPARSE) {
+      const int kend = max(kend0, kend1);
+      for (; kj < kend; ++kj) {
+        use = (kj < kend0 && __ldg(r0 + kj) != 0) | ((kj < kend1 && __ldg(r1 + kj) != 0) << 1);
+        if (use) return kj;
+      }
+      use = 0;  // past the end (callers stop after nu steps)
+      return kj;
+    } else {
+      use = (kj < n0) | ((kj < n1) << 1);
+      return kj;
+    }
+  }
+};
 
 // Index checks of the debug build (compiled with ATTN_DEBUG_BOUNDS): an index
 // the kernel is about to use for a global access must lie in [0, limit);
@@ -381,6 +446,32 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
   }
 }
 
+// With one MMA issuer per Q tile, a tile skips the K/V tiles of its unit
+// that only the other tile computes, so it may come to wait on a ring slot
+// whose previous occupant has not even landed.  A parity wait is only exact
+// for the barrier's current phase or the one before, so the issuer first
+// waits until the loader has claimed the slot for ring index `idx` (after
+// the slot's previous tile was released, which implies it had landed); the
+// FULL barrier is then in the phase for `idx` or past it.  The loader
+// publishes the index with release semantics, the issuer reads it with
+// acquire semantics; the wait is bounded like mbar_wait_spin.
+__device__ __forceinline__ bool slot_claimed(uint32_t pos_addr, int idx, const WaitCtx &wc,
+                                             uint32_t role) {
+  if (ld_acquire_shared(pos_addr) == idx) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_shared(pos_addr) == idx) return true;
+    if ((it & 127u) == 0) {
+      if (*wc.abort) return false;
+      if (global_timer_ns() - t0 > wc.timeout_ns) {
+        *wc.abort = 1;
+        atomicOr(wc.status, kStatusTimeout | role);
+        return false;
+      }
+    }
+  }
+}
+
 // Bounded wait used while draining after an abort: ignores the abort flag.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,
                                                 const WaitCtx &wc) {
@@ -401,6 +492,27 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr,
   const uint32_t hi = ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
+
+// d = 64 (bf16, dense): the two O accumulators take only 128 of the 512
+// TMEM columns, so each tile's P gets 64 columns of its own instead of
+// overwriting S.  A tile's next S then needs only that its softmax has read
+// the last S out (S_FREE), not the P.V of it, so it is computed while the
+// softmax still works on the current one.  (Block-sparse units keep P over
+// S: with two different K lists, issuing a tile's next S ahead of its P.V
+// can leave each tile waiting on a slot the other still holds.)
+template <int D, bool FP8, bool SPARSE>
+constexpr bool kSplitP = (D == 64) && !FP8 && !SPARSE;
+
+// Which MMA role a variant runs.  Where P lies over S (d = 128, FP8) and
+// both tiles compute every K tile in step, one thread serves both tiles in
+// a fixed order (mma_role): each tile's next S goes out right behind its
+// P.V, which keeps the S -> softmax -> P.V chain short; two independent
+// issuers there interleave the tiles' MMAs in the tensor pipe and delay
+// every S (measured 22 % slower).  The split layout takes S off that chain,
+// and block-sparse pairs compute different K tiles, so those run one
+// issuing thread per Q tile (mma_role_tile).
+template <int D, bool FP8, bool SPARSE>
+constexpr bool kPerTileIssuer = SPARSE || kSplitP<D, FP8, SPARSE>;
 
 // ------------------------------------------------------------------ loader
 
@@ -429,13 +541,7 @@ __device__ __forceinline__ void producer_role(uint32_t base,
   for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
     const Unit w = get_unit<CAUSAL, SPARSE>(u, p);
     const int nt[2] = {w.n0, w.n1};
-    const uint8_t *srow = nullptr;
-    int kend = 0, kj = -1;  // block-sparse: the K tile of step j
-    if constexpr (SPARSE) {
-      const int tiles = (p.n + 127) >> 7, qt = w.q0 >> 7;
-      srow = sparse_row(p, w.bh, qt, tiles);
-      kend = CAUSAL ? qt + 1 : tiles;
-    }
+    KWalk<CAUSAL, SPARSE> walk(p, w);
     for (int t = 0; MODE != kLoadV && t < 2; ++t) {
       if (nt[t] == 0) continue;
       if (qocc[t] > 0) {
@@ -456,15 +562,20 @@ __device__ __forceinline__ void producer_role(uint32_t base,
       ++q_issued[t];
     }
     if (!ok) break;
-    const int nmax = max(nt[0], nt[1]);
-    for (int j = 0; j < nmax; ++j) {
-      if constexpr (SPARSE) kj = sparse_next(srow, kj + 1, kend);
-      else kj = j;
+    for (int j = 0; j < w.nu; ++j) {
+      int use;
+      const int kj = walk.next(use);
       if (MODE != kLoadV) {
         const int ks = k_issued % L::kKStages;
         ok = mbar_wait(bar(L::K_EMPTY + ks), ((k_issued / L::kKStages) & 1) ^ 1,
                        wc, kRoleProducer);
         if (!ok) break;
+        if constexpr (kPerTileIssuer<D, FP8, SPARSE>) {
+          // the slot's release takes one arrival per Q tile: give the one of
+          // a tile that does not compute with this K tile, then publish
+          st_release_shared(base + L::kSlotPos + 4 * ks, k_issued);
+          if (use != 3) mbar_arrive(bar(L::K_EMPTY + ks));
+        }
         mbar_arrive_expect_tx(bar(L::K_FULL + ks), L::kTileBytes);
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d_hint(base + L::kK + ks * L::kTileBytes + s * L::kPanelBytes,
@@ -478,6 +589,10 @@ __device__ __forceinline__ void producer_role(uint32_t base,
         ok = mbar_wait(bar(L::V_EMPTY + vs), ((v_issued / L::kVStages) & 1) ^ 1,
                        wc, kRoleProducer);
         if (!ok) break;
+        if constexpr (kPerTileIssuer<D, FP8, SPARSE>) {
+          st_release_shared(base + L::kSlotPos + 4 * (L::kKStages + vs), v_issued);
+          if (use != 3) mbar_arrive(bar(L::V_EMPTY + vs));
+        }
         mbar_arrive_expect_tx(bar(L::V_FULL + vs), L::kTileBytes);
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d_hint(base + L::kV + vs * L::kTileBytes + s * L::kPanelBytes,
@@ -661,6 +776,123 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
   mbar_wait_drain(bar(L::DRAIN), 0, wc);
 }
 
+// One MMA-issuing thread per Q tile (warp 9 for tile 0, warp 11 for tile 1),
+// each walking its own tile's steps in order with blocking waits, so that
+// neither tile's MMAs queue behind the other's barriers.  Per K tile j the
+// tile issues S_j = Q K_j^T and O += P_j V_j; P_j lies over S_j's columns,
+// so S_{j+1} follows P_j V_j in the same thread (the tensor pipe then reads
+// P_j before overwriting it), except in the split layout (dense units
+// only), where P has columns of its own and S_{j+1} goes out as soon as the
+// softmax has read S_j (S_FREE).  A K or V slot's EMPTY barrier counts one
+// arrival per Q tile: a tcgen05.commit from each tile that computes with
+// it, and one from the loader for a tile that does not.
+template <int D, bool CAUSAL, bool FP8, bool SPARSE>
+__device__ __forceinline__ void mma_role_tile(uint32_t base, uint32_t tmem,
+                                              const FwdParams &p, const WaitCtx &wc,
+                                              const int t) {
+  using L = Smem<D, FP8>;
+  constexpr bool kSplit = kSplitP<D, FP8, SPARSE>;
+  auto bar = [&](int i) { return base + L::kBars + 8u * i; };
+  const uint32_t tS = tmem + 128 * t;
+  const uint32_t tO = tmem + 256 + D * t;
+  const uint32_t tP = kSplit ? tmem + 256 + 2 * D + 64 * t : tS;
+  const uint32_t sQ = base + L::kQ + t * L::kTileBytes;
+  int qocc = 0, pcnt = 0, oocc = 0, sdone = 0;
+  int ring = 0;  // ring index of the unit's first K/V tile
+  bool ok = true;
+
+  for (int k = 0, u = unit_at<CAUSAL>(0); ok && u < p.num_units; u = unit_at<CAUSAL>(++k)) {
+    const Unit w = get_unit<CAUSAL, SPARSE>(u, p);
+    const int n = t ? w.n1 : w.n0;
+    if (n == 0) {  // nothing to compute in this unit
+      ring += w.nu;
+      continue;
+    }
+    KWalk<CAUSAL, SPARSE> walk(p, w);
+    int pos = -1;
+    // the place in the unit's K/V list of the next K tile this Q tile computes
+    auto step = [&]() {
+      int use;
+      do {
+        walk.next(use);
+        ++pos;
+      } while (!((use >> t) & 1) && pos < w.nu);
+      return pos;
+    };
+    auto issue_s = [&](int at, int j) -> bool {
+      if (kSplit && sdone > 0) {  // the softmax has read the previous S out
+        if (!mbar_wait_spin(bar(L::S_FREE + t), (sdone - 1) & 1, wc, kRoleMma)) return false;
+      }
+      const int ka = ring + at;
+      if (!slot_claimed(base + L::kSlotPos + 4 * (ka % L::kKStages), ka, wc, kRoleMma) ||
+          !mbar_wait_spin(bar(L::K_FULL + ka % L::kKStages), (ka / L::kKStages) & 1, wc,
+                          kRoleMma))
+        return false;
+      tc_fence_after_sync();
+      issue_qk<D, FP8>(tS, sQ, base + L::kK + (ka % L::kKStages) * L::kTileBytes);
+      mma_commit(bar(L::S_FULL + t));
+      if (j + 1 == n) mma_commit(bar(L::Q_EMPTY + t));  // last read of Q_t
+      mma_commit(bar(L::K_EMPTY + ka % L::kKStages));
+      ++sdone;
+      return true;
+    };
+
+    ok = mbar_wait_spin(bar(L::Q_FULL + t), qocc & 1, wc, kRoleMma);
+    ++qocc;
+    if (!ok) break;
+    int at = step(), nat = 0;
+    ok = issue_s(at, 0);
+    for (int j = 0; j < n && ok; ++j) {
+      if (kSplit && j + 1 < n) {
+        nat = step();
+        ok = issue_s(nat, j + 1);
+        if (!ok) break;
+      }
+      // O += P_j V_j: the first 64 keys once P_HALF, the rest once P_FULL
+      // (FP8: all at once); the unit's first P.V also waits for the previous
+      // unit's epilogue to read O out of TMEM
+      ok = mbar_wait_spin(bar((FP8 ? L::P_FULL : L::P_HALF) + t), pcnt & 1, wc, kRoleMma);
+      if (!ok) break;
+      const int va = ring + at;
+      ok = slot_claimed(base + L::kSlotPos + 4 * (L::kKStages + va % L::kVStages), va, wc,
+                        kRoleMma) &&
+           mbar_wait_spin(bar(L::V_FULL + va % L::kVStages), (va / L::kVStages) & 1, wc,
+                          kRoleMma);
+      if (!ok) break;
+      if (j == 0 && oocc > 0) {
+        ok = mbar_wait_spin(bar(L::O_EMPTY + t), (oocc - 1) & 1, wc, kRoleMma);
+        if (!ok) break;
+      }
+      tc_fence_after_sync();
+      const uint32_t vt = base + L::kV + (va % L::kVStages) * L::kTileBytes;
+      if constexpr (FP8) {
+        issue_pv<D, FP8>(tO, tP, vt, j > 0);
+      } else {
+        issue_pv<D, FP8, 0, 4>(tO, tP, vt, j > 0);
+        ok = mbar_wait_spin(bar(L::P_FULL + t), pcnt & 1, wc, kRoleMma);
+        if (!ok) break;
+        tc_fence_after_sync();
+        issue_pv<D, FP8, 4, 8>(tO, tP, vt, true);
+      }
+      ++pcnt;
+      mma_commit(bar(L::O_FULL + t));
+      mma_commit(bar(L::V_EMPTY + va % L::kVStages));
+      if (!kSplit && j + 1 < n) {
+        nat = step();
+        ok = issue_s(nat, j + 1);
+        if (!ok) break;
+      }
+      at = nat;
+    }
+    if (!ok) break;
+    ring += w.nu;
+    ++oocc;
+  }
+  // All tensor-core work (both issuers') must finish before TMEM is released.
+  mma_commit(bar(L::DRAIN));
+  mbar_wait_drain(bar(L::DRAIN), 0, wc);
+}
+
 // ------------------------------------------------------------------ softmax
 
 template <int D>
@@ -791,8 +1023,11 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
   const int wq = warp & 3;          // TMEM lane quarter of this warp
   const int r = wq * 32 + lane;     // query row within the tile
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  constexpr bool kSplit = kSplitP<D, FP8, SPARSE>;
   const uint32_t tS = lane_base + t * 128;
   const uint32_t tO = lane_base + 256 + t * D;
+  // where P goes: over S, or (split layout) its own 64 columns after O1
+  const uint32_t tP = kSplit ? lane_base + 256 + 2 * D + t * 64 : tS;
   const float cl2 = p.c_log2;
   int scnt = 0, ocnt = 0;
   bool ok = true;
@@ -802,7 +1037,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     const int n = t ? w.n1 : w.n0;
     const int qs = w.q0 + kBlockM * t;
     if constexpr (SPARSE) {
-      if (n == 0 && t == 0 && qs < p.n) {
+      if (n == 0 && qs < p.n) {
         // No K tile computed for these rows: every score is masked, and the
         // output is written as O = 0, lse = -inf (a reading: the softmax of
         // an empty row is undefined).
@@ -866,6 +1101,12 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
       }
       uint32_t s[4][32];
       load_scores(tS, s, mask, limit);
+      if constexpr (kSplit) {
+        // S is in registers: its columns may take the next S
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::S_FREE + t));
+      }
 
       // Row max and the lazy base update: the base only moves when some row
       // of the warp gains more than 2^8 (warp-uniform decision, per-row
@@ -900,9 +1141,21 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
         // that announcement: the P.V then adds to the rescaled O.  O holds
         // the earlier P.V products only; the S_FULL commit for this tile was
         // issued after the previous P.V, so that MMA has completed.
+        // In the split layout this tile's next S may have been issued
+        // before the last P.V, so that P.V is awaited here (O_FULL) before
+        // P's columns are overwritten or O rescaled.
         uint32_t pk[2][32];
         row_sum = exp_row<D, 0>(s, c, m_run, pk[0]);
-        tmem_st_32x32b_x32(tS + 0, pk[0]);
+        if constexpr (kSplit) {
+          if (j > 0) {
+            ok = mbar_wait(bar(L::O_FULL + t), ocnt & 1, wc, kRoleSoftmax);
+            ++ocnt;
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after_sync();
+          }
+        }
+        tmem_st_32x32b_x32(tP + 0, pk[0]);
         if (update) rescale_o<D>(tO, alpha);
         row_sum += exp_row<D, 1, 0, 8>(s, c, m_run, pk[1]);
         tmem_wait_st();
@@ -910,7 +1163,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::P_HALF + t));
         row_sum += exp_row<D, 1, 8, 32>(s, c, m_run, pk[1]);
-        tmem_st_32x32b_x32(tS + 32, pk[1]);
+        tmem_st_32x32b_x32(tP + 32, pk[1]);
       }
       l_run += row_sum;
       if constexpr (FP8) {
@@ -926,7 +1179,8 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
     if (!ok) break;
 
     // ---- epilogue: O / l -> bf16 -> this row of O in HBM; lse
-    ocnt += n;
+    // (the last P.V's O_FULL phase; the split layout has consumed the others)
+    ocnt += kSplit ? 1 : n;
     ok = mbar_wait(bar(L::O_FULL + t), (ocnt - 1) & 1, wc, kRoleEpilogue);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
@@ -1085,19 +1339,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(b0 + 8 * (L::S_FULL + t), 1);
       mbar_init(b0 + 8 * (L::P_FULL + t), 4);
       mbar_init(b0 + 8 * (L::P_HALF + t), 4);
+      mbar_init(b0 + 8 * (L::S_FREE + t), 4);
       mbar_init(b0 + 8 * (L::O_FULL + t), 1);
       mbar_init(b0 + 8 * (L::O_EMPTY + t), 4);
     }
-    mbar_init(b0 + 8 * L::DRAIN, 1);
+    // with one issuer per Q tile, both commit to DRAIN and to every EMPTY
+    const uint32_t issuers = kPerTileIssuer<D, FP8, SPARSE> ? 2 : 1;
+    mbar_init(b0 + 8 * L::DRAIN, issuers);
     for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(b0 + 8 * (L::K_FULL + s), 1);
-      mbar_init(b0 + 8 * (L::K_EMPTY + s), 1);
+      mbar_init(b0 + 8 * (L::K_EMPTY + s), issuers);
     }
     for (int s = 0; s < L::kVStages; ++s) {
       mbar_init(b0 + 8 * (L::V_FULL + s), 1);
-      mbar_init(b0 + 8 * (L::V_EMPTY + s), 1);
+      mbar_init(b0 + 8 * (L::V_EMPTY + s), issuers);
     }
     *abort_flag = 0;
+    for (int s = 0; s < L::kKStages + L::kVStages; ++s)
+      reinterpret_cast<volatile int *>(smem + L::kSlotPos)[s] = -1;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -1128,7 +1387,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0)
         producer_role<D, CAUSAL, kLoadV, FP8, SPARSE>(base, &tm_q, &tm_k, &tm_v, p, wc);
     } else if (warp == kMmaWarp) {
-      if (lane == 0) mma_role<D, CAUSAL, FP8, SPARSE>(base, tmem, p, wc);
+      if (lane == 0) {
+        if constexpr (kPerTileIssuer<D, FP8, SPARSE>)
+          mma_role_tile<D, CAUSAL, FP8, SPARSE>(base, tmem, p, wc, 0);
+        else
+          mma_role<D, CAUSAL, FP8, SPARSE>(base, tmem, p, wc);
+      }
+    } else if (warp == kMmaWarp2) {
+      if constexpr (kPerTileIssuer<D, FP8, SPARSE>) {
+        if (lane == 0) mma_role_tile<D, CAUSAL, FP8, SPARSE>(base, tmem, p, wc, 1);
+      }
     }
     __syncwarp();
   }

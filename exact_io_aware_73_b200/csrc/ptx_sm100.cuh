@@ -63,6 +63,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// 32-bit shared-memory store with release / load with acquire semantics at
+// CTA scope (a flag one thread publishes and another polls).
+__device__ __forceinline__ void st_release_shared(uint32_t addr, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_shared(uint32_t addr) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // Same probe, but the thread may sleep (not issuing) until the phase
 // completes or about `hint_ns` nanoseconds pass.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar,
