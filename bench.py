@@ -478,7 +478,7 @@ def cpu_baseline_fp8(w, qkv, signs, budget_s: float, seed: int = 13):
         t1 = time.perf_counter()
         oracle.attention_fp8_rows(z["q8"], z["qs"], z["k8"], z["ks"], z["v8"],
                                   z["vs"], w.causal, scale_qk, rows,
-                                  threads=threads)
+                                  threads=threads, tau=oracle.FP8_KERNEL_TAU)
         dt = time.perf_counter() - t1
         elapsed += dt
         rows_done += batch

@@ -56,11 +56,12 @@
 // K tile, one per head for V).  Both GEMMs run as tcgen05.mma kind::f8f6f4
 // (K = 32 per instruction, 128-byte rows = one swizzle panel at d = 128).  The
 // score multiplier scale * log2(e) * q_scale * k_scale changes per K tile;
-// the running max is exact (every increase rescales O), and P is carried as
-// 2^(x - m + 8) <= 256 so that E4M3's smallest code still reaches 2^-17 of
-// the row maximum; P goes to TMEM as four E4M3 bytes per column.  The row
-// sum adds the unrounded P; V's per-head scale multiplies the output in the
-// epilogue and lse subtracts the 2^8 again.
+// a row's base m moves only when its tile maximum exceeds it by more than
+// 2^4, and P is carried as 2^(x - m + 4) <= 256, so that every probability
+// down to 2^-10 of the row maximum is an E4M3 normal number; P goes to TMEM
+// as four E4M3 bytes per column.  The row sum adds the unrounded P; V's
+// per-head scale multiplies the output in the epilogue and lse subtracts the
+// 2^4 again.
 #pragma once
 
 #include <cstdint>
@@ -90,6 +91,12 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchR
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P <= 2^8
+// FP8: a row's base moves when its tile maximum exceeds it by more than
+// kFp8Threshold; P = 2^(x - m + kFp8Offset) then stays <= 2^8 (E4M3 holds up
+// to 448), and every p >= 2^-(14 - kFp8Threshold) of the row maximum is an
+// E4M3 normal number.
+constexpr float kFp8Threshold = 4.0f;
+constexpr float kFp8Offset = 8.0f - kFp8Threshold;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Device status word bits.
@@ -976,8 +983,8 @@ __device__ __forceinline__ float exp_row(const uint32_t (&s)[4][32], float cl2,
   return (a0 + a1) + (b0 + b1);
 }
 
-// FP8 version of exp_row: p = 2^(s * c - m) (m already lowered by 8, so
-// p <= 256), row sum of the unrounded p, and four E4M3 codes per 32-bit
+// FP8 version of exp_row: p = 2^(s * c - m) (m already lowered by
+// kFp8Offset, so p <= 256), row sum of the unrounded p, and four E4M3 codes per 32-bit
 // column for the P.V MMA (key 4c in the lowest byte of column c).
 __device__ __forceinline__ float exp_row_fp8(const uint32_t (&s)[4][32], float c,
                                              float m, uint32_t (&pk)[32]) {
@@ -1112,16 +1119,26 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
       // of the warp gains more than 2^8 (warp-uniform decision, per-row
       // values); P then stays below 256 and O / l is unchanged because m and
       // l always move together.  The first tile of a row sets the base.
-      // FP8 keeps the exact running max (threshold 0): with P in E4M3 the
-      // base fixes which probabilities fall below the smallest code.
+      // FP8: the base of a row moves when its own tile maximum exceeds it by
+      // more than kFp8Threshold (a per-row decision, so each row's base is a
+      // function of that row alone); the warp rescales O when any row moved,
+      // the others by exactly 1.
       const float m_tile = row_max_raw(s) * c;
       float alpha = 1.f;
       bool update = false;
       if (j == 0) {
         m_run = m_tile;
+      } else if constexpr (FP8) {
+        const bool mine = m_tile > m_run + kFp8Threshold;
+        update = __any_sync(0xffffffffu, mine);
+        if (update) {
+          const float m_new = mine ? m_tile : m_run;
+          alpha = ex2_approx(m_run - m_new);
+          l_run *= alpha;
+          m_run = m_new;
+        }
       } else {
-        update = __any_sync(0xffffffffu,
-                            m_tile > m_run + (FP8 ? 0.f : kRescaleThreshold));
+        update = __any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold);
         if (update) {
           const float m_new = fmaxf(m_run, m_tile);
           alpha = ex2_approx(m_run - m_new);
@@ -1132,7 +1149,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
       float row_sum;
       if constexpr (FP8) {
         uint32_t pk[32];
-        row_sum = exp_row_fp8(s, c, m_run - 8.f, pk);
+        row_sum = exp_row_fp8(s, c, m_run - kFp8Offset, pk);
         tmem_st_32x32b_x32(tS + 0, pk);
       } else {
         // The first half's P is stored while the second half is computed,
@@ -1199,7 +1216,7 @@ __device__ __forceinline__ void softmax_role(uint32_t base, uint32_t tmem,
                         in_bounds(qs, p.n, p.status) &&
                         in_bounds(grow, static_cast<int64_t>(p.bh) * p.n, p.status);
     // this block's log-sum-exp (natural log)
-    const float lse_this = (m_run - (FP8 ? 8.f : 0.f) + lg2_approx(l_run)) * kLn2;
+    const float lse_this = (m_run - (FP8 ? kFp8Offset : 0.f) + lg2_approx(l_run)) * kLn2;
     float lse_out = lse_this;
     if (p.merge_mode == kMergeNone) {
       // The row of O leaves TMEM first, so that its columns go back to the

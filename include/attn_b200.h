@@ -257,11 +257,14 @@ int attn_fwd_host_noalloc(const void *q, const void *k, const void *v,
  *              [B, H]).
  *   attention  O = softmax(scale_qk * Qhat Khat^T [causal mask]) Vhat on the
  *              dequantized operands (Qhat = codes * scale, ...), computed as
- *              the blocked online softmax in 128-key blocks with an exact
- *              running maximum m (log2 units): P = 2^(x - m + 8) <= 256 is
- *              rounded to E4M3 for the P.V product, the row sum adds the
- *              unrounded P, and lse = ln(sum_j exp(scale_qk Qhat_i . Khat_j))
- *              (fp32, natural log) -- independent of the rounding of P.
+ *              the blocked online softmax in 128-key blocks with a running
+ *              base m (log2 units) per row that moves to the block maximum
+ *              only when that exceeds it by more than 4: P = 2^(x - m + 4)
+ *              <= 256 is rounded to E4M3 for the P.V product (every
+ *              probability down to 2^-10 of the row maximum is then an E4M3
+ *              normal number), the row sum adds the unrounded P, and
+ *              lse = ln(sum_j exp(scale_qk Qhat_i . Khat_j)) (fp32, natural
+ *              log) -- independent of the rounding of P.
  * The three entries exist for head dimension d = 128 only (at d = 64 the
  * exponentials, not the tensor cores, bound the forward, and FP8 buys
  * nothing); other d give ATTN_ERR_UNSUPPORTED_HEAD_DIM.

@@ -32,6 +32,7 @@ from .oracle import (  # noqa: F401
     fp8_quantize,
     attention_fp8,
     attention_fp8_rows,
+    FP8_KERNEL_TAU,
     quantize_qkv_fp8,
     attention_decode,
     attention_decode_rows_bf16,

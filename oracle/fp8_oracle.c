@@ -30,11 +30,14 @@
  *     the P.V sum);
  *   * the attention itself is the blocked online softmax of [MM] "Algoritma
  *     Flash Attention" over the dequantized operands, key blocks of Bc = 128,
- *     with an exact running maximum m (natural-log units) and the block's
- *     probabilities carried as p = 256 * exp(s - m) (<= 256 < 448), rounded
- *     to fp32 and then to E4M3 before they multiply V (the FP8 P.V product);
- *     the row sum l adds the unrounded p; O = acc / l and
- *     lse = m + ln(l) - 8 ln 2.
+ *     with a running base m (natural-log units) per row: the first block's
+ *     maximum, then a later block's maximum mb whenever (mb - m) / ln 2
+ *     exceeds tau (tau = 0: the exact running maximum).  The block's
+ *     probabilities are carried as p = 2^(8 - tau) exp(s - m) (<= 256 <
+ *     448), rounded to fp32 and then to E4M3 before they multiply V (the
+ *     FP8 P.V product); the row sum l adds the unrounded p; O = acc / l and
+ *     lse = m + ln(l) - (8 - tau) ln 2.  Bc, tau and the 2^(8 - tau) are the
+ *     kernel's choices, not the pages'.
  *
  * Arithmetic is IEEE double except where a rounding step is part of the
  * method (fp32 before E4M3).  Layouts: codes are row-major [BH, N, d] bytes;
@@ -217,12 +220,20 @@ static void boundary_distance(double p, double *rel_dist, double *step) {
  * [N, d]; qhat: the row's dequantized query.  If flip_delta > 0, *flip_bound
  * receives sum over keys whose p lies within relative flip_delta of an E4M3
  * rounding boundary of (code spacing) * max_t |Vhat[key, t]|, divided by l:
- * the most a one-step change of those codes can move any output of the row. */
+ * the most a one-step change of those codes can move any output of the row.
+ * A relative error flip_delta in p is an error of flip_delta / ln 2 in the
+ * exponent (log2 units), so when a base decision (block gap against tau)
+ * lies within twice that of tau, a kernel computing the scores in fp32 may
+ * decide it the other way and carry every later p of the row on another
+ * base: *flip_bound is then +infinity (the row's codes are not predicted). */
 static void fp8_row(const double *qhat, const double *Khat, const double *Vhat,
                     int64_t N, int64_t d, int64_t i, int causal, double scale,
-                    int64_t Bc, double *s, double *acc, double *orow,
+                    int64_t Bc, double tau, double *s, double *acc, double *orow,
                     double *lse, double flip_delta, double *flip_bound) {
+  const double ln2 = log(2.0);
+  const double offset = exp2(8.0 - tau);
   double m = -INFINITY, l = 0.0, flip = 0.0;
+  int ambiguous = 0;
   for (int64_t t = 0; t < d; ++t) acc[t] = 0.0;
   const int64_t kend = causal ? i + 1 : N;
   for (int64_t k0 = 0; k0 < kend; k0 += Bc) {
@@ -235,16 +246,29 @@ static void fp8_row(const double *qhat, const double *Khat, const double *Vhat,
       s[c - k0] = scale * dot;
       if (s[c - k0] > mb) mb = s[c - k0];
     }
-    /* exact running maximum; rescale what was accumulated */
-    const double mnew = (m > mb) ? m : mb;
-    const double alpha = (m == -INFINITY) ? 0.0 : exp(m - mnew);
-    l *= alpha;
-    flip *= alpha;
-    for (int64_t t = 0; t < d; ++t) acc[t] *= alpha;
-    m = mnew;
-    /* p = 256 exp(s - m); l adds p; the P.V product uses E4M3(fp32(p)) */
+    /* the base: the first block's maximum, later a block maximum that
+       exceeds it by more than tau (log2 units); rescale what was
+       accumulated */
+    if (m == -INFINITY) {
+      m = mb;
+    } else {
+      const double gap = (mb - m) / ln2;
+      /* (at tau = 0 the two choices of a near tie are nearly the same base,
+         which the flip bound covers) */
+      if (flip_delta > 0.0 && tau > 0.0 && fabs(gap - tau) <= 2.0 * flip_delta / ln2)
+        ambiguous = 1;
+      if (gap > tau) {
+        const double alpha = exp(m - mb);
+        l *= alpha;
+        flip *= alpha;
+        for (int64_t t = 0; t < d; ++t) acc[t] *= alpha;
+        m = mb;
+      }
+    }
+    /* p = 2^(8 - tau) exp(s - m); l adds p; the P.V product uses
+       E4M3(fp32(p)) */
     for (int64_t c = k0; c < k1; ++c) {
-      const double p = 256.0 * exp(s[c - k0] - m);
+      const double p = offset * exp(s[c - k0] - m);
       l += p;
       const double pq = oracle_e4m3_decode(oracle_e4m3_encode((float)p));
       for (int64_t t = 0; t < d; ++t) acc[t] += pq * Vhat[c * d + t];
@@ -261,8 +285,8 @@ static void fp8_row(const double *qhat, const double *Khat, const double *Vhat,
     }
   }
   for (int64_t t = 0; t < d; ++t) orow[t] = acc[t] / l;
-  *lse = m + log(l) - 8.0 * log(2.0);
-  if (flip_bound) *flip_bound = flip / l;
+  *lse = m + log(l) - (8.0 - tau) * ln2;
+  if (flip_bound) *flip_bound = ambiguous ? INFINITY : flip / l;
 }
 
 static void dequant_head(const uint8_t *codes, const double *scales, int64_t N,
@@ -283,11 +307,12 @@ int oracle_attention_fp8_rows(const uint8_t *q8, const double *q_scale,
                               const uint8_t *v8, const double *v_scale,
                               int64_t BH, int64_t N, int64_t d, int causal,
                               double scale, int64_t q_block, int64_t k_block,
-                              int64_t Bc, const int64_t *rows, int64_t nrows,
+                              int64_t Bc, double tau, const int64_t *rows, int64_t nrows,
                               double *O, double *lse, double flip_delta,
                               double *flip_bound, int threads) {
   if (!q8 || !q_scale || !k8 || !k_scale || !v8 || !v_scale || !rows || !O ||
-      !lse || BH < 1 || N < 1 || d < 1 || q_block < 1 || k_block < 1 || Bc < 1)
+      !lse || BH < 1 || N < 1 || d < 1 || q_block < 1 || k_block < 1 || Bc < 1 ||
+      !(tau >= 0.0 && tau <= 8.0))
     return FP8_EBADARG;
   for (int64_t r = 0; r < nrows; ++r)
     if (rows[r] < 0 || rows[r] >= BH * N) return FP8_EBADARG;
@@ -329,7 +354,7 @@ int oracle_attention_fp8_rows(const uint8_t *q8, const double *q_scale,
           const double qs = q_scale[bh * qblocks + i / q_block];
           for (int64_t t = 0; t < d; ++t)
             qhat[t] = oracle_e4m3_decode(q8[rows[r] * d + t]) * qs;
-          fp8_row(qhat, Khat, Vhat, N, d, i, causal, scale, Bc, s, acc,
+          fp8_row(qhat, Khat, Vhat, N, d, i, causal, scale, Bc, tau, s, acc,
                   O + r * d, lse + r, flip_delta, flip_bound ? flip_bound + r : NULL);
         }
       }

@@ -72,8 +72,8 @@ def _load():
                                             i8p, i64, u8p, dp]
         lib.oracle_attention_fp8_rows.argtypes = [
             u8p, dp, u8p, dp, u8p, dp, i64, i64, i64, ctypes.c_int,
-            ctypes.c_double, i64, i64, i64, i64p, i64, dp, dp, ctypes.c_double,
-            dp, ctypes.c_int]
+            ctypes.c_double, i64, i64, i64, ctypes.c_double, i64p, i64, dp, dp,
+            ctypes.c_double, dp, ctypes.c_int]
         for f in (lib.oracle_e4m3_encode_array, lib.oracle_hadamard_rotate,
                   lib.oracle_fp8_quantize, lib.oracle_attention_fp8_rows):
             f.restype = ctypes.c_int
@@ -331,12 +331,20 @@ def fp8_quantize(bits, rotate: bool, signs=None, block_rows: int = 128):
     return codes, scales
 
 
+# The base threshold of the FP8 kernel (log2 units): a row's base moves to a
+# block maximum only when that exceeds it by more than this.
+FP8_KERNEL_TAU = 4.0
+
+
 def attention_fp8_rows(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
                        scale: float, rows, block: int = 128, flip_delta=0.0,
-                       threads=None):
+                       threads=None, tau=0.0):
     """FP8 attention on codes [.., N, d] for flat rows (bh * N + i); Q and K
-    scales per `block` rows, V one scale per head.  Returns (O, lse,
-    flip_bound) with flip_bound None unless flip_delta > 0."""
+    scales per `block` rows, V one scale per head; the base of a row moves
+    when a block maximum exceeds it by more than `tau` (log2 units; 0: the
+    exact running maximum).  Returns (O, lse, flip_bound) with flip_bound
+    None unless flip_delta > 0 (+inf for a row with a base decision within
+    the score error of tau)."""
     q8, k8, v8 = (np.ascontiguousarray(a, dtype=np.uint8) for a in (q8, k8, v8))
     N, d = q8.shape[-2], q8.shape[-1]
     BH = q8.size // (N * d)
@@ -348,7 +356,7 @@ def attention_fp8_rows(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
     _check(_load().oracle_attention_fp8_rows(
         _u8ptr(q8), _dptr(qs), _u8ptr(k8), _dptr(ks), _u8ptr(v8), _dptr(vs),
         BH, N, d, int(bool(causal)), float(scale), int(block), int(block), 128,
-        rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.size,
+        float(tau), rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.size,
         _dptr(O), _dptr(lse), float(flip_delta),
         _dptr(fb) if fb is not None else None, _threads(threads)),
         "attention_fp8_rows")
@@ -356,14 +364,15 @@ def attention_fp8_rows(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
 
 
 def attention_fp8(q8, q_scale, k8, k_scale, v8, v_scale, causal: bool,
-                  scale: float, block: int = 128, flip_delta=0.0, threads=None):
+                  scale: float, block: int = 128, flip_delta=0.0, threads=None,
+                  tau=0.0):
     """attention_fp8_rows over every row; O shaped like the codes."""
     shape = q8.shape
     N, d = shape[-2], shape[-1]
     rows = np.arange(q8.size // d, dtype=np.int64)
     O, lse, fb = attention_fp8_rows(q8, q_scale, k8, k_scale, v8, v_scale,
                                     causal, scale, rows, block, flip_delta,
-                                    threads)
+                                    threads, tau)
     return (O.reshape(shape), lse.reshape(shape[:-1]),
             None if fb is None else fb.reshape(shape[:-1]))
 

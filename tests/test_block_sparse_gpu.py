@@ -100,6 +100,43 @@ def test_empty_mask_gives_zero_and_minus_infinity():
     assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
 
 
+def _mask_patterns(T):
+    """Masks whose pairs of consecutive query tiles keep very different key
+    tiles: alternating parity (disjoint lists), one tile keeping only the
+    last key tile while its partner keeps all, and the first tile of every
+    pair keeping nothing."""
+    kj = np.arange(T)
+    alt = ((kj[None, :] % 2) == (np.arange(T)[:, None] % 2)).astype(np.uint8)
+    lone = np.ones((T, T), np.uint8)
+    lone[0::2, :] = 0
+    lone[0::2, T - 1] = 1
+    first_empty = np.ones((T, T), np.uint8)
+    first_empty[0::2, :] = 0
+    return {"alternating": alt, "lone_last": lone, "first_empty": first_empty}
+
+
+@pytest.mark.parametrize("pattern", ["alternating", "lone_last", "first_empty"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(2048, 64), (1900, 128)])
+def test_pairs_with_different_key_lists(oracle_mod, pattern, causal, N, d):
+    """A unit is two consecutive query tiles that load the union of their
+    lists; each computes only its own key tiles (one issuing thread per
+    tile), so these masks make the tiles of a pair skip many of the ring's
+    slots."""
+    w = W.shape_case(1, 2, N, d, causal, seed=500 + N + d)
+    q, k, v = W.make_qkv(w)
+    T = (N + 127) // 128
+    m = torch.from_numpy(_mask_patterns(T)[pattern])
+    o, lse = attn.attn_fwd_block_sparse(q.cuda(), k.cuda(), v.cuda(), m.cuda(),
+                                        causal=causal, scale=w.scale)
+    assert attn.status() == 0
+    bits = [oracle_mod.bf16_bits(t) for t in (q, k, v)]
+    o_ref, l_ref = oracle_mod.attention_block_sparse_bf16(*bits, causal, w.scale,
+                                                          m.numpy())
+    _compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref,
+             f"{pattern} {w.name}")
+
+
 @pytest.mark.parametrize("name", sorted(W.SPARSE_WORKLOADS))
 def test_block_sparse_workloads_sampled_rows(oracle_mod, name):
     """The benchmark's block-sparse workloads, in the launch the benchmark

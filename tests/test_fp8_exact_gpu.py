@@ -19,14 +19,17 @@ Per output element (row i, column t), with p_j the exact probabilities of
 row i (normalised so that the row maximum is 1) and l = sum_j p_j:
 
   * E4M3 keeps 3 mantissa bits: any value in its normal range is stored
-    with relative error <= 2^-4.  Under any fixed scaling of a row, the
-    normal range reaches at most 2^-14 below the row's largest probability
-    (largest normal binade 2^8, smallest 2^-6).  So every p_j >= 2^-14 is
-    carried within 2^-4 p_j, and a smaller one is off by at most p_j
-    (subnormal or flushed to zero):
+    with relative error <= 2^-4.  The kernel carries a row's probabilities
+    on a base that lags the row's running maximum by at most tau = 4 (log2
+    units) and keeps the largest below 2^8 (the format's top binade holds up
+    to 448), so its largest probability lies between 2^(8 - tau) and 2^8,
+    and the normal range (down to 2^-6) reaches at least 2^-(14 - tau) =
+    2^-10 below it.  This is the error contract of the threshold: every
+    p_j >= 2^-(14 - tau) is carried within 2^-4 p_j, and a smaller one is
+    off by at most p_j (subnormal or flushed to zero):
         |O - O*| <= 2^-4 A + U,
         A = sum_j p_j |v_jt| / l           (exact attention on |V^|)
-        U = sum_{p_j < 2^-14} p_j |v_jt| / l.
+        U = sum_{p_j < 2^-(14 - tau)} p_j |v_jt| / l.
   * The scores come from fp32 sums of exact E4M3 products; with the fp32
     multiplier, the FMA and ex2.approx that gives a relative error delta in
     every p before it is encoded (delta as in test_fp8_gpu.py): 2 delta A
@@ -51,7 +54,8 @@ pytestmark = pytest.mark.gpu
 D = 128
 LOG2E = 1.4426950408889634
 E4M3_REL = 2.0 ** -4          # half the relative step of 3 mantissa bits
-E4M3_RANGE = 2.0 ** -14       # smallest normal binade / largest binade
+TAU = 4.0                     # the kernel's base threshold (log2 units)
+E4M3_RANGE = 2.0 ** -(14 - TAU)  # normal range below the row maximum
 
 
 @pytest.fixture(scope="module", autouse=True)

@@ -17,8 +17,15 @@ The attention is floating point.  Tolerance, derived from the arithmetic
     accumulation of exact E4M3 products (<= 2^-20 of sum |q_t k_t| per dot
     product, for the score and for the running max), the fp32 rounding of
     the multiplier and of the FMA (2^-22 of |x|), and ex2.approx (2^-21).
-    The oracle reports per row the most those one-step changes can move an
-    output (flip_bound: code spacing x max|V| / l summed over such keys);
+    The oracle reports per row the most those
+    one-step changes can move an output (flip_bound: code spacing x max|V|
+    / l summed over such keys);
+  * the kernel moves a row's base only when a key block's maximum exceeds
+    it by more than tau = 4 (log2 units; the oracle runs the same rule); a
+    row where some block's gap lies within the score error of tau could be
+    decided the other way in fp32, so the oracle gives it an infinite flip
+    bound and the comparison here skips it (test_fp8_exact_gpu.py still
+    bounds it against exact attention);
   * bf16 rounding of the stored output: 2^-8 of |O| (twice the half-ulp);
   * fp32 accumulation of P.V and l: (keys / 32 + 16) x 2^-24 x max|V|.
 lse is independent of P's rounding: |lse - lse_ref| <= 1e-4 (1 + |lse_ref|).
@@ -36,6 +43,7 @@ pytestmark = pytest.mark.gpu
 
 D = 128
 LOG2E = 1.4426950408889634
+EXP2_REL = 2.0 ** -21   # ex2.approx
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -81,12 +89,15 @@ def _flip_delta(oracle_mod, z, scale_qk, causal):
             A = np.tril(A)
             S = np.tril(S)
         worst = max(worst, 2 * 2.0 ** -20 * A.max() * c + 2.0 ** -22 * 2 * np.abs(S).max() * c)
-    return math.log(2.0) * worst + 2.0 ** -21
+    return math.log(2.0) * worst + EXP2_REL
 
 
 def _compare(got_o, got_lse, ref_o, ref_lse, flip, vmax, nkeys, what):
     got_o = got_o.reshape(ref_o.shape)
     got_lse = got_lse.reshape(ref_lse.shape)
+    # rows whose base decision the oracle cannot predict (infinite flip
+    # bound) are left to the exact-attention bound; they must stay rare
+    assert np.isinf(flip).mean() <= 0.01, f"{what}: {np.isinf(flip).sum()} undecided rows"
     assert np.all(np.isfinite(got_o)) and np.all(np.isfinite(got_lse)), what
     tol = (flip.reshape(ref_lse.shape)[..., None] + 2.0 ** -8 * np.abs(ref_o)
            + (nkeys / 32 + 16) * 2.0 ** -24 * vmax)
@@ -153,7 +164,7 @@ def test_fp8_forward_parity(oracle_mod, B, H, N, causal):
     delta = _flip_delta(oracle_mod, z, scale_qk, causal)
     O_ref, l_ref, flip = oracle_mod.attention_fp8(
         z["q8"], z["qs"], z["k8"], z["ks"], z["v8"], z["vs"], causal, scale_qk,
-        flip_delta=delta)
+        flip_delta=delta, tau=oracle_mod.FP8_KERNEL_TAU)
     vmax = float(np.abs(oracle_mod.e4m3_decode(z["v8"])).max() * z["vs"].max())
     # the whole path from bf16
     o, lse = attn.attn_fwd_fp8(q.cuda(), k.cuda(), v.cuda(), causal=causal,
@@ -182,7 +193,7 @@ def test_fp8_naive_path_parity(oracle_mod):
     delta = _flip_delta(oracle_mod, z, scale32, True)
     O_ref, l_ref, flip = oracle_mod.attention_fp8(
         z["q8"], z["qs"], z["k8"], z["ks"], z["v8"], z["vs"], True, scale32,
-        flip_delta=delta)
+        flip_delta=delta, tau=oracle_mod.FP8_KERNEL_TAU)
     vmax = float(np.abs(oracle_mod.e4m3_decode(z["v8"])).max() * z["vs"].max())
     o, lse = attn.attn_fwd_fp8(q.cuda(), k.cuda(), v.cuda(), causal=True,
                                scale=scale32, signs=None)
@@ -192,7 +203,7 @@ def test_fp8_naive_path_parity(oracle_mod):
 
 
 def test_zero_queries_average_values_on_gpu(oracle_mod):
-    """Q = 0: every probability is 2^8 exactly (no rounding anywhere), so O is
+    """Q = 0: every probability is 2^4 exactly (no rounding anywhere), so O is
     the mean of the dequantized V rows (prefix mean when causal)."""
     N = 300
     w, _, k, v, signs = _case(1, 1, N, False, seed=91)
@@ -263,10 +274,10 @@ def test_fp8_full_size_sampled_rows(oracle_mod, causal):
         S = qh @ kh.T
         c = scale_qk * LOG2E
         delta = math.log(2.0) * (2 * 2.0 ** -20 * A.max() * c +
-                                 2.0 ** -22 * 2 * np.abs(S).max() * c) + 2.0 ** -21
+                                 2.0 ** -22 * 2 * np.abs(S).max() * c) + EXP2_REL
         O_ref, l_ref, flip = oracle_mod.attention_fp8_rows(
             z["q8"], z["qs"], z["k8"], z["ks"], z["v8"], z["vs"], causal,
-            scale_qk, rows, flip_delta=delta)
+            scale_qk, rows, flip_delta=delta, tau=oracle_mod.FP8_KERNEL_TAU)
         vmax = float(np.abs(oracle_mod.e4m3_decode(z["v8"])).max() * z["vs"].max())
         _compare(o[0, h, rows], lse[0, h, rows], O_ref, l_ref, flip, vmax, w.N,
                  f"{w.name} causal={causal} head {h}")

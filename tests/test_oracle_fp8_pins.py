@@ -311,3 +311,66 @@ def test_rotation_lowers_fp8_error_with_outlier_channels(oracle_mod):
     plain0, rotated0 = errs(False)
     assert 0.8 < plain0 / rotated0 < 1.25
     assert rotated < 0.08 and rotated0 < 0.08
+
+
+# ------------------------------------------------------------ lazy base
+
+def _attend_log2_scores(oracle_mod, scores, v, tau):
+    """FP8 oracle on one query whose scores (log2 units) against the keys are
+    `scores` (scale ln 2, q = e0, k[:, 0] = scores), values v [N, d]."""
+    N, d = len(scores), v.shape[1]
+    q = np.zeros((1, 1, d))
+    q[0, 0, 0] = 1.0
+    k = np.zeros((1, N, d))
+    k[0, :, 0] = scores
+    q8, k8, v8 = (_codes_from_values(oracle_mod, a) for a in (q, k, v[None]))
+    tiles = -(-N // 128)
+    # the query is row 0 of a one-row problem: pad Q to N rows of zeros
+    q8 = np.concatenate([q8, np.zeros((1, N - 1, d), np.uint8)], axis=1)
+    O, lse, _ = oracle_mod.attention_fp8_rows(
+        q8, np.ones((1, tiles)), k8, np.ones((1, tiles)), v8, [1.0], False,
+        math.log(2.0), [0], tau=tau)
+    return O[0], lse[0]
+
+
+@pytest.mark.parametrize("tau", [0.0, 4.0])
+def test_probability_offset_follows_the_threshold(oracle_mod, tau):
+    """p = 2^(8 - tau) exp(s - m): two keys at 0 and -14 (log2 units) below
+    the base.  With tau = 0 the small one is 2^-6, an exact E4M3 normal; with
+    tau = 4 it is 2^-10, half the smallest subnormal, which rounds to even:
+    0.  lse adds the unrounded p either way."""
+    v = np.array([[0.0, 1.0], [1.0, 0.0]])
+    O, lse = _attend_log2_scores(oracle_mod, [0.0, -14.0], v, tau)
+    want = 2.0 ** -14 / (1 + 2.0 ** -14) if tau == 0 else 0.0
+    assert O[0] == pytest.approx(want, rel=1e-14, abs=0)
+    assert O[1] == pytest.approx(1 / (1 + 2.0 ** -14), rel=1e-14)
+    assert lse == pytest.approx(math.log1p(2.0 ** -14), rel=1e-12)
+
+
+@pytest.mark.parametrize("tau", [0.0, 4.0])
+def test_base_moves_only_past_the_threshold(oracle_mod, tau):
+    """Three key blocks whose maxima are 0, 3 and 8 (log2 units).  With
+    tau = 4 the base stays at 0 through the second block (gap 3) and moves
+    to 8 at the third (gap 8); every p is then a power of two that E4M3
+    holds exactly: 16 and 2^-9 in the first two blocks (the key at -13), 16
+    in the third.  So the result equals exact attention; a base that moved
+    at gap 3 would flush the -13 key (2^-12 -> 0), one that stayed at gap 8
+    would saturate (2^12 -> 448).  tau = 0 is exact as well (256, 2^-8)."""
+    N = 384
+    scores = np.full(N, -30.0)
+    v = np.zeros((N, 4))
+    for col, (key, sc) in enumerate([(0, 0.0), (128, 3.0), (129, -13.0), (256, 8.0)]):
+        scores[key] = sc
+        v[key, col] = 1.0
+    O, lse = _attend_log2_scores(oracle_mod, scores, v, tau)
+    w = np.exp2(scores)
+    exact = (w @ v) / w.sum()
+    np.testing.assert_allclose(O, exact, rtol=1e-13, atol=0)
+    assert lse == pytest.approx(math.log(w.sum()) * 1.0, rel=1e-13)
+
+
+def test_kernel_threshold_is_within_e4m3_range(oracle_mod):
+    """The kernel's threshold keeps p <= 2^8 < 448 and the normal range at
+    2^-(14 - tau) of the row maximum."""
+    assert 0 < oracle_mod.FP8_KERNEL_TAU <= 8
+    assert 2.0 ** 8 < 448

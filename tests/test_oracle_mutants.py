@@ -72,8 +72,14 @@ FP8_MUTANTS = {
                         "(popcount_u32((uint32_t)(a | t)) & 1)"),
     "fp8_scale_half_range": ("while (ldexp(amax, e) > E4M3_MAX) --e;",
                              "while (ldexp(amax, e) > E4M3_MAX / 2) --e;"),
-    "fp8_no_probability_offset": ("const double p = 256.0 * exp(s[c - k0] - m);",
+    "fp8_no_probability_offset": ("const double p = offset * exp(s[c - k0] - m);",
                                   "const double p = exp(s[c - k0] - m);"),
+    "fp8_offset_ignores_threshold": ("const double offset = exp2(8.0 - tau);",
+                                     "const double offset = 256.0;"),
+    "fp8_base_ignores_threshold": ("if (gap > tau) {", "if (gap > 0.0) {"),
+    "fp8_base_never_moves": ("if (gap > tau) {", "if (gap > tau + 8.0) {"),
+    "fp8_lse_offset_fixed": ("*lse = m + log(l) - (8.0 - tau) * ln2;",
+                             "*lse = m + log(l) - 8.0 * ln2;"),
     "fp8_sum_of_rounded_p": ("      l += p;\n",
                              "      l += oracle_e4m3_decode(oracle_e4m3_encode((float)p));\n"),
     "fp8_no_output_rescale": ("for (int64_t t = 0; t < d; ++t) acc[t] *= alpha;", ""),
