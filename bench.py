@@ -25,6 +25,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -123,9 +124,21 @@ def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
 
 # The exponential roof: the softmax evaluates one exp2 per visible score, B H
 # N^2 of them (halved under the causal mask, the FLOP convention's count), on
-# the MUFU unit at 16 per clock per SM.  The d = 64 kernel evaluates a quarter
-# of them on the FMA pipe instead, so its MUFU share is 3/4 of the count.
+# the MUFU unit at 16 per clock per SM.  The kernel evaluates a fixed share of
+# them (pairs out of every 8, per head dimension, read from its source) on
+# the FMA pipe instead.
 MUFU_EX2_PER_CLK_PER_SM = 16
+
+
+def fma_pipe_pairs_per8(d: int) -> int:
+    """Pairs of exponentials out of 8 that the forward kernel evaluates on
+    the FMA pipe at head dimension d (its ATTN_EXP2_EMU_PER8_D<d> default)."""
+    with open(os.path.join(CSRC, "attn_fwd_kernel.cuh"), encoding="utf-8") as fh:
+        src = fh.read()
+    m = re.search(r"#define ATTN_EXP2_EMU_PER8_D%d (\d+)" % d, src)
+    if m is None:
+        raise RuntimeError(f"no exponential split for d = {d} in the kernel source")
+    return int(m.group(1))
 DEFAULT_SM_MHZ = 1965.0
 
 
@@ -144,7 +157,7 @@ def exp_roof(flops: float, d: int, ms_per_step: float, sm_count: int,
             "peak_basis": (f"{MUFU_EX2_PER_CLK_PER_SM} ex2 per clock per SM x "
                            f"{sm_count} SMs x {mhz:.0f} MHz (median SM clock in "
                            "the timed region)"),
-            "mufu_share": 0.75 if d == 64 else 1.0}
+            "mufu_share": 1.0 - fma_pipe_pairs_per8(d) / 8.0}
 
 
 def load_peaks():

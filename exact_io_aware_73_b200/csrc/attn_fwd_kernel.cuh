@@ -111,10 +111,12 @@ constexpr uint32_t kRoleDrain = 1u << 12;
 // Pairs of exponentials (out of every 8 pairs of a score row) evaluated on the
 // FMA pipe by exp2_poly_x2 instead of the MUFU unit; the rest use ex2.approx.
 // At d = 64 the MUFU carries twice the exponentials per tensor-core FLOP of
-// d = 128 and is the binding unit, so a quarter of them move to the FMA pipe;
-// at d = 128 measurement favoured the MUFU alone.
+// d = 128, so an eighth of them move to the FMA pipe (a quarter measured best
+// before P got TMEM columns of its own; with the next S off the softmax's
+// chain the FMA pipe's extra instructions cost more than they save); at
+// d = 128 measurement favoured the MUFU alone.
 #ifndef ATTN_EXP2_EMU_PER8
-#define ATTN_EXP2_EMU_PER8_D64 2
+#define ATTN_EXP2_EMU_PER8_D64 1
 #define ATTN_EXP2_EMU_PER8_D128 0
 #else
 #define ATTN_EXP2_EMU_PER8_D64 ATTN_EXP2_EMU_PER8
