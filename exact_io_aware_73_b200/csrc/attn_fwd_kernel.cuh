@@ -502,15 +502,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr,
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// d = 64 (bf16, dense): the two O accumulators take only 128 of the 512
-// TMEM columns, so each tile's P gets 64 columns of its own instead of
+// d = 64 (bf16): the two O accumulators take only 128 of the 512 TMEM
+// columns, so each tile's P gets 64 columns of its own instead of
 // overwriting S.  A tile's next S then needs only that its softmax has read
 // the last S out (S_FREE), not the P.V of it, so it is computed while the
-// softmax still works on the current one.  (Block-sparse units keep P over
-// S: with two different K lists, issuing a tile's next S ahead of its P.V
-// can leave each tile waiting on a slot the other still holds.)
+// softmax still works on the current one.  (In block-sparse units the two
+// tiles compute different K tiles, and a tile that waited for its next K
+// tile before its P.V could wait on a slot the other tile holds until it
+// gets that P.V's V slot: there the next S goes ahead only when its K tile
+// has already landed.)
 template <int D, bool FP8, bool SPARSE>
-constexpr bool kSplitP = (D == 64) && !FP8 && !SPARSE;
+constexpr bool kSplitP = (D == 64) && !FP8;
 
 // Which MMA role a variant runs.  Where P lies over S (d = 128, FP8) and
 // both tiles compute every K tile in step, one thread serves both tiles in
@@ -790,9 +792,9 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
 // neither tile's MMAs queue behind the other's barriers.  Per K tile j the
 // tile issues S_j = Q K_j^T and O += P_j V_j; P_j lies over S_j's columns,
 // so S_{j+1} follows P_j V_j in the same thread (the tensor pipe then reads
-// P_j before overwriting it), except in the split layout (dense units
-// only), where P has columns of its own and S_{j+1} goes out as soon as the
-// softmax has read S_j (S_FREE).  A K or V slot's EMPTY barrier counts one
+// P_j before overwriting it), except in the split layout (d = 64), where P
+// has columns of its own and S_{j+1} goes out as soon as the softmax has
+// read S_j (S_FREE) -- in block-sparse units only if K_{j+1} has landed.  A K or V slot's EMPTY barrier counts one
 // arrival per Q tile: a tcgen05.commit from each tile that computes with
 // it, and one from the loader for a tile that does not.
 template <int D, bool CAUSAL, bool FP8, bool SPARSE>
@@ -852,10 +854,23 @@ __device__ __forceinline__ void mma_role_tile(uint32_t base, uint32_t tmem,
     int at = step(), nat = 0;
     ok = issue_s(at, 0);
     for (int j = 0; j < n && ok; ++j) {
+      bool early = false;  // S_{j+1} issued ahead of P_j V_j
       if (kSplit && j + 1 < n) {
         nat = step();
-        ok = issue_s(nat, j + 1);
-        if (!ok) break;
+        early = true;
+        if constexpr (SPARSE) {
+          // only if K_{j+1} has landed: wait for the softmax to read S_j,
+          // then look (without waiting) at K_{j+1}'s slot
+          ok = mbar_wait_spin(bar(L::S_FREE + t), (sdone - 1) & 1, wc, kRoleMma);
+          if (!ok) break;
+          const int ka = ring + nat;
+          early = ld_acquire_shared(base + L::kSlotPos + 4 * (ka % L::kKStages)) == ka &&
+                  mbar_test_wait(bar(L::K_FULL + ka % L::kKStages), (ka / L::kKStages) & 1);
+        }
+        if (early) {
+          ok = issue_s(nat, j + 1);
+          if (!ok) break;
+        }
       }
       // O += P_j V_j: the first 64 keys once P_HALF, the rest once P_FULL
       // (FP8: all at once); the unit's first P.V also waits for the previous
@@ -886,8 +901,8 @@ __device__ __forceinline__ void mma_role_tile(uint32_t base, uint32_t tmem,
       ++pcnt;
       mma_commit(bar(L::O_FULL + t));
       mma_commit(bar(L::V_EMPTY + va % L::kVStages));
-      if (!kSplit && j + 1 < n) {
-        nat = step();
+      if (!early && j + 1 < n) {
+        if (!kSplit) nat = step();
         ok = issue_s(nat, j + 1);
         if (!ok) break;
       }
