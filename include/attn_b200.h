@@ -224,12 +224,12 @@ int attn_selftest_exp2(const float *x, float *y, int n, int mode,
  * for d = 128, about 32,700).
  *
  * Set-up: the first call on each device looks up the device address of the
- * scratch array (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture.  Sharing: every call on a device
- * uses the same array, which keeps the last call's contents (the status
- * word is cleared at the start of every call).  Calls that overlap on the
- * GPU -- from different host threads or on different streams -- race on the
- * array and corrupt each other's results; serialise them.
+ * scratch array (cudaGetSymbolAddress) with that device current.  Sharing:
+ * every call on a device uses the same array, which keeps the last call's
+ * contents (the status word is cleared at the start of every call).  Calls
+ * that overlap on the GPU -- from different host threads or on different
+ * streams -- race on the array and corrupt each other's results; serialise
+ * them.
  */
 int attn_fwd_host_noalloc(const void *q, const void *k, const void *v,
                           void *o, float *lse, int B, int H, int N, int d,

@@ -170,10 +170,14 @@ def test_large_scores_stress_rescale(oracle_mod):
         _compare(o, lse, o_ref, lse_ref, f"scale={scale}")
 
 
-def test_increasing_scores_force_every_rescale(oracle_mod):
+@pytest.mark.parametrize("H,d", [(1, 64), (80, 64), (40, 128)])
+def test_increasing_scores_force_every_rescale(oracle_mod, H, d):
     """Scores that grow along the key axis make the running max rise on every
-    key/value tile, exercising the output correction each iteration."""
-    B, H, N, d = 1, 1, 1024, 64
+    key/value tile, exercising the output correction each iteration; with
+    more heads than CTAs each CTA runs several units, so the correction also
+    meets the unit boundaries (the next unit's first S and P.V against the
+    previous unit's epilogue)."""
+    B, N = 1, 1024
     q = torch.zeros(B, H, N, d)
     q[..., 0] = 1.0
     k = torch.zeros(B, H, N, d)

@@ -137,6 +137,34 @@ def test_pairs_with_different_key_lists(oracle_mod, pattern, causal, N, d):
              f"{pattern} {w.name}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_sparse_forced_rescale_over_many_units(oracle_mod, d):
+    """Scores that grow along the key axis force the output correction on
+    every kept K tile; 40 heads of 4 pairs put several units on each CTA,
+    and the alternating-parity mask gives the two tiles of a pair disjoint
+    key lists."""
+    B, H, N = 1, 40, 1024
+    q = torch.zeros(B, H, N, d)
+    q[..., 0] = 1.0
+    k = torch.zeros(B, H, N, d)
+    k[..., 0] = torch.linspace(0, 400, N)
+    g = torch.Generator().manual_seed(17)
+    v = torch.randn(B, H, N, d, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    T = N // 128
+    m = _mask_patterns(T)["alternating"].copy()
+    m[:, 0] = 1  # every row keeps K tile 0 too
+    for causal in (False, True):
+        o, lse = attn.attn_fwd_block_sparse(q.cuda(), k.cuda(), v.cuda(),
+                                            torch.from_numpy(m).cuda(), causal=causal,
+                                            scale=1.0)
+        assert attn.status() == 0
+        bits = [oracle_mod.bf16_bits(t) for t in (q, k, v)]
+        o_ref, l_ref = oracle_mod.attention_block_sparse_bf16(*bits, causal, 1.0, m)
+        _compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref,
+                 f"forced rescale d={d} causal={causal}")
+
+
 @pytest.mark.parametrize("name", sorted(W.SPARSE_WORKLOADS))
 def test_block_sparse_workloads_sampled_rows(oracle_mod, name):
     """The benchmark's block-sparse workloads, in the launch the benchmark
