@@ -57,8 +57,10 @@ struct BwdParams {
   const float *lse;      // [BH, N] forward log-sum-exp, natural log (prep only)
   // Workspace, rows padded to npad = 128 * tiles so every 128-row TMA tile of
   // these fp32 vectors starts on a 512-byte boundary; padding rows hold 0.
-  float *lse2;           // [BH, npad] lse * log2(e)
-  float *dsum;           // [BH, npad] D_i = sum_t dO_it O_it
+  // Both are stored negated: the compute warps add them (packed f32x2
+  // arithmetic has no negated operand).
+  float *lse2;           // [BH, npad] -lse * log2(e)
+  float *dsum;           // [BH, npad] -D_i, D_i = sum_t dO_it O_it
   uint16_t *dq, *dk, *dv;  // [BH, N, D] outputs
   uint32_t *status;
   int bh, n, npad, tiles, num_units;
@@ -69,8 +71,8 @@ struct BwdParams {
 
 // ------------------------------------------------------------------ prep
 
-// D_i = sum_t dO_it * O_it and lse_i * log2(e) for every row, fp32, into the
-// padded workspace vectors (0 in padding rows); one warp per row.
+// -D_i (D_i = sum_t dO_it * O_it) and -lse_i * log2(e) for every row, fp32,
+// into the padded workspace vectors (0 in padding rows); one warp per row.
 template <int D>
 __global__ void __launch_bounds__(256)
     attn_bwd_prep_kernel(const BwdParams p) {
@@ -96,8 +98,8 @@ __global__ void __launch_bounds__(256)
       l2 = p.lse[row] * 1.4426950408889634f;
     }
     if (lane == 0) {
-      p.dsum[prow] = acc;
-      p.lse2[prow] = l2;
+      p.dsum[prow] = -acc;
+      p.lse2[prow] = -l2;
     }
   }
 }
@@ -307,8 +309,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool row_ok = row < p.n;
       const int64_t grow = static_cast<int64_t>(bh) * p.n + row;
       const int64_t prow = static_cast<int64_t>(bh) * p.npad + row;
-      const float nlse = -p.lse2[prow];
-      const float drow = p.dsum[prow];
+      const uint64_t nlse2 = f32x2(p.lse2[prow], p.lse2[prow]);  // -lse log2(e)
+      const uint64_t ndrow2 = f32x2(p.dsum[prow], p.dsum[prow]);  // -D
+      const uint64_t c2 = f32x2(p.c_log2, p.c_log2);
       for (int j = 0; j < nkv; ++j) {
         // ---- P phase: P_j from S_j, kept in registers; S released
         ok = mbar_wait(bar(L::S_FULL), s_cnt & 1, wc, kRoleSoftmax);
@@ -325,9 +328,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld_32x32b_x32(tS + lb + c * 32, sv);
           tmem_wait_ld(sv);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float e = ex2_approx(fmaf(__uint_as_float(sv[i]), p.c_log2, nlse));
-            pr[cc * 32 + i] = (mask && c * 32 + i > limit) ? 0.f : e;
+          for (int i = 0; i < 32; i += 2) {
+            const uint64_t x2 = fma_f32x2(
+                f32x2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, nlse2);
+            float x0, x1;
+            f32x2_split(x2, x0, x1);
+            pr[cc * 32 + i] = ex2_approx(x0);
+            pr[cc * 32 + i + 1] = ex2_approx(x1);
+          }
+          if (mask) {  // the last K tile only
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i > limit) pr[cc * 32 + i] = 0.f;
           }
         }
         tc_fence_before_sync();
@@ -350,10 +362,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int c = 2 * hc + cc;
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(pr[cc * 32 + 2 * i] * (__uint_as_float(dv[cc][2 * i]) - drow),
-                                pr[cc * 32 + 2 * i + 1] *
-                                    (__uint_as_float(dv[cc][2 * i + 1]) - drow));
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t t2 = add_f32x2(
+                f32x2(__uint_as_float(dv[cc][2 * i]), __uint_as_float(dv[cc][2 * i + 1])),
+                ndrow2);
+            float d0, d1;
+            f32x2_split(mul_f32x2(f32x2(pr[cc * 32 + 2 * i], pr[cc * 32 + 2 * i + 1]), t2),
+                        d0, d1);
+            pk[i] = pack_bf16x2(d0, d1);
+          }
           tmem_st_32x32b_x16(tdP + lb + c * 16, pk);  // bf16 dS over dP columns
         }
         tmem_wait_st();
@@ -641,25 +658,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_ld(sv[0]);
         reg_fence(sv[1]);
         bwd_pair_sync(wq);  // both halves hold their S^T before P^T overwrites it
+        const uint64_t c2 = f32x2(p.c_log2, p.c_log2);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * hc + cc;  // 32-column chunk of the tile
-          uint32_t ppk[16];
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
+            // -lse log2(e) of four query columns
             const float4 lv = ld_shared_f4(vec + (c * 32 + 4 * g) * 4);
-            const float lse4[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int qc = c * 32 + 4 * g + e;  // query column in the tile
-              float pe = ex2_approx(fmaf(__uint_as_float(sv[cc][4 * g + e]), p.c_log2,
-                                         -lse4[e]));
-              if ((diag && qc < r) || (tail && qc > qlimit)) pe = 0.f;
-              pr[cc * 32 + 4 * g + e] = pe;
-            }
-            ppk[2 * g] = pack_bf16x2(pr[cc * 32 + 4 * g], pr[cc * 32 + 4 * g + 1]);
-            ppk[2 * g + 1] = pack_bf16x2(pr[cc * 32 + 4 * g + 2], pr[cc * 32 + 4 * g + 3]);
+            const uint64_t xa = fma_f32x2(f32x2(__uint_as_float(sv[cc][4 * g]),
+                                                __uint_as_float(sv[cc][4 * g + 1])),
+                                          c2, f32x2(lv.x, lv.y));
+            const uint64_t xb = fma_f32x2(f32x2(__uint_as_float(sv[cc][4 * g + 2]),
+                                                __uint_as_float(sv[cc][4 * g + 3])),
+                                          c2, f32x2(lv.z, lv.w));
+            float x0, x1, x2, x3;
+            f32x2_split(xa, x0, x1);
+            f32x2_split(xb, x2, x3);
+            pr[cc * 32 + 4 * g] = ex2_approx(x0);
+            pr[cc * 32 + 4 * g + 1] = ex2_approx(x1);
+            pr[cc * 32 + 4 * g + 2] = ex2_approx(x2);
+            pr[cc * 32 + 4 * g + 3] = ex2_approx(x3);
           }
+          if (diag || tail) {  // the diagonal and the ragged last Q tile only
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int qc = c * 32 + e;  // query column in the tile
+              if ((diag && qc < r) || (tail && qc > qlimit)) pr[cc * 32 + e] = 0.f;
+            }
+          }
+          uint32_t ppk[16];
+#pragma unroll
+          for (int g = 0; g < 16; ++g)
+            ppk[g] = pack_bf16x2(pr[cc * 32 + 2 * g], pr[cc * 32 + 2 * g + 1]);
           tmem_st_32x32b_x16(tS + lb + c * 16, ppk);   // P^T over S^T
         }
         tmem_wait_st();
@@ -684,13 +715,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t dpk[16];
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
-            const float4 dd = ld_shared_f4(vec + 512 + (c * 32 + 4 * g) * 4);
+            const float4 dd = ld_shared_f4(vec + 512 + (c * 32 + 4 * g) * 4);  // -D
             const int q4 = cc * 32 + 4 * g;  // index into pr
-            dpk[2 * g] = pack_bf16x2(pr[q4] * (__uint_as_float(dv[cc][4 * g]) - dd.x),
-                                     pr[q4 + 1] * (__uint_as_float(dv[cc][4 * g + 1]) - dd.y));
-            dpk[2 * g + 1] =
-                pack_bf16x2(pr[q4 + 2] * (__uint_as_float(dv[cc][4 * g + 2]) - dd.z),
-                            pr[q4 + 3] * (__uint_as_float(dv[cc][4 * g + 3]) - dd.w));
+            const uint64_t ta = add_f32x2(f32x2(__uint_as_float(dv[cc][4 * g]),
+                                                __uint_as_float(dv[cc][4 * g + 1])),
+                                          f32x2(dd.x, dd.y));
+            const uint64_t tb = add_f32x2(f32x2(__uint_as_float(dv[cc][4 * g + 2]),
+                                                __uint_as_float(dv[cc][4 * g + 3])),
+                                          f32x2(dd.z, dd.w));
+            float d0, d1, d2, d3;
+            f32x2_split(mul_f32x2(f32x2(pr[q4], pr[q4 + 1]), ta), d0, d1);
+            f32x2_split(mul_f32x2(f32x2(pr[q4 + 2], pr[q4 + 3]), tb), d2, d3);
+            dpk[2 * g] = pack_bf16x2(d0, d1);
+            dpk[2 * g + 1] = pack_bf16x2(d2, d3);
           }
           tmem_st_32x32b_x16(tdP + lb + c * 16, dpk);  // dS^T over dP^T
         }
