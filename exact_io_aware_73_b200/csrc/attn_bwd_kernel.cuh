@@ -51,6 +51,31 @@ __device__ __forceinline__ void bwd_pair_sync(int wq) {
   tc_fence_after_sync();
 }
 
+// Pairs of exponentials (out of every 8) that the compute warps evaluate on
+// the FMA pipe (exp2_poly_x2) instead of the MUFU unit: at d = 64 the
+// exponentials weigh twice as much per tensor-core FLOP as at d = 128, and
+// two pairs in eight measured best (the polynomial's relative error, below
+// 8e-5, is far inside the bf16 rounding of P).
+#ifndef ATTN_BWD_EXP2_EMU_PER8_D64
+#define ATTN_BWD_EXP2_EMU_PER8_D64 2
+#endif
+template <int D>
+constexpr int kBwdEmuPer8 = (D == 64) ? ATTN_BWD_EXP2_EMU_PER8_D64 : 0;
+
+// Two exponentials of a pair: the FMA-pipe polynomial for the first
+// kBwdEmuPer8<D> pairs of every 8, ex2.approx otherwise.
+template <int D>
+__device__ __forceinline__ void bwd_exp2_pair(int pair, uint64_t x2, float &p0, float &p1) {
+  float x0, x1;
+  f32x2_split(x2, x0, x1);
+  if ((pair & 7) < kBwdEmuPer8<D>) {
+    f32x2_split(exp2_poly_x2(x0, x1), p0, p1);
+  } else {
+    p0 = ex2_approx(x0);
+    p1 = ex2_approx(x1);
+  }
+}
+
 struct BwdParams {
   const uint16_t *o;     // [BH, N, D] forward output (prep only)
   const uint16_t *dout;  // [BH, N, D] upstream gradient (prep only)
@@ -331,10 +356,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int i = 0; i < 32; i += 2) {
             const uint64_t x2 = fma_f32x2(
                 f32x2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, nlse2);
-            float x0, x1;
-            f32x2_split(x2, x0, x1);
-            pr[cc * 32 + i] = ex2_approx(x0);
-            pr[cc * 32 + i + 1] = ex2_approx(x1);
+            bwd_exp2_pair<D>(i >> 1, x2, pr[cc * 32 + i], pr[cc * 32 + i + 1]);
           }
           if (mask) {  // the last K tile only
 #pragma unroll
@@ -672,13 +694,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t xb = fma_f32x2(f32x2(__uint_as_float(sv[cc][4 * g + 2]),
                                                 __uint_as_float(sv[cc][4 * g + 3])),
                                           c2, f32x2(lv.z, lv.w));
-            float x0, x1, x2, x3;
-            f32x2_split(xa, x0, x1);
-            f32x2_split(xb, x2, x3);
-            pr[cc * 32 + 4 * g] = ex2_approx(x0);
-            pr[cc * 32 + 4 * g + 1] = ex2_approx(x1);
-            pr[cc * 32 + 4 * g + 2] = ex2_approx(x2);
-            pr[cc * 32 + 4 * g + 3] = ex2_approx(x3);
+            bwd_exp2_pair<D>(2 * g, xa, pr[cc * 32 + 4 * g], pr[cc * 32 + 4 * g + 1]);
+            bwd_exp2_pair<D>(2 * g + 1, xb, pr[cc * 32 + 4 * g + 2], pr[cc * 32 + 4 * g + 3]);
           }
           if (diag || tail) {  // the diagonal and the ragged last Q tile only
 #pragma unroll
