@@ -199,7 +199,11 @@ def test_decode_needles_at_maximum_key_count(causal, kernel):
 @pytest.mark.parametrize("causal", [False, True])
 def test_backward_needles_long(causal):
     """N = 2^20 + 77, d = 64: dV_t = sum of dO over the rows whose weight
-    sits on key t (fp64 sums on the host); every other row of dV is 0."""
+    sits on key t (fp64 sums on the host); every other row of dV is 0 up to
+    the floor of the FMA-pipe exponential: it clamps its argument at -125,
+    so a score far below its row's maximum still weighs 2^-125 instead of
+    underflowing to 0, and such a row of dV sums at most N of those times
+    |dO| (below 2^-100 here)."""
     BH, N, d = 1, (1 << 20) + 77, 64
     t2v = 128 * 4096
     t2 = torch.tensor([t2v], device="cuda")
@@ -222,7 +226,7 @@ def test_backward_needles_long(causal):
         assert np.all(np.abs(dvh[t] - w) <= bound), (t, np.abs(dvh[t] - w).max())
     others = np.ones(N, dtype=bool)
     others[[0, t2v]] = False
-    assert np.all(dvh[others] == 0.0)
+    assert np.all(np.abs(dvh[others]) <= 2.0 ** -100)
     assert np.all(np.isfinite(dq.float().cpu().numpy()))
     assert np.all(np.isfinite(dk.float().cpu().numpy()))
 
