@@ -794,9 +794,10 @@ __device__ __forceinline__ void mma_role(uint32_t base, uint32_t tmem,
 // so S_{j+1} follows P_j V_j in the same thread (the tensor pipe then reads
 // P_j before overwriting it), except in the split layout (d = 64), where P
 // has columns of its own and S_{j+1} goes out as soon as the softmax has
-// read S_j (S_FREE) -- in block-sparse units only if K_{j+1} has landed.  A K or V slot's EMPTY barrier counts one
-// arrival per Q tile: a tcgen05.commit from each tile that computes with
-// it, and one from the loader for a tile that does not.
+// read S_j (S_FREE) -- in block-sparse units only if K_{j+1} has landed.
+// A K or V slot's EMPTY barrier counts one arrival per Q tile: a
+// tcgen05.commit from each tile that computes with it, and one from the
+// loader for a tile that does not.
 template <int D, bool CAUSAL, bool FP8, bool SPARSE>
 __device__ __forceinline__ void mma_role_tile(uint32_t base, uint32_t tmem,
                                               const FwdParams &p, const WaitCtx &wc,
