@@ -181,3 +181,28 @@ def test_block_sparse_workloads_sampled_rows(oracle_mod, name):
         *bits, w.causal, w.scale, m.numpy(), rows)
     _compare(o.float().cpu().numpy().reshape(-1, w.d)[rows],
              lse.cpu().numpy().reshape(-1)[rows], o_ref, l_ref, name)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_masks_and_shapes(oracle_mod, seed):
+    """Random shapes (ragged N, d = 64 or 128, causal or not) with random
+    per-head masks of random density: pairs of query tiles whose key lists
+    overlap anywhere from fully to not at all, empty rows included."""
+    rng = np.random.default_rng(900 + seed)
+    d = 64 if seed % 2 else 128
+    B, H = 1, int(rng.integers(1, 4))
+    N = int(rng.integers(129, 1800))
+    causal = bool(rng.integers(0, 2))
+    w = W.shape_case(B, H, N, d, causal, seed=950 + seed)
+    q, k, v = W.make_qkv(w)
+    T = (N + 127) // 128
+    density = float(rng.uniform(0.05, 0.95))
+    m = (rng.random((B * H, T, T)) < density).astype(np.uint8)
+    o, lse = attn.attn_fwd_block_sparse(q.cuda(), k.cuda(), v.cuda(),
+                                        torch.from_numpy(m).cuda(), causal=causal,
+                                        scale=w.scale)
+    assert attn.status() == 0
+    bits = [oracle_mod.bf16_bits(t) for t in (q, k, v)]
+    o_ref, l_ref = oracle_mod.attention_block_sparse_bf16(*bits, causal, w.scale, m)
+    _compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref,
+             f"seed {seed}: {w.name} density {density:.2f}")
